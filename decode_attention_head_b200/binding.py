@@ -1,0 +1,174 @@
+"""ctypes binding of libwushkv (include/wushkv.h): argument marshalling only.
+
+Every step of the append and decode-attention path runs in the library's CUDA
+kernels; PyTorch only provides device memory and streams.  If the library is
+missing the import of this module fails: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwushkv.so")
+
+OK, EINVAL, EUNSUPPORTED, ECUDA, ESINGULAR = 0, -1, -2, -3, -4
+STATUS_OVERFLOW, STATUS_EMPTY, STATUS_TIMEOUT, STATUS_BADSTATE = 1, 2, 4, 8
+_ERR = {EINVAL: "invalid argument", EUNSUPPORTED: "unsupported configuration", ECUDA: "CUDA launch failed",
+        ESINGULAR: "singular key transform"}
+SYMBOLS = ("wushkv_pack_layout", "wushkv_compensation", "wushkv_append", "wushkv_decode_attn")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("bits", ctypes.c_int32), ("capacity", ctypes.c_int32),
+                ("s_sink", ctypes.c_int32), ("s_keep", ctypes.c_int32), ("s_flush", ctypes.c_int32),
+                ("chunk_max", ctypes.c_int32), ("p_lo", ctypes.c_float), ("p_hi", ctypes.c_float)]
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [("codes_bytes", ctypes.c_size_t), ("params_bytes", ctypes.c_size_t),
+                ("sink_bytes", ctypes.c_size_t), ("ring_bytes", ctypes.c_size_t),
+                ("state_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t),
+                ("cap_alloc", ctypes.c_int32), ("ring_slots", ctypes.c_int32), ("code_bytes", ctypes.c_int32),
+                ("n_splits", ctypes.c_int32), ("split_tokens", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class CacheBufs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("k_codes", "v_codes", "k_params", "v_params", "k_sink", "v_sink",
+                                               "k_ring", "v_ring", "state")]
+
+
+class WushKVError(RuntimeError):
+    pass
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libwushkv.so not built ({LIB_PATH}); run decode_attention_head_b200.build.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.wushkv_pack_layout.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Layout)]
+    lib.wushkv_compensation.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]
+    lib.wushkv_append.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
+    lib.wushkv_decode_attn.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_void_p]
+    for name in SYMBOLS:
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != OK:
+        raise WushKVError(f"{what}: {_ERR.get(rc, rc)}")
+
+
+def make_config(batch, n_kv_heads, n_q_heads, bits, capacity, s_sink, s_keep, s_flush=16, chunk_max=1,
+                p_lo=1.0, p_hi=99.0, head_dim=128) -> Config:
+    return Config(batch, n_kv_heads, n_q_heads, head_dim, bits, capacity, s_sink, s_keep, s_flush, chunk_max,
+                  p_lo, p_hi)
+
+
+def pack_layout(cfg: Config) -> Layout:
+    out = Layout()
+    _check(lib.wushkv_pack_layout(ctypes.byref(cfg), ctypes.byref(out)), "wushkv_pack_layout")
+    return out
+
+
+def compensation(t_k: torch.Tensor) -> torch.Tensor:
+    """T_K^{-1} (fp32, host) of host fp16 T_K [H_kv, 128, 128] via the library's Gauss-Jordan."""
+    t = t_k.detach().to("cpu", torch.float16).contiguous()
+    out = torch.empty(t.shape, dtype=torch.float32)
+    _check(lib.wushkv_compensation(t.data_ptr(), t.shape[0], out.data_ptr()), "wushkv_compensation")
+    return out
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+class KVCache:
+    """One layer's cache buffers, allocated with torch on `device` per the library's layout."""
+
+    def __init__(self, cfg: Config, device="cuda"):
+        self.cfg = cfg
+        self.layout = pack_layout(cfg)
+        L = self.layout
+        u8 = dict(dtype=torch.uint8, device=device)
+        self.k_codes = torch.zeros(L.codes_bytes, **u8)
+        self.v_codes = torch.zeros(L.codes_bytes, **u8)
+        self.k_params = torch.zeros(L.params_bytes // 4, dtype=torch.int32, device=device)
+        self.v_params = torch.zeros(L.params_bytes // 4, dtype=torch.int32, device=device)
+        self.k_sink = torch.zeros(L.sink_bytes // 2, dtype=torch.float16, device=device)
+        self.v_sink = torch.zeros(L.sink_bytes // 2, dtype=torch.float16, device=device)
+        self.k_ring = torch.zeros(L.ring_bytes // 2, dtype=torch.float16, device=device)
+        self.v_ring = torch.zeros(L.ring_bytes // 2, dtype=torch.float16, device=device)
+        self.state = torch.zeros(L.state_bytes // 4, dtype=torch.int32, device=device)
+        self.workspace = torch.empty(L.workspace_bytes, **u8)
+        self.bufs = CacheBufs(*(t.data_ptr() for t in (self.k_codes, self.v_codes, self.k_params, self.v_params,
+                                                        self.k_sink, self.v_sink, self.k_ring, self.v_ring,
+                                                        self.state)))
+
+    @property
+    def units(self) -> int:
+        return self.cfg.batch * self.cfg.n_kv_heads
+
+    def lengths(self):
+        """(S, S_quant) per (sequence, KV head): int32 [B, H_kv] each (device tensors)."""
+        st = self.state[: 2 * self.units].view(self.cfg.batch, self.cfg.n_kv_heads, 2)
+        return st[..., 0], st[..., 1]
+
+    def status(self) -> int:
+        return int(self.state[2 * self.units].item())
+
+    def reset(self) -> None:
+        self.state.zero_()
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, t_k: torch.Tensor, stream=None) -> None:
+        """k_new, v_new: fp16 [B, n_new, H_kv, 128] on the device; t_k fp16 [H_kv, 128, 128]."""
+        n_new = k_new.shape[1]
+        _check(lib.wushkv_append(ctypes.byref(self.cfg), ctypes.byref(self.bufs), k_new.data_ptr(),
+                                 v_new.data_ptr(), n_new, t_k.data_ptr(), _stream_ptr(stream)), "wushkv_append")
+
+    def decode_attn(self, q: torch.Tensor, t_k_inv: torch.Tensor, softmax_scale: float,
+                    out: Optional[torch.Tensor] = None, out_fp16: bool = False, stream=None) -> torch.Tensor:
+        """q fp16 [B, H_q, 128]; t_k_inv fp32 [H_kv, 128, 128] (T_K^{-1}); returns out [B, H_q, 128]."""
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float16 if out_fp16 else torch.float32, device=q.device)
+        _check(lib.wushkv_decode_attn(ctypes.byref(self.cfg), ctypes.byref(self.bufs), q.data_ptr(),
+                                      t_k_inv.data_ptr(), float(softmax_scale), 1 if out.dtype == torch.float16 else 0,
+                                      out.data_ptr(), self.workspace.data_ptr(), _stream_ptr(stream)),
+               "wushkv_decode_attn")
+        return out
+
+    # -- typed views of the buffers (for tests and tools) ------------------------
+    def codes_view(self, kind: str) -> torch.Tensor:
+        """uint8 [B, H_kv, cap_alloc, code_bytes]."""
+        t = self.k_codes if kind == "k" else self.v_codes
+        return t.view(self.cfg.batch, self.cfg.n_kv_heads, self.layout.cap_alloc, self.layout.code_bytes)
+
+    def params_view(self, kind: str) -> torch.Tensor:
+        """fp16 [B, H_kv, cap_alloc, 2] = (s, z)."""
+        t = self.k_params if kind == "k" else self.v_params
+        return t.view(torch.float16).view(self.cfg.batch, self.cfg.n_kv_heads, self.layout.cap_alloc, 2)
+
+    def sink_view(self, kind: str) -> torch.Tensor:
+        t = self.k_sink if kind == "k" else self.v_sink
+        return t.view(self.cfg.batch, self.cfg.n_kv_heads, -1, 128)
+
+    def ring_view(self, kind: str) -> torch.Tensor:
+        t = self.k_ring if kind == "k" else self.v_ring
+        return t.view(self.cfg.batch, self.cfg.n_kv_heads, self.layout.ring_slots, 128)
+
+
+def config_for_workload(wl, extra_capacity: int = 1024, chunk_max: int = 1) -> Config:
+    """Library config of a synthetic workload (synth.Workload); capacity = context + extra."""
+    return make_config(wl.batch, wl.n_kv_heads, wl.n_q_heads, wl.bits, wl.context + extra_capacity,
+                       wl.s_sink, wl.s_keep, wl.s_flush, chunk_max, wl.p_lo, wl.p_hi, wl.head_dim)

@@ -1,0 +1,234 @@
+// C-ABI entry points of libwushkv (declared in include/wushkv.h): configuration
+// validation, buffer layout, the host-side compensation-matrix helper, and launch.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include "internal.h"
+
+namespace wushkv {
+
+static inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+static inline size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+int derive(const wushkv_config* cfg, Derived* d) {
+  if (!cfg || !d) return WUSHKV_EINVAL;
+  if (cfg->head_dim != kHeadDim) return WUSHKV_EUNSUPPORTED;
+  if (cfg->bits != 2 && cfg->bits != 4) return WUSHKV_EUNSUPPORTED;
+  if (cfg->batch < 1 || cfg->n_kv_heads < 1 || cfg->n_q_heads < 1 || cfg->capacity < 1) return WUSHKV_EINVAL;
+  if (cfg->n_q_heads % cfg->n_kv_heads) return WUSHKV_EINVAL;
+  const int g = cfg->n_q_heads / cfg->n_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return WUSHKV_EUNSUPPORTED;
+  if (cfg->s_sink < 0 || cfg->s_keep < 0 || cfg->s_flush < 1 || cfg->chunk_max < 1) return WUSHKV_EINVAL;
+  if (!(cfg->p_lo >= 0.f) || !(cfg->p_hi <= 100.f) || !(cfg->p_lo < cfg->p_hi)) return WUSHKV_EINVAL;
+  const long long units = (long long)cfg->batch * cfg->n_kv_heads;
+  if (units > (1 << 24) || cfg->capacity > (1 << 28)) return WUSHKV_EINVAL;
+
+  d->units = (int)units;
+  d->group = g;
+  d->cap_alloc = (int)round_up((size_t)cfg->capacity, kTileTokens);
+  d->ring = cfg->s_keep + cfg->s_flush - 1 + cfg->chunk_max;
+  d->sink_dim = cfg->s_sink > 0 ? cfg->s_sink : 1;
+  d->code_bytes = 16 * cfg->bits;
+  // percentile ranks: pos = p/100 * 127 in double, i = floor(pos), f = fp32(pos - i)
+  const double pos_lo = (double)cfg->p_lo / 100.0 * (double)(kHeadDim - 1);
+  const double pos_hi = (double)cfg->p_hi / 100.0 * (double)(kHeadDim - 1);
+  d->i_lo = (int)std::floor(pos_lo);
+  d->i_hi = (int)std::floor(pos_hi);
+  d->f_lo = (float)(pos_lo - d->i_lo);
+  d->f_hi = (float)(pos_hi - d->i_hi);
+  const int need_lo = d->i_lo + 2;               // s[i_lo], s[i_lo+1]
+  const int need_hi = kHeadDim - d->i_hi;        // s[i_hi] from the top
+  d->nsel = need_lo > need_hi ? need_lo : need_hi;
+  if (d->nsel < 2) d->nsel = 2;
+  if (d->nsel > 4) return WUSHKV_EUNSUPPORTED;
+
+  // decode work split: ~kDecodeCtasPerSM quantized items per SM over all units
+  int per_unit = ceil_div(kB200SMs * kDecodeCtasPerSM, d->units);
+  if (per_unit < 1) per_unit = 1;
+  if (per_unit > kMaxSplits) per_unit = kMaxSplits;
+  int L = ceil_div(ceil_div(d->cap_alloc, per_unit), kTileTokens) * kTileTokens;
+  if (L < kTileTokens) L = kTileTokens;
+  d->split_tokens = L;
+  d->n_split = ceil_div(d->cap_alloc, L);
+
+  const size_t U = (size_t)d->units;
+  d->codes_bytes = U * d->cap_alloc * d->code_bytes;
+  d->params_bytes = U * d->cap_alloc * 4;
+  d->sink_bytes = U * d->sink_dim * kHeadDim * 2;
+  d->ring_bytes = U * (size_t)d->ring * kHeadDim * 2;
+  d->state_bytes = round_up((2 * U + 1) * 4, 16);
+  size_t off = 0;
+  d->ws_tickets = off;
+  off = round_up(off + U * 4, 256);
+  d->ws_qfrag = off;
+  off = round_up(off + U * 4 * 4 * 64 * 4, 256);
+  d->ws_hconst = off;
+  off = round_up(off + U * 8 * 2 * 4, 256);
+  d->ws_qprime = off;
+  off = round_up(off + U * g * kHeadDim * 4, 256);
+  d->ws_partials = off;
+  off = round_up(off + U * (size_t)(d->n_split + 1) * g * 132 * 4, 256);
+  d->ws_total = off;
+  return WUSHKV_OK;
+}
+
+static bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+static bool cache_ok(const wushkv_cache* c) {
+  return c && aligned16(c->k_codes) && aligned16(c->v_codes) && aligned16(c->k_params) &&
+         aligned16(c->v_params) && aligned16(c->k_sink) && aligned16(c->v_sink) && aligned16(c->k_ring) &&
+         aligned16(c->v_ring) && aligned16(c->state);
+}
+
+}  // namespace wushkv
+
+using namespace wushkv;
+
+extern "C" int wushkv_pack_layout(const wushkv_config* cfg, wushkv_layout* out) {
+  if (!out) return WUSHKV_EINVAL;
+  Derived d;
+  const int rc = derive(cfg, &d);
+  if (rc != WUSHKV_OK) return rc;
+  std::memset(out, 0, sizeof(*out));
+  out->codes_bytes = d.codes_bytes;
+  out->params_bytes = d.params_bytes;
+  out->sink_bytes = d.sink_bytes;
+  out->ring_bytes = d.ring_bytes;
+  out->state_bytes = d.state_bytes;
+  out->workspace_bytes = d.ws_total;
+  out->cap_alloc = d.cap_alloc;
+  out->ring_slots = d.ring;
+  out->code_bytes = d.code_bytes;
+  out->n_splits = d.n_split;
+  out->split_tokens = d.split_tokens;
+  return WUSHKV_OK;
+}
+
+extern "C" int wushkv_compensation(const uint16_t* t_k, int32_t n_kv_heads, float* t_k_inv) {
+  if (!t_k || !t_k_inv || n_kv_heads < 1) return WUSHKV_EINVAL;
+  const int n = kHeadDim;
+  std::vector<double> a((size_t)n * 2 * n);
+  for (int h = 0; h < n_kv_heads; ++h) {
+    // [T | I], Gauss-Jordan with partial pivoting -> [I | T^{-1}]
+    for (int r = 0; r < n; ++r) {
+      for (int c = 0; c < n; ++c) {
+        __half_raw raw;
+        raw.x = t_k[((size_t)h * n + r) * n + c];
+        a[(size_t)r * 2 * n + c] = (double)__half2float(__half(raw));
+        a[(size_t)r * 2 * n + n + c] = (r == c) ? 1.0 : 0.0;
+      }
+    }
+    for (int col = 0; col < n; ++col) {
+      int piv = col;
+      double best = std::fabs(a[(size_t)col * 2 * n + col]);
+      for (int r = col + 1; r < n; ++r) {
+        const double v = std::fabs(a[(size_t)r * 2 * n + col]);
+        if (v > best) {
+          best = v;
+          piv = r;
+        }
+      }
+      if (!(best > 0.0)) return WUSHKV_ESINGULAR;
+      if (piv != col)
+        for (int c = 0; c < 2 * n; ++c) std::swap(a[(size_t)piv * 2 * n + c], a[(size_t)col * 2 * n + c]);
+      const double inv = 1.0 / a[(size_t)col * 2 * n + col];
+      for (int c = 0; c < 2 * n; ++c) a[(size_t)col * 2 * n + c] *= inv;
+      for (int r = 0; r < n; ++r) {
+        if (r == col) continue;
+        const double f = a[(size_t)r * 2 * n + col];
+        if (f == 0.0) continue;
+        for (int c = 0; c < 2 * n; ++c) a[(size_t)r * 2 * n + c] -= f * a[(size_t)col * 2 * n + c];
+      }
+    }
+    for (int r = 0; r < n; ++r)
+      for (int c = 0; c < n; ++c) t_k_inv[((size_t)h * n + r) * n + c] = (float)a[(size_t)r * 2 * n + n + c];
+  }
+  return WUSHKV_OK;
+}
+
+extern "C" int wushkv_append(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new,
+                             const void* v_new, int32_t n_new, const void* t_k, void* stream) {
+  Derived d;
+  const int rc = derive(cfg, &d);
+  if (rc != WUSHKV_OK) return rc;
+  if (!cache_ok(cache) || n_new < 0 || !aligned16(t_k)) return WUSHKV_EINVAL;
+  if (n_new > 0 && (!aligned16(k_new) || !aligned16(v_new))) return WUSHKV_EINVAL;
+  AppendArgs a;
+  a.B = cfg->batch;
+  a.Hkv = cfg->n_kv_heads;
+  a.cap = cfg->capacity;
+  a.cap_alloc = d.cap_alloc;
+  a.s_sink = cfg->s_sink;
+  a.s_keep = cfg->s_keep;
+  a.s_flush = cfg->s_flush;
+  a.R = d.ring;
+  a.sink_dim = d.sink_dim;
+  a.n_new = n_new;
+  a.k_codes = static_cast<uint8_t*>(cache->k_codes);
+  a.v_codes = static_cast<uint8_t*>(cache->v_codes);
+  a.k_params = static_cast<uint32_t*>(cache->k_params);
+  a.v_params = static_cast<uint32_t*>(cache->v_params);
+  a.k_sink = static_cast<__half*>(cache->k_sink);
+  a.v_sink = static_cast<__half*>(cache->v_sink);
+  a.k_ring = static_cast<__half*>(cache->k_ring);
+  a.v_ring = static_cast<__half*>(cache->v_ring);
+  a.state = cache->state;
+  a.status = reinterpret_cast<uint32_t*>(cache->state + 2 * (size_t)d.units);
+  a.k_new = static_cast<const __half*>(k_new);
+  a.v_new = static_cast<const __half*>(v_new);
+  a.t_k = static_cast<const __half*>(t_k);
+  a.i_lo = d.i_lo;
+  a.i_hi = d.i_hi;
+  a.f_lo = d.f_lo;
+  a.f_hi = d.f_hi;
+  const bool small = n_new <= cfg->chunk_max;
+  const cudaError_t e = launch_append(d, cfg->bits, small, a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA;
+}
+
+extern "C" int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* cache, const void* q,
+                                  const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
+                                  void* workspace, void* stream) {
+  Derived d;
+  const int rc = derive(cfg, &d);
+  if (rc != WUSHKV_OK) return rc;
+  if (!cache_ok(cache) || !aligned16(q) || !aligned16(t_k_inv) || !aligned16(out) || !aligned16(workspace))
+    return WUSHKV_EINVAL;
+  if (!std::isfinite(softmax_scale) || (out_fp16 != 0 && out_fp16 != 1)) return WUSHKV_EINVAL;
+  DecodeArgs a;
+  a.B = cfg->batch;
+  a.Hkv = cfg->n_kv_heads;
+  a.Hq = cfg->n_q_heads;
+  a.cap_alloc = d.cap_alloc;
+  a.s_sink = cfg->s_sink;
+  a.R = d.ring;
+  a.sink_dim = d.sink_dim;
+  a.n_split = d.n_split;
+  a.split_tokens = d.split_tokens;
+  a.k_codes = static_cast<const uint8_t*>(cache->k_codes);
+  a.v_codes = static_cast<const uint8_t*>(cache->v_codes);
+  a.k_params = static_cast<const uint32_t*>(cache->k_params);
+  a.v_params = static_cast<const uint32_t*>(cache->v_params);
+  a.k_sink = static_cast<const __half*>(cache->k_sink);
+  a.v_sink = static_cast<const __half*>(cache->v_sink);
+  a.k_ring = static_cast<const __half*>(cache->k_ring);
+  a.v_ring = static_cast<const __half*>(cache->v_ring);
+  a.state = cache->state;
+  a.status = reinterpret_cast<uint32_t*>(cache->state + 2 * (size_t)d.units);
+  a.q = static_cast<const __half*>(q);
+  a.t_k_inv = t_k_inv;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.out = out;
+  a.out_fp16 = out_fp16;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.tickets = reinterpret_cast<uint32_t*>(ws + d.ws_tickets);
+  a.qfrag = reinterpret_cast<uint32_t*>(ws + d.ws_qfrag);
+  a.hconst = reinterpret_cast<float*>(ws + d.ws_hconst);
+  a.qprime = reinterpret_cast<float*>(ws + d.ws_qprime);
+  a.partials = reinterpret_cast<float*>(ws + d.ws_partials);
+  const cudaError_t e = launch_decode(d, cfg->bits, a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA;
+}

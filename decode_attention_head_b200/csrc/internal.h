@@ -1,0 +1,83 @@
+// Internal interfaces between the C-ABI layer (abi.cu) and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include "../../include/wushkv.h"
+
+namespace wushkv {
+
+constexpr int kHeadDim = 128;
+constexpr int kTileTokens = 64;       // positions per decode pipeline stage (and cap_alloc granule)
+constexpr int kB200SMs = 148;         // split policy sizes the decode grid for this many SMs
+constexpr int kDecodeCtasPerSM = 3;   // resident decode CTAs per SM the policy aims at
+constexpr int kMaxSplits = 255;       // quantized work items per (sequence, KV head)
+
+struct Derived {
+  int units;        // B * H_kv
+  int group;        // H_q / H_kv
+  int cap_alloc;    // capacity rounded up to 64
+  int ring;         // ring slots
+  int sink_dim;     // max(s_sink, 1)
+  int code_bytes;   // 16 * bits
+  int nsel;         // extreme order statistics the quantizer keeps (2..4)
+  int i_lo, i_hi;
+  float f_lo, f_hi;
+  int n_split, split_tokens;
+  // workspace offsets (bytes)
+  size_t ws_tickets, ws_qfrag, ws_hconst, ws_qprime, ws_partials, ws_total;
+  // cache buffer sizes (bytes)
+  size_t codes_bytes, params_bytes, sink_bytes, ring_bytes, state_bytes;
+};
+
+// Validates cfg and fills d; returns WUSHKV_OK / WUSHKV_EINVAL / WUSHKV_EUNSUPPORTED.
+int derive(const wushkv_config* cfg, Derived* d);
+
+struct AppendArgs {
+  int B, Hkv, cap, cap_alloc, s_sink, s_keep, s_flush, R, sink_dim, n_new;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  uint32_t* k_params;
+  uint32_t* v_params;
+  __half* k_sink;
+  __half* v_sink;
+  __half* k_ring;
+  __half* v_ring;
+  int32_t* state;
+  uint32_t* status;
+  const __half* k_new;
+  const __half* v_new;
+  const __half* t_k;
+  int i_lo, i_hi;
+  float f_lo, f_hi;
+};
+
+struct DecodeArgs {
+  int B, Hkv, Hq, cap_alloc, s_sink, R, sink_dim, n_split, split_tokens;
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const uint32_t* k_params;
+  const uint32_t* v_params;
+  const __half* k_sink;
+  const __half* v_sink;
+  const __half* k_ring;
+  const __half* v_ring;
+  const int32_t* state;
+  uint32_t* status;
+  const __half* q;
+  const float* t_k_inv;
+  float scale_log2;  // softmax_scale * log2(e)
+  void* out;
+  int out_fp16;
+  uint32_t* tickets;
+  uint32_t* qfrag;
+  float* hconst;
+  float* qprime;
+  float* partials;
+};
+
+cudaError_t launch_append(const Derived& d, int bits, bool small, const AppendArgs& a, cudaStream_t st);
+cudaError_t launch_decode(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st);
+
+}  // namespace wushkv

@@ -1,0 +1,182 @@
+// Per-token percentile-clipped asymmetric affine quantizer, one thread per token-head
+// ("WUSH-KV: KV Cache Quantization with Data-Adaptive Transforms", §5.3: percentile
+// clipping with asymmetric affine scaling and an adaptive zero point; §1: per-token
+// clipped quantizers).
+//
+// For the 128 fp16 values x of one token's head vector:
+//   lo, hi = p_lo / p_hi percentiles, linear interpolation at rank p/100*127 between
+//            sorted values, P = s[i] + f*(s[i+1] - s[i]) in fp32, each op rounded alone
+//   s = fp16_rn((hi - lo) / (2^bits - 1)),  z = fp16_rn(lo)
+//   code = clamp(round_half_even(fp32(x - z) / s), 0, 2^bits - 1); s == 0 -> 0
+// Only the NSEL smallest and NSEL largest values are needed (NSEL <= 4 covers the
+// ranks of percentiles within 4 of either end); they are selected with half2 min/max
+// insertion networks (exact: the values are fp16 and fp16 comparisons are exact).
+// The division is done as a multiplication by the correctly rounded reciprocal; where
+// that product lies within its error bound of a rounding midpoint, the exact IEEE
+// division decides, so the code always equals round(fl32(fl32(x - z) / s)).
+#pragma once
+#include <cuda_fp16.h>
+#include <cstdint>
+#include "ptx.cuh"
+
+namespace wushkv {
+
+struct QuantSpec {
+  int i_lo, i_hi;   // ranks floor(p/100 * 127)
+  float f_lo, f_hi; // fractional parts, fp32
+};
+
+// Insert x into the ascending list a[0..K-1] of the K smallest seen so far (both halves
+// of the half2 independently).
+template <int K>
+__device__ __forceinline__ void insert_small(__half2 (&a)[K], __half2 x) {
+  __half2 mx[K];
+#pragma unroll
+  for (int j = 0; j < K - 1; ++j) mx[j] = __hmax2(a[j], x);
+  a[0] = __hmin2(a[0], x);
+#pragma unroll
+  for (int j = 1; j < K; ++j) a[j] = __hmin2(a[j], mx[j - 1]);
+}
+
+// Insert x into the descending list b[0..K-1] of the K largest seen so far.
+template <int K>
+__device__ __forceinline__ void insert_large(__half2 (&b)[K], __half2 x) {
+  __half2 mn[K];
+#pragma unroll
+  for (int j = 0; j < K - 1; ++j) mn[j] = __hmin2(b[j], x);
+  b[0] = __hmax2(b[0], x);
+#pragma unroll
+  for (int j = 1; j < K; ++j) b[j] = __hmax2(b[j], mn[j - 1]);
+}
+
+template <int K>
+__device__ __forceinline__ void merge_small(float (&a)[K], const float (&b)[K]) {
+#pragma unroll
+  for (int i = 0; i < K; ++i) {
+    float x = b[i];
+    float mx[K];
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) mx[j] = fmaxf(a[j], x);
+    a[0] = fminf(a[0], x);
+#pragma unroll
+    for (int j = 1; j < K; ++j) a[j] = fminf(a[j], mx[j - 1]);
+  }
+}
+
+template <int K>
+__device__ __forceinline__ void merge_large(float (&a)[K], const float (&b)[K]) {
+#pragma unroll
+  for (int i = 0; i < K; ++i) {
+    float x = b[i];
+    float mn[K];
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) mn[j] = fminf(a[j], x);
+    a[0] = fmaxf(a[0], x);
+#pragma unroll
+    for (int j = 1; j < K; ++j) a[j] = fmaxf(a[j], mn[j - 1]);
+  }
+}
+
+// P = s_i + f * (s_j - s_i), three separately rounded fp32 operations.
+__device__ __forceinline__ float interp(float si, float sj, float f) {
+  return __fadd_rn(si, __fmul_rn(f, __fsub_rn(sj, si)));
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t quantize_one(float v, float zf, float sf, float rcp) {
+  constexpr float kLevels = float((1 << BITS) - 1);
+  const float t = __fsub_rn(v, zf);
+  float q = __fmul_rn(t, rcp);
+  float c = rintf(q);
+  const float dist = fabsf(__fsub_rn(q, c));
+  // |q - fl(t/s)| <= 1.8e-7 |q|: only a midpoint inside that band can change the rounding
+  if (dist > 0.5f - fmaf(2.5e-7f, fabsf(q), 1e-30f)) {
+    c = rintf(__fdiv_rn(t, sf));
+  }
+  c = fminf(fmaxf(c, 0.0f), kLevels);
+  return static_cast<uint32_t>(c);
+}
+
+// Quantize the 128 fp16 values at x (global or shared, 16-byte aligned) and write the
+// packed codes (16*BITS bytes, 16-byte aligned) and the half2 (s, z).
+template <int BITS, int NSEL>
+__device__ __noinline__ void quantize_row(const __half* __restrict__ x, uint8_t* __restrict__ codes_out,
+                                          uint32_t* __restrict__ params_out, const QuantSpec qs) {
+  __half2 v[64];
+  const uint4* src = reinterpret_cast<const uint4*>(x);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    uint4 u = src[i];
+    v[4 * i + 0] = u32_as_h2(u.x);
+    v[4 * i + 1] = u32_as_h2(u.y);
+    v[4 * i + 2] = u32_as_h2(u.z);
+    v[4 * i + 3] = u32_as_h2(u.w);
+  }
+  // --- order statistics at both ends
+  const __half2 pinf = __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));
+  const __half2 ninf = __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));
+  __half2 a[NSEL], b[NSEL];
+#pragma unroll
+  for (int j = 0; j < NSEL; ++j) {
+    a[j] = pinf;
+    b[j] = ninf;
+  }
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    insert_small<NSEL>(a, v[i]);
+    insert_large<NSEL>(b, v[i]);
+  }
+  float lo_s[NSEL], lo_t[NSEL], hi_s[NSEL], hi_t[NSEL];
+#pragma unroll
+  for (int j = 0; j < NSEL; ++j) {
+    lo_s[j] = __low2float(a[j]);
+    lo_t[j] = __high2float(a[j]);
+    hi_s[j] = __low2float(b[j]);
+    hi_t[j] = __high2float(b[j]);
+  }
+  merge_small<NSEL>(lo_s, lo_t);  // lo_s[j] = s[j]
+  merge_large<NSEL>(hi_s, hi_t);  // hi_s[j] = s[127 - j]
+  // s[i] for i in {i_lo, i_lo+1} from the bottom list, {i_hi, min(i_hi+1,127)} from the top
+  float slo0 = 0.f, slo1 = 0.f, shi0 = 0.f, shi1 = 0.f;
+  const int jh0 = 127 - qs.i_hi;
+  const int jh1 = 127 - min(qs.i_hi + 1, 127);
+#pragma unroll
+  for (int j = 0; j < NSEL; ++j) {
+    if (j == qs.i_lo) slo0 = lo_s[j];
+    if (j == qs.i_lo + 1) slo1 = lo_s[j];
+    if (j == jh0) shi0 = hi_s[j];
+    if (j == jh1) shi1 = hi_s[j];
+  }
+  const float lo = interp(slo0, slo1, qs.f_lo);
+  const float hi = interp(shi0, shi1, qs.f_hi);
+  const float scale32 = __fdiv_rn(__fsub_rn(hi, lo), float((1 << BITS) - 1));
+  const __half s_h = __float2half_rn(scale32);
+  const __half z_h = __float2half_rn(lo);
+  const float sf = __half2float(s_h);
+  const float zf = __half2float(z_h);
+
+  constexpr int NW = 4 * BITS;  // 32-bit words of packed codes
+  uint32_t w[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) w[i] = 0u;
+  if (sf != 0.0f) {
+    const float rcp = __frcp_rn(sf);
+#pragma unroll
+    for (int k = 0; k < 64; ++k) {
+      const float2 f = __half22float2(v[k]);
+      const uint32_t c0 = quantize_one<BITS>(f.x, zf, sf, rcp);
+      const uint32_t c1 = quantize_one<BITS>(f.y, zf, sf, rcp);
+      if (BITS == 2) {
+        w[k / 8] |= (c0 | (c1 << 2)) << (4 * (k % 8));
+      } else {
+        w[k / 4] |= (c0 | (c1 << 4)) << (8 * (k % 4));
+      }
+    }
+  }
+  uint4* dst = reinterpret_cast<uint4*>(codes_out);
+#pragma unroll
+  for (int i = 0; i < NW / 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  *params_out = h2_as_u32(__halves2half2(s_h, z_h));
+}
+
+}  // namespace wushkv

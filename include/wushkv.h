@@ -1,0 +1,167 @@
+/*
+ * wushkv.h -- C ABI of libwushkv: the WUSH-KV append + decode-attention hot path
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method ("WUSH-KV: KV Cache Quantization with Data-Adaptive Transforms"):
+ *   - append (§4.1, §4.2, §4.4, §5.3): every new post-RoPE key k of KV head h is
+ *     transformed, k' = T_K k (T_K a full invertible 128x128 matrix fixed at
+ *     calibration); the value v arrives already in its transformed basis (the value
+ *     transform is folded into the weights, §4.5) and is stored as given.  The first
+ *     s_sink positions and the newest s_keep positions stay fp16; the rest is
+ *     quantized per token with a percentile-clipped asymmetric affine quantizer to
+ *     2 or 4 bits, in batches of s_flush positions (Algorithm 2 prose, §4.4).
+ *   - decode attention (§4.1, §4.2): each query is compensated, q' = T_K^{-T} q, so
+ *     q'.k' = q.k; keys and values are dequantized on the fly and the fp16 sink and
+ *     recent windows are merged in one exact softmax over all S cached positions.
+ *     The output stays in the value-transform basis (the output projection undoes it).
+ *
+ * Conventions shared by every entry point:
+ *   - head_dim d must be 128; bits must be 2 or 4; n_q_heads / n_kv_heads = g must
+ *     be 1, 2, 4 or 8; query head j reads KV head j / g.
+ *   - fp16 means IEEE binary16 stored as uint16; half2 means two fp16 in 4 bytes,
+ *     the first (lower address) element in the low half.
+ *   - All device buffers are allocated and owned by the caller (sizes from
+ *     wushkv_pack_layout), must be 16-byte aligned, and stay valid until the work
+ *     queued on `stream` has finished.  The library allocates nothing and keeps no
+ *     global state.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   - Calls are asynchronous: a zero return means the work was validated and
+ *     queued.  Conditions only the device can see (capacity overflow, decode of an
+ *     empty sequence, a bounded wait that gave up) are OR-ed into the cache's
+ *     status word (below); nothing traps.
+ *   - Inputs must be finite (no NaN/Inf).
+ *
+ * Return codes: WUSHKV_OK, or a negative WUSHKV_E* value; on error nothing is queued
+ * and no buffer is touched.
+ */
+#ifndef WUSHKV_H
+#define WUSHKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WUSHKV_OK 0
+#define WUSHKV_EINVAL (-1)       /* null/misaligned pointer, bad window or percentile values */
+#define WUSHKV_EUNSUPPORTED (-2) /* head_dim != 128, bits not 2/4, g not 1/2/4/8, percentiles
+                                    needing more than the 4 extreme order statistics */
+#define WUSHKV_ECUDA (-3)        /* a CUDA launch or query failed */
+#define WUSHKV_ESINGULAR (-4)    /* wushkv_compensation: T_K is singular */
+
+/* Bits of the device status word (state buffer, int32 index 2*batch*n_kv_heads). */
+#define WUSHKV_STATUS_OVERFLOW 1u /* an append would exceed `capacity`: that sequence was skipped */
+#define WUSHKV_STATUS_EMPTY 2u    /* decode of a sequence with S == 0: its output rows are zero */
+#define WUSHKV_STATUS_TIMEOUT 4u  /* a bounded in-kernel wait gave up (a library bug, not an input error) */
+#define WUSHKV_STATUS_BADSTATE 8u /* a state entry was out of range (S < 0, S > capacity, S_quant outside
+                                     [0, S]): that (sequence, KV head) was skipped / read as empty */
+
+/* Cache configuration; one cache holds one attention layer. */
+typedef struct wushkv_config {
+  int32_t batch;       /* B, sequences */
+  int32_t n_kv_heads;  /* H_kv */
+  int32_t n_q_heads;   /* H_q, a multiple of H_kv with H_q / H_kv in {1, 2, 4, 8} */
+  int32_t head_dim;    /* d, must be 128 */
+  int32_t bits;        /* 2 or 4 */
+  int32_t capacity;    /* positions per sequence, >= 1 */
+  int32_t s_sink;      /* S_sink >= 0: first positions kept fp16 for good */
+  int32_t s_keep;      /* S_keep >= 0: newest positions kept fp16 */
+  int32_t s_flush;     /* S_flush >= 1: quantization batch */
+  int32_t chunk_max;   /* >= 1: appends of at most chunk_max tokens stay fp16 until the next
+                          append (the pages' order: append, attend, then quantize); larger
+                          appends are quantized on arrival */
+  float p_lo;          /* clipping percentiles, 0 <= p_lo < p_hi <= 100; the needed order */
+  float p_hi;          /* statistics must lie within 4 of either end (e.g. 1/99, 0.5/99.5) */
+} wushkv_config;
+
+/* Byte sizes of the caller-allocated buffers (wushkv_pack_layout). */
+typedef struct wushkv_layout {
+  size_t codes_bytes;     /* each of k_codes, v_codes: uint8 [B][H_kv][cap_alloc][code_bytes] */
+  size_t params_bytes;    /* each of k_params, v_params: half2 (s, z) [B][H_kv][cap_alloc] */
+  size_t sink_bytes;      /* each of k_sink, v_sink: fp16 [B][H_kv][max(s_sink,1)][128] */
+  size_t ring_bytes;      /* each of k_ring, v_ring: fp16 [B][H_kv][ring_slots][128] */
+  size_t state_bytes;     /* int32 [B*H_kv][2] = (S, S_quant) per (sequence, KV head), then the
+                             status word; zero it to start from an empty cache */
+  size_t workspace_bytes; /* wushkv_decode_attn scratch; no initialisation needed */
+  int32_t cap_alloc;      /* capacity rounded up to a multiple of 64 */
+  int32_t ring_slots;     /* s_keep + s_flush - 1 + chunk_max; position p lives in slot p % ring_slots */
+  int32_t code_bytes;     /* 128 * bits / 8 bytes of packed codes per token and head */
+  int32_t n_splits;       /* decode work items per (sequence, KV head) over the quantized region */
+  int32_t split_tokens;   /* positions per decode work item (multiple of 64) */
+  int32_t reserved;
+} wushkv_layout;
+
+/* Device pointers of one layer's cache.
+ *  codes: code j (0..127) of position p is in byte (j*bits)/8 at bit offset (j*bits)%8 of
+ *         the code_bytes-long record of p (little-endian within the byte); records are
+ *         indexed by absolute position p; only S_sink <= p < S_quant are meaningful.
+ *  params: (s, z) of position p; the token's values dequantize to z + s * code.
+ *  sink:  k' / v of positions p < s_sink at index p.
+ *  ring:  k' / v of fp16 positions p >= max(S_quant, s_sink) at slot p % ring_slots.
+ *  k' (keys in the transformed basis) is what every key buffer holds. */
+typedef struct wushkv_cache {
+  void* k_codes;
+  void* v_codes;
+  void* k_params;
+  void* v_params;
+  void* k_sink;
+  void* v_sink;
+  void* k_ring;
+  void* v_ring;
+  int32_t* state;
+} wushkv_cache;
+
+/* Validate `cfg` and fill `out` with the buffer sizes the caller must allocate.
+ * Host only; touches no device.  Returns WUSHKV_OK, WUSHKV_EINVAL or WUSHKV_EUNSUPPORTED. */
+int wushkv_pack_layout(const wushkv_config* cfg, wushkv_layout* out);
+
+/* One-time calibration helper (host only): the compensation matrix for the query side.
+ * t_k:   host fp16 [n_kv_heads][128][128], T_K row-major acting on column vectors
+ *        (k'[r] = sum_i T_K[r][i] k[i]).
+ * t_k_inv: host fp32 [n_kv_heads][128][128] output, T_K^{-1} row-major, computed in double
+ *        precision by Gauss-Jordan elimination with partial pivoting, then rounded.
+ * The query compensation of §4.2, q' = T_K^{-T} q, reads it as q'[j] = sum_i t_k_inv[i][j] q[i].
+ * Returns WUSHKV_OK, WUSHKV_EINVAL or WUSHKV_ESINGULAR. */
+int wushkv_compensation(const uint16_t* t_k, int32_t n_kv_heads, float* t_k_inv);
+
+/* Append n_new >= 0 tokens to every sequence (§4.1, §4.2, §4.4 "Full-Precision Cache
+ * Window", §5.3 quantizer).
+ * k_new, v_new: device fp16 [B][n_new][H_kv][128]; keys after head-norm and RoPE,
+ *               values already in the value-transform basis.
+ * t_k:          device fp16 [H_kv][128][128], T_K row-major; k' = fp16_rn(T_K k), fp32 accumulation.
+ * Steps, per (sequence, KV head) with state (S, S_quant):
+ *   if S + n_new > capacity: set WUSHKV_STATUS_OVERFLOW, leave the sequence unchanged;
+ *   n_new <= chunk_max: flush under length S (closes the previous chunk), then store the
+ *                       n_new tokens fp16 (sink or ring), S += n_new;
+ *   n_new >  chunk_max: store, S += n_new, flush under the new S (tokens that the flush
+ *                       covers are quantized straight from registers).
+ *   flush under L: lo0 = max(S_quant, s_sink); e = L - s_keep - lo0; if e >= s_flush,
+ *                  quantize positions [lo0, lo0 + floor(e/s_flush)*s_flush) and move S_quant.
+ *   quantize one token's 128 values x (fp16): sort; lo/hi = the p_lo/p_hi percentiles,
+ *     linear interpolation at rank p/100*127 in fp32 (s[i] + f*(s[i+1]-s[i]), each op
+ *     rounded); s = fp16_rn((hi - lo)/(2^bits - 1)), z = fp16_rn(lo);
+ *     code = clamp(round_half_even(fp32(x - z) / s), 0, 2^bits - 1), code = 0 when s == 0.
+ * Returns WUSHKV_OK, WUSHKV_EINVAL, WUSHKV_EUNSUPPORTED or WUSHKV_ECUDA. */
+int wushkv_append(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new,
+                  const void* v_new, int32_t n_new, const void* t_k, void* stream);
+
+/* Decode attention of one query per sequence over the whole cache (§4.1, §4.2, §4.4).
+ * q:        device fp16 [B][H_q][128], after head-norm and RoPE.
+ * t_k_inv:  device fp32 [H_kv][128][128], T_K^{-1} row-major (see wushkv_compensation).
+ * softmax_scale: logits are softmax_scale * q.k (1/sqrt(128) for standard attention).
+ * out_fp16: 0 -> out is fp32 [B][H_q][128]; 1 -> fp16.
+ * workspace: device scratch of layout.workspace_bytes (no initialisation needed).
+ * out[b][j] = sum_p softmax_p(softmax_scale * q'_j . khat_p) vhat_p over p < S, with
+ *   q'_j = T_K^{-T} q_j, khat_p / vhat_p the stored fp16 k'/v in the windows and
+ *   z + s*code in the quantized region.  S == 0 gives zeros and WUSHKV_STATUS_EMPTY.
+ * Returns WUSHKV_OK, WUSHKV_EINVAL, WUSHKV_EUNSUPPORTED or WUSHKV_ECUDA. */
+int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* cache, const void* q,
+                       const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
+                       void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WUSHKV_H */

@@ -1,0 +1,89 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point the
+header declares, sizes buffers as documented, and rejects bad arguments before any
+device work."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wushkv.h")
+
+
+@pytest.fixture(scope="module")
+def bnd():
+    from decode_attention_head_b200 import build
+    build.build()
+    from decode_attention_head_b200 import binding
+    return binding
+
+
+def test_exports_every_declared_symbol(bnd):
+    text = open(HEADER).read()
+    declared = set(re.findall(r"^\s*int\s+(wushkv_\w+)\s*\(", text, flags=re.M))
+    assert declared == set(bnd.SYMBOLS)
+    for name in declared:
+        assert hasattr(bnd.lib, name)
+    # the exported names of the .so, read from the dynamic symbol table via ctypes
+    for name in declared:
+        assert ctypes.cast(getattr(bnd.lib, name), ctypes.c_void_p).value
+
+
+def test_layout_sizes(bnd):
+    cfg = bnd.make_config(8, 8, 32, 2, 32768 + 1000, 4, 128, 16, 1)
+    L = bnd.pack_layout(cfg)
+    assert L.cap_alloc == 33792 and L.cap_alloc % 64 == 0
+    assert L.code_bytes == 32
+    assert L.ring_slots == 128 + 16 - 1 + 1
+    assert L.codes_bytes == 64 * 33792 * 32
+    assert L.params_bytes == 64 * 33792 * 4
+    assert L.sink_bytes == 64 * 4 * 128 * 2
+    assert L.ring_bytes == 64 * 144 * 128 * 2
+    assert L.state_bytes >= (2 * 64 + 1) * 4
+    assert L.split_tokens % 64 == 0 and L.n_splits * L.split_tokens >= L.cap_alloc
+    assert L.workspace_bytes > 0
+    cfg4 = bnd.make_config(64, 32, 32, 4, 8192, 4, 64, 16, 1, 0.5, 99.5)
+    L4 = bnd.pack_layout(cfg4)
+    assert L4.code_bytes == 64 and L4.codes_bytes == 64 * 32 * 8192 * 64
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("head_dim", 64, -2), ("bits", 3, -2), ("n_q_heads", 24, -2), ("n_q_heads", 7, -1), ("n_q_heads", 12, -2),
+    ("s_flush", 0, -1), ("chunk_max", 0, -1), ("capacity", 0, -1), ("s_sink", -1, -1),
+    ("p_lo", 99.0, -1), ("p_hi", 101.0, -1), ("p_lo", 10.0, -2)])
+def test_bad_configs_rejected(bnd, field, value, code):
+    cfg = bnd.make_config(2, 2, 8, 2, 1000, 4, 32, 16, 1)
+    setattr(cfg, field, value)
+    out = bnd.Layout()
+    assert bnd.lib.wushkv_pack_layout(ctypes.byref(cfg), ctypes.byref(out)) == code
+
+
+def test_bad_pointers_rejected_before_device_work(bnd):
+    cfg = bnd.make_config(1, 1, 4, 2, 256, 4, 32, 16, 1)
+    bufs = bnd.CacheBufs()          # all null
+    rc = bnd.lib.wushkv_append(ctypes.byref(cfg), ctypes.byref(bufs), None, None, 1, None, None)
+    assert rc == bnd.EINVAL
+    rc = bnd.lib.wushkv_decode_attn(ctypes.byref(cfg), ctypes.byref(bufs), None, None, ctypes.c_float(0.1), 0,
+                                    None, None, None)
+    assert rc == bnd.EINVAL
+    assert bnd.lib.wushkv_pack_layout(None, None) == bnd.EINVAL
+
+
+def test_compensation_inverts_fp16_transform(bnd):
+    rng = np.random.default_rng(7)
+    q, r = np.linalg.qr(rng.standard_normal((3, 128, 128)))
+    t = (q * rng.uniform(0.5, 2, (3, 1, 128))).astype(np.float16)
+    inv = bnd.compensation(torch.from_numpy(t)).numpy()
+    ref = np.linalg.inv(t.astype(np.float64))
+    np.testing.assert_allclose(inv, ref, rtol=0, atol=1e-5 * np.abs(ref).max())
+    eye = np.einsum("hij,hjk->hik", t.astype(np.float64), inv.astype(np.float64))
+    np.testing.assert_allclose(eye, np.broadcast_to(np.eye(128), eye.shape), atol=1e-4)
+
+
+def test_compensation_rejects_singular(bnd):
+    t = torch.zeros(1, 128, 128, dtype=torch.float16)
+    with pytest.raises(bnd.WushKVError):
+        bnd.compensation(t)
