@@ -42,14 +42,14 @@ def percentile_rank(p: float, d: int):
 def percentile_fp32(x_sorted: np.ndarray, i: int, f: np.float32) -> np.ndarray:
     """Linear interpolation between order statistics, in fp32.
 
-    P = s[i] + f * (s[i+1] - s[i]), three separately rounded fp32 operations;
-    P = s[d-1] when i is the last rank.  x_sorted: float32 [..., d] ascending.
+    P = s[i] + f * (s[i+1] - s[i]), three separately rounded fp32 operations,
+    with s[d] read as s[d-1] (the 100th percentile is the maximum, plus +0).
+    Written this way the result never depends on how a sort orders -0 and +0.
+    x_sorted: float32 [..., d] ascending.
     """
     d = x_sorted.shape[-1]
     a = x_sorted[..., i]
-    if i >= d - 1:
-        return a.astype(np.float32)
-    b = x_sorted[..., i + 1]
+    b = x_sorted[..., min(i + 1, d - 1)]
     diff = np.subtract(b, a, dtype=np.float32)
     step = np.multiply(np.float32(f), diff, dtype=np.float32)
     return np.add(a, step, dtype=np.float32)
