@@ -686,7 +686,7 @@ cudaError_t launch_decode_t(const Derived& d, const DecodeArgs& a, cudaStream_t 
   if (e != cudaSuccess) return e;
   const int nitems = d.n_split + 1;
   const size_t smem = main_smem_bytes<BITS, G>(nitems);
-  e = cudaFuncSetAttribute(decode_main_kernel<BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = ensure_smem_attr(decode_main_kernel<BITS, G>, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(nitems, d.units);
   decode_main_kernel<BITS, G><<<grid, kThreads, smem, st>>>(a);

@@ -77,6 +77,20 @@ struct DecodeArgs {
   float* partials;
 };
 
+// Raise a kernel's dynamic shared-memory limit once per device (a function attribute,
+// not a stream operation, so it is kept out of the launch path and of graph capture).
+template <typename F>
+cudaError_t ensure_smem_attr(F* fn, int bytes) {
+  static int done[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = bytes;
+  return e;
+}
+
 cudaError_t launch_append(const Derived& d, int bits, bool small, const AppendArgs& a, cudaStream_t st);
 cudaError_t launch_decode(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st);
 

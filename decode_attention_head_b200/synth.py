@@ -238,3 +238,48 @@ def scaled(wl: Workload, **changes) -> Workload:
 
 def default_softmax_scale(d: int = HEAD_DIM) -> float:
     return 1.0 / math.sqrt(d)
+
+
+def bulk_tokens(wl: Workload, layer: int, start: int, n: int, device="cpu", which: str = "k",
+                gen_seed: Optional[int] = None) -> torch.Tensor:
+    """Keys or values of positions [start, start+n) for all (b, h) in one draw: fp16 [B, n, H_kv, d].
+
+    Same recipe as `keys` / `values` (outlier channels per KV head, RMSNorm, RoPE at the
+    positions, Student-t(5) values), but one generator per call, so it is fast on a GPU
+    and not element-identical to the per-unit streams.
+    """
+    tag = _TAG_K if which == "k" else _TAG_V
+    seed = unit_seed(wl.seed, tag + 50, layer, start, n) if gen_seed is None else gen_seed
+    g = _gen(device, seed)
+    B, H, d = wl.batch, wl.n_kv_heads, wl.head_dim
+    if tag == _TAG_V and wl.v_dist == "student_t5":
+        z = torch.randn(B, n, H, d, generator=g, device=device)
+        chi = torch.zeros_like(z)
+        for _ in range(5):
+            chi.add_(torch.randn(B, n, H, d, generator=g, device=device).pow_(2))
+        x = z.div_(chi.div_(5.0).sqrt_())
+    else:
+        x = torch.randn(B, n, H, d, generator=g, device=device)
+        for h in range(H):
+            ch = _outlier_channels(wl, tag, layer, h).to(device)
+            x[:, :, h, ch] *= 20.0
+    if tag == _TAG_K:
+        if wl.qk_rmsnorm:
+            x = _rmsnorm(x)
+        if wl.rope_theta is not None:
+            pos = torch.arange(start, start + n, device=device)
+            x = _rope(x.transpose(1, 2), pos, wl.rope_theta).transpose(1, 2)
+    return x.to(torch.float16).contiguous()
+
+
+def bulk_queries(wl: Workload, layer: int, position: int, device="cpu", gen_seed: Optional[int] = None):
+    """Decode queries of every sequence at `position` in one draw: fp16 [B, H_q, d]."""
+    seed = unit_seed(wl.seed, _TAG_Q + 50, layer, position) if gen_seed is None else gen_seed
+    g = _gen(device, seed)
+    x = torch.randn(wl.batch, wl.n_q_heads, wl.head_dim, generator=g, device=device)
+    if wl.qk_rmsnorm:
+        x = _rmsnorm(x)
+    if wl.rope_theta is not None:
+        pos = torch.full((wl.n_q_heads,), position, device=device)
+        x = _rope(x, pos, wl.rope_theta)
+    return x.to(torch.float16)
