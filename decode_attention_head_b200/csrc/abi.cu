@@ -45,8 +45,8 @@ int derive(const wushkv_config* cfg, Derived* d) {
   if (d->nsel < 2) d->nsel = 2;
   if (d->nsel > 4) return WUSHKV_EUNSUPPORTED;
 
-  // decode work split: ~kDecodeCtasPerSM quantized items per SM over all units
-  int per_unit = ceil_div(kB200SMs * kDecodeCtasPerSM, d->units);
+  // decode work split: at most one wave of items over all units
+  int per_unit = (kB200SMs * decode_ctas_per_sm(g)) / d->units;
   if (per_unit < 1) per_unit = 1;
   if (per_unit > kMaxSplits) per_unit = kMaxSplits;
   int L = ceil_div(ceil_div(d->cap_alloc, per_unit), kTileTokens) * kTileTokens;
@@ -70,7 +70,7 @@ int derive(const wushkv_config* cfg, Derived* d) {
   d->ws_qprime = off;
   off = round_up(off + U * g * kHeadDim * 4, 256);
   d->ws_partials = off;
-  off = round_up(off + U * (size_t)(d->n_split + 1) * g * 132 * 4, 256);
+  off = round_up(off + U * (size_t)d->n_split * g * 132 * 4, 256);
   d->ws_total = off;
   return WUSHKV_OK;
 }

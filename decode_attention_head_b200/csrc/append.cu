@@ -286,7 +286,7 @@ cudaError_t launch_append_t(const Derived& d, bool small, const AppendArgs& a, c
   flush_ring_kernel<BITS, NSEL><<<d.units, 128, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = ensure_smem_attr(append_bulk_kernel<BITS, NSEL>, (int)kBulkSmem);
+  e = ensure_smem_attr<append_bulk_kernel<BITS, NSEL>>((int)kBulkSmem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n_new + kBulkSlab - 1) / kBulkSlab, d.units);
   append_bulk_kernel<BITS, NSEL><<<grid, 128, kBulkSmem, st>>>(a);

@@ -4,22 +4,24 @@
 // §4.4 fp16 sink / recent windows around the quantized middle region).
 //
 // Two launches per call:
-//  1. decode_prologue: per (sequence, KV head), q'_j = T_K^{-T} q_j for its g query
-//     heads (fp32), and q' re-expressed as a 31-bit fixed-point integer split into
-//     four signed 8-bit limbs, laid out as mma.sync B fragments.  Also zeroes the
-//     per-unit completion ticket.
-//  2. decode_main: grid (1 + n_split, units).  Work item 0 of a unit attends over its
-//     fp16 windows; item s >= 1 over positions [(s-1)L, sL) of the quantized region.
-//     A quantized item streams 64-position tiles (K codes, V codes, K and V (s,z))
-//     into shared memory with bulk copies on an mbarrier ring (one producer warp, four
-//     consumer warps), and per 16-position slice:
-//       QK  : u8 codes x s8 query limbs on tensor cores (mma m16n8k32, int32 exact),
+//  1. decode_prologue (one CTA per (sequence, KV head)): q'_j = T_K^{-T} q_j for its g
+//     query heads (fp32), q' re-expressed as a 31-bit fixed-point integer split into
+//     four signed 8-bit limbs laid out as mma.sync B fragments, and the per-unit
+//     completion ticket reset.  It releases the main kernel at once (programmatic
+//     dependent launch), so the main kernel's KV stream starts while it runs.
+//  2. decode_main: grid (n_split, units).  Item s of a unit attends over positions
+//     [sL, (s+1)L) of the quantized region [S_sink, S_quant) and over its share of the
+//     unit's fp16 window positions (sink [0, S_sink) and recent [S_quant, S)).
+//     The quantized positions stream through shared memory in 128-position stages
+//     (K codes, V codes, K and V (s, z)) via bulk copies on an mbarrier ring: one
+//     producer warp, four consumer warps, 32 positions per consumer warp per stage:
+//       QK  : u8 codes x s8 query limbs on tensor cores (mma m16n8k32, exact int32),
 //             logit = log2e*scale*(z*sum(q') + s*sigma*D)  (dequantization folded);
-//       softmax: online, base 2, rescale only when the running max grows;
-//       PV  : fp16 codes x fp16 p*s on tensor cores (mma m16n8k16, fp32 accumulate),
-//             plus sum(p*z) for the zero-point term.
-//     Each item merges its four warps and writes (m, l, o); the last item of a unit
-//     to finish (atomic ticket, no waiting) merges all items and writes the output.
+//       softmax: online, base 2, the running max rescales only when it grows;
+//       PV  : fp16 codes x fp16 (p*s as hi + lo) on tensor cores (mma m16n8k16,
+//             fp32 accumulate), plus sum(p*z) for the zero-point term.
+//     Each item merges its warps and writes (m, l, o); the last item of a unit to
+//     finish (atomic ticket, no waiting) merges all items and writes the output.
 //
 // Code unpacking needs no shifts on the key side: masking a packed 32-bit word with
 // 0x03030303 << 2j leaves, in each byte, one code times 4^j -- an exact u8 operand.
@@ -43,17 +45,23 @@ namespace {
 
 constexpr float kQMax = 1073741824.0f;  // |fixed-point query| <= 2^30; four signed 8-bit limbs hold +-2.1e9
 constexpr int kFragWords = 4 * 4 * 64;   // per unit: [kstep 4][n-tile <= 4][lane 32][2] words
-constexpr int kThreads = 160;   // 4 consumer warps + 1 producer warp
-constexpr int kPartStride = 132;  // floats per (item, head) partial: m, l, pad, pad, o[128]
+constexpr int kThreads = 160;            // 4 consumer warps + 1 producer warp
+constexpr int kConsumers = 4;
+constexpr int kSlice = 32;               // positions per consumer warp per stage
+constexpr int kPartStride = 132;         // floats per (item, head) partial: m, l, pad, pad, o[128]
+static_assert(kTileTokens == kConsumers * kSlice, "a stage holds one slice per consumer warp");
 
 // 2^n as an fp32 bit pattern, exact for -126 <= n <= 127.
 __device__ __forceinline__ float pow2i(int n) { return __int_as_float((n + 127) << 23); }
 
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 template <int BITS>
 struct Cfg {
   static constexpr int CB = 16 * BITS;
-  static constexpr int NSTAGE = BITS == 2 ? 8 : 4;
-  static constexpr int STAGE = 2 * kTileTokens * CB + 2 * kTileTokens * 4;
+  static constexpr int NSTAGE = BITS == 2 ? 4 : 3;
+  static constexpr int STAGE = kTileTokens * (2 * CB + 8);
 };
 
 template <int G>
@@ -67,7 +75,7 @@ struct GCfg {
 template <int BITS>
 __host__ __device__ __forceinline__ void key_slot(int dim, int& kstep, int& t4, int& r, int& byte, int& log2scale) {
   if (BITS == 2) {
-    const int w = dim >> 4;   // word of 16 codes
+    const int w = dim >> 4;  // word of 16 codes
     byte = (dim & 15) >> 2;
     const int plane = dim & 3;
     t4 = w >> 1;
@@ -75,7 +83,7 @@ __host__ __device__ __forceinline__ void key_slot(int dim, int& kstep, int& t4, 
     kstep = plane;
     log2scale = 2 * plane;
   } else {
-    const int w = dim >> 3;   // word of 8 codes
+    const int w = dim >> 3;  // word of 8 codes
     byte = (dim & 7) >> 1;
     const int plane = dim & 1;
     t4 = w >> 2;
@@ -91,12 +99,12 @@ __host__ __device__ __forceinline__ void key_slot(int dim, int& kstep, int& t4, 
 template <int BITS>
 __device__ __forceinline__ void value_row(int mt, int g, int hi, int& dim, int& log2scale) {
   if (BITS == 2) {
-    dim = 16 * g + 8 * hi + mt;                 // code mt of the chunk
-    log2scale = (mt & 1) && mt != 7 ? 6 : 8;    // placed at bits 6..7 or 8..9
+    dim = 16 * g + 8 * hi + mt;               // code mt of the chunk
+    log2scale = (mt & 1) && mt != 7 ? 6 : 8;  // placed at bits 6..7 or 8..9
   } else {
     const int ws = mt >> 2, mi = mt & 3;
     dim = 16 * g + 8 * ws + 4 * hi + mi;
-    log2scale = 6;                              // placed at bits 6..9
+    log2scale = 6;  // placed at bits 6..9
   }
 }
 
@@ -127,498 +135,589 @@ __device__ __forceinline__ uint32_t vcode4(uint32_t x, int mi) {
 }
 
 // ---------------------------------------------------------------------------------
+// Prologue: 256 threads; thread (half, j) sums half of q'[j] = sum_i Tinv[i][j] q[i].
 template <int BITS, int G>
-__global__ void __launch_bounds__(128) decode_prologue_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(256) decode_prologue_kernel(const DecodeArgs a) {
   constexpr int NT = GCfg<G>::NT;
   __shared__ float qs[G][kHeadDim];
+  __shared__ float part[G][kHeadDim];
   __shared__ uint32_t frag[4][NT][32][2];
   __shared__ float red_max[G][4], red_sum[G][4];
+  griddep_launch();
   const int unit = blockIdx.x;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
-  const int j = threadIdx.x, warp = j >> 5, lane = j & 31;
+  const int tid = threadIdx.x, j = tid & 127, half = tid >> 7;
+  const int warp = j >> 5, lane = j & 31;
 
-  for (int hh = 0; hh < G; ++hh) qs[hh][j] = __half2float(a.q[((size_t)b * a.Hq + h * G + hh) * kHeadDim + j]);
+  for (int i = tid; i < G * kHeadDim; i += 256) {
+    const int hh = i / kHeadDim, c = i % kHeadDim;
+    qs[hh][c] = __half2float(a.q[((size_t)b * a.Hq + h * G + hh) * kHeadDim + c]);
+  }
   uint32_t* fz = &frag[0][0][0][0];
-  for (int i = j; i < 4 * NT * 64; i += 128) fz[i] = 0u;
+  for (int i = tid; i < 4 * NT * 64; i += 256) fz[i] = 0u;
   __syncthreads();
 
-  // q'[j] = sum_i Tinv[i][j] q[i]
   float qp[G];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) qp[hh] = 0.f;
-  const float* Ti = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim;
-  for (int i = 0; i < kHeadDim; ++i) {
-    const float t = Ti[(size_t)i * kHeadDim + j];
+  const float* Ti = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim + (size_t)(64 * half) * kHeadDim + j;
+  for (int i0 = 0; i0 < 64; i0 += 16) {
+    float t[16];
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) qp[hh] = fmaf(t, qs[hh][i], qp[hh]);
+    for (int u = 0; u < 16; ++u) t[u] = __ldg(Ti + (size_t)(i0 + u) * kHeadDim);
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) qp[hh] = fmaf(t[u], qs[hh][64 * half + i0 + u], qp[hh]);
   }
+  if (half == 1) {
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) part[hh][j] = qp[hh];
+  }
+  __syncthreads();
   int kstep, t4, r, byte, l2s;
   key_slot<BITS>(j, kstep, t4, r, byte, l2s);
   const float inv_scale = 1.0f / float(1 << l2s);
+  if (half == 0) {
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    a.qprime[((size_t)unit * G + hh) * kHeadDim + j] = qp[hh] * a.scale_log2;
-    float m = fabsf(qp[hh]) * inv_scale, s = qp[hh];
+    for (int hh = 0; hh < G; ++hh) {
+      qp[hh] += part[hh][j];
+      a.qprime[((size_t)unit * G + hh) * kHeadDim + j] = qp[hh] * a.scale_log2;
+      float m = fabsf(qp[hh]) * inv_scale, s = qp[hh];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      s += __shfl_xor_sync(0xffffffffu, s, o);
-    }
-    if (lane == 0) {
-      red_max[hh][warp] = m;
-      red_sum[hh][warp] = s;
+      for (int o = 16; o > 0; o >>= 1) {
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        s += __shfl_xor_sync(0xffffffffu, s, o);
+      }
+      if (lane == 0) {
+        red_max[hh][warp] = m;
+        red_sum[hh][warp] = s;
+      }
     }
   }
   __syncthreads();
-  uint8_t* fb = reinterpret_cast<uint8_t*>(&frag[0][0][0][0]);
+  if (half == 0) {
+    uint8_t* fb = reinterpret_cast<uint8_t*>(&frag[0][0][0][0]);
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    const float amax = fmaxf(fmaxf(red_max[hh][0], red_max[hh][1]), fmaxf(red_max[hh][2], red_max[hh][3]));
-    const float sum = (red_sum[hh][0] + red_sum[hh][1]) + (red_sum[hh][2] + red_sum[hh][3]);
-    const float sigma = amax > 0.f ? amax / kQMax : 1.0f;
-    // balanced base-256 digits of Q, each in [-128, 127]
-    long long Q = __float2ll_rn(qp[hh] * inv_scale / sigma);
-    int limbs[4];
+    for (int hh = 0; hh < G; ++hh) {
+      const float amax = fmaxf(fmaxf(red_max[hh][0], red_max[hh][1]), fmaxf(red_max[hh][2], red_max[hh][3]));
+      const float sum = (red_sum[hh][0] + red_sum[hh][1]) + (red_sum[hh][2] + red_sum[hh][3]);
+      const float sigma = amax > 0.f ? amax / kQMax : 1.0f;
+      // balanced base-256 digits of Q, each in [-128, 127]
+      long long Q = __float2ll_rn(qp[hh] * inv_scale / sigma);
+      int limbs[4];
 #pragma unroll
-    for (int l = 0; l < 4; ++l) {
-      const long long d = ((Q + 128) & 255) - 128;
-      limbs[l] = (int)d;
-      Q = (Q - d) >> 8;
-    }
+      for (int l = 0; l < 4; ++l) {
+        const long long d = ((Q + 128) & 255) - 128;
+        limbs[l] = (int)d;
+        Q = (Q - d) >> 8;
+      }
 #pragma unroll
-    for (int l = 0; l < 4; ++l) {
-      const int nt = (l >> 1) * GCfg<G>::NHS + (hh >> 2);
-      const int col = 2 * (hh & 3) + (l & 1);
-      const int ln = 4 * col + t4;
-      fb[(((kstep * NT + nt) * 32 + ln) * 2 + r) * 4 + byte] = static_cast<uint8_t>(limbs[l] & 255);
-    }
-    if (j == 0) {
-      a.hconst[((size_t)unit * 8 + hh) * 2 + 0] = a.scale_log2 * sum;
-      a.hconst[((size_t)unit * 8 + hh) * 2 + 1] = a.scale_log2 * sigma;
+      for (int l = 0; l < 4; ++l) {
+        const int nt = (l >> 1) * GCfg<G>::NHS + (hh >> 2);
+        const int col = 2 * (hh & 3) + (l & 1);
+        const int ln = 4 * col + t4;
+        fb[(((kstep * NT + nt) * 32 + ln) * 2 + r) * 4 + byte] = static_cast<uint8_t>(limbs[l] & 255);
+      }
+      if (j == 0) {
+        a.hconst[((size_t)unit * 8 + hh) * 2 + 0] = a.scale_log2 * sum;
+        a.hconst[((size_t)unit * 8 + hh) * 2 + 1] = a.scale_log2 * sigma;
+      }
     }
   }
   __syncthreads();
   uint32_t* dst = a.qfrag + (size_t)unit * kFragWords;
-  for (int i = j; i < 4 * NT * 64; i += 128) dst[i] = fz[i];
-  if (j == 0) a.tickets[unit] = 0u;
+  for (int i = tid; i < 4 * NT * 64; i += 256) dst[i] = fz[i];
+  if (tid == 0) a.tickets[unit] = 0u;
 }
 
 // ---------------------------------------------------------------------------------
-struct WarpMerge {  // per consumer warp, per head
-  float m[4][8], l[4][8], bias[4][8];
+struct Merge {  // per pseudo-warp (0..3 quantized path, 4..7 window path) and head
+  float m[8][8], l[8][8], bias[8][8];
 };
 
 template <int BITS, int G>
-__global__ void __launch_bounds__(kThreads) decode_main_kernel(const DecodeArgs a) {
+struct Shared {
+  static constexpr int kStages = Cfg<BITS>::NSTAGE * Cfg<BITS>::STAGE;
+  static constexpr int kPv = kConsumers * G * kHeadDim * 4;  // [4][G][128] fp32, reuses the stages
+  static constexpr int kArena = kStages > kPv ? kStages : kPv;
+  static size_t bytes(int nitems) {
+    return (size_t)kArena + 2 * Cfg<BITS>::NSTAGE * 8 + sizeof(Merge) + (size_t)kPv + (size_t)nitems * G * 4;
+  }
+};
+
+// Per-warp online-softmax state of the quantized path.
+template <int NHS>
+struct QState {
+  float m[NHS], l[NHS], bias[NHS];
+  float o[8][4];
+  int kacc;
+};
+
+// One consumer warp's 32-position slice of a stage.  FULL: every position is in range.
+template <int BITS, int G, bool FULL>
+__device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, int tpos, int vlo, int vhi,
+                                      const uint32_t (&bq)[4][GCfg<G>::NT][2], const float (&Ah)[GCfg<G>::NHS],
+                                      const float (&Bh)[GCfg<G>::NHS], const bool (&hvalid)[GCfg<G>::NHS],
+                                      QState<GCfg<G>::NHS>& s, int g, int t4) {
+  constexpr int NT = GCfg<G>::NT, NHS = GCfg<G>::NHS;
+  constexpr int CB = 16 * BITS;
+  const uint8_t* kc = st;
+  const uint8_t* vc = st + kTileTokens * CB;
+  const uint32_t* kpar = reinterpret_cast<const uint32_t*>(st + 2 * kTileTokens * CB);
+  const uint32_t* vpar = kpar + kTileTokens;
+
+  // ---- QK^T over two 16-position m-tiles: rows base + 16i + g (+8)
+  int acc[2][NT][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[i][nt][0] = acc[i][nt][1] = acc[i][nt][2] = acc[i][nt][3] = 0;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int r0 = base + 16 * i + g, r1 = r0 + 8;
+    if (BITS == 2) {
+      const uint2 ka = *reinterpret_cast<const uint2*>(kc + r0 * CB + 8 * t4);
+      const uint2 kb = *reinterpret_cast<const uint2*>(kc + r1 * CB + 8 * t4);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t mk = 0x03030303u << (2 * j);
+        const uint32_t A[4] = {ka.x & mk, kb.x & mk, ka.y & mk, kb.y & mk};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[i][nt], A, bq[j][nt]);
+      }
+    } else {
+      const uint4 ka = *reinterpret_cast<const uint4*>(kc + r0 * CB + 16 * t4);
+      const uint4 kb = *reinterpret_cast<const uint4*>(kc + r1 * CB + 16 * t4);
+      const uint32_t kaw[4] = {ka.x, ka.y, ka.z, ka.w};
+      const uint32_t kbw[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t mk = (j & 1) ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
+        const int wa = 2 * (j >> 1);
+        const uint32_t A[4] = {kaw[wa] & mk, kbw[wa] & mk, kaw[wa + 1] & mk, kbw[wa + 1] & mk};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[i][nt], A, bq[j][nt]);
+      }
+    }
+  }
+
+  // ---- logits (base 2) of this lane's 4 positions: rows base + 16i + g + 8u
+  float2 ksz[2][2], vsz[2][2];
+  bool val[2][2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = base + 16 * i + g + 8 * u;
+      ksz[i][u] = __half22float2(u32_as_h2(kpar[r]));
+      vsz[i][u] = __half22float2(u32_as_h2(vpar[r]));
+      val[i][u] = FULL || (tpos + r >= vlo && tpos + r < vhi);
+    }
+  float x[2][2][NHS], alpha[NHS];
+  bool grow = false;
+#pragma unroll
+  for (int hs = 0; hs < NHS; ++hs) {
+    float mx = -CUDART_INF_F;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        // q'.c / sigma = sum_l 256^l D_l; pairs of limbs combine exactly in int32
+        const int d01 = acc[i][hs][2 * u] + 256 * acc[i][hs][2 * u + 1];
+        const int d23 = acc[i][NHS + hs][2 * u] + 256 * acc[i][NHS + hs][2 * u + 1];
+        const float f = fmaf(65536.0f, (float)d23, (float)d01);
+        const float xv = fmaf(Bh[hs] * ksz[i][u].x, f, Ah[hs] * ksz[i][u].y);
+        x[i][u][hs] = (val[i][u] && hvalid[hs]) ? xv : -CUDART_INF_F;
+        mx = fmaxf(mx, x[i][u][hs]);
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    const float mn = fmaxf(s.m[hs], mx);
+    alpha[hs] = 1.0f;
+    if (mn > s.m[hs]) {
+      alpha[hs] = exp2f(s.m[hs] - mn);
+      grow = true;
+    }
+    s.m[hs] = mn;
+  }
+  // ---- p*s enters the PV product scaled by 2^kacc: the largest weight of a slice sits near
+  // 2^13..2^14 and small weights stay in fp16's normal range; kacc only decreases
+  float smax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int u = 0; u < 2; ++u) smax = fmaxf(smax, val[i][u] ? vsz[i][u].x : 0.f);
+  smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
+  smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
+  smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
+  float fk = 1.0f;
+  if (smax > 0.f) {
+    const int k = 13 - (((__float_as_int(smax) >> 23) & 255) - 127);  // smax * 2^k < 2^14
+    if (k < s.kacc) {  // warp-uniform
+      fk = pow2i(max(k - s.kacc, -126));
+      s.kacc = k;
+    }
+  }
+  if (__any_sync(0xffffffffu, grow) || fk != 1.0f) {
+    // o columns are heads 2t4, 2t4+1 (lo parts in 4..7 when g <= 4); their alpha lives in
+    // lanes 4g + (head & 3)
+    float ac0 = __shfl_sync(0xffffffffu, alpha[0], 4 * g + ((2 * t4) & 3));
+    float ac1 = __shfl_sync(0xffffffffu, alpha[0], 4 * g + ((2 * t4 + 1) & 3));
+    if (NHS == 2) {
+      const float bc0 = __shfl_sync(0xffffffffu, alpha[NHS - 1], 4 * g + ((2 * t4) & 3));
+      const float bc1 = __shfl_sync(0xffffffffu, alpha[NHS - 1], 4 * g + ((2 * t4 + 1) & 3));
+      if (t4 >= 2) {
+        ac0 = bc0;
+        ac1 = bc1;
+      }
+    }
+    ac0 *= fk;
+    ac1 *= fk;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      s.o[mt][0] *= ac0;
+      s.o[mt][1] *= ac1;
+      s.o[mt][2] *= ac0;
+      s.o[mt][3] *= ac1;
+    }
+#pragma unroll
+    for (int hs = 0; hs < NHS; ++hs) {
+      s.l[hs] *= alpha[hs];
+      s.bias[hs] *= alpha[hs];
+    }
+  }
+  const float wscale = pow2i(s.kacc);
+
+  // ---- PV, one 16-position k-block per m-tile pair i
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    // p*s as an fp16 pair hi + lo (hi = fp16(p*s), lo = fp16(p*s - hi)): the PV product
+    // then carries ~22 bits of p*s, matching the fp32 l it is normalised by
+    uint32_t pk[NHS], pkl[NHS];
+#pragma unroll
+    for (int hs = 0; hs < NHS; ++hs) {
+      const float ms = s.m[hs] == -CUDART_INF_F ? 0.f : s.m[hs];
+      const float p0 = exp2f(x[i][0][hs] - ms);
+      const float p1 = exp2f(x[i][1][hs] - ms);
+      s.l[hs] += p0 + p1;
+      // masked positions may hold any bits in (s, z): never multiply them
+      const float w0 = val[i][0] ? p0 * vsz[i][0].x * wscale : 0.f;
+      const float w1 = val[i][1] ? p1 * vsz[i][1].x * wscale : 0.f;
+      const float b0 = val[i][0] ? p0 * vsz[i][0].y : 0.f;
+      const float b1 = val[i][1] ? p1 * vsz[i][1].y : 0.f;
+      s.bias[hs] += b0 + b1;
+      const __half2 hi2 = __floats2half2_rn(w0, w1);
+      const float2 hif = __half22float2(hi2);
+      pk[hs] = h2_as_u32(hi2);
+      pkl[hs] = h2_as_u32(__floats2half2_rn(w0 - hif.x, w1 - hif.y));
+    }
+    // B operand: rows k=2t4,2t4+1 <- positions t4, t4+8; k=2t4+8,+9 <- t4+4, t4+12 (of the
+    // block); column n = head n (n < 4 or g == 8); for g <= 4 columns 4..7 carry lo parts
+    const int src0 = 4 * t4 + (g & 3), src1 = 4 * (t4 + 4) + (g & 3);
+    uint32_t pb[2], pbl[2];
+    {
+      const uint32_t h0 = __shfl_sync(0xffffffffu, pk[0], src0);
+      const uint32_t h1 = __shfl_sync(0xffffffffu, pk[0], src1);
+      const uint32_t l0 = __shfl_sync(0xffffffffu, pkl[0], src0);
+      const uint32_t l1 = __shfl_sync(0xffffffffu, pkl[0], src1);
+      if (NHS == 2) {
+        const uint32_t h2 = __shfl_sync(0xffffffffu, pk[NHS - 1], src0);
+        const uint32_t h3 = __shfl_sync(0xffffffffu, pk[NHS - 1], src1);
+        const uint32_t l2 = __shfl_sync(0xffffffffu, pkl[NHS - 1], src0);
+        const uint32_t l3 = __shfl_sync(0xffffffffu, pkl[NHS - 1], src1);
+        pb[0] = g < 4 ? h0 : h2;
+        pb[1] = g < 4 ? h1 : h3;
+        pbl[0] = g < 4 ? l0 : l2;
+        pbl[1] = g < 4 ? l1 : l3;
+      } else {
+        pb[0] = g < 4 ? h0 : l0;
+        pb[1] = g < 4 ? h1 : l1;
+        pbl[0] = pbl[1] = 0u;
+      }
+    }
+    const int ta = base + 16 * i + t4;
+    if (BITS == 2) {
+      const uint32_t* vw = reinterpret_cast<const uint32_t*>(vc);
+      const uint32_t w0 = vw[ta * 8 + g], w1 = vw[(ta + 8) * 8 + g];
+      const uint32_t w2 = vw[(ta + 4) * 8 + g], w3 = vw[(ta + 12) * 8 + g];
+      const uint32_t xl1 = __byte_perm(w0, w1, 0x5410), xh1 = __byte_perm(w0, w1, 0x7632);
+      const uint32_t xl2 = __byte_perm(w2, w3, 0x5410), xh2 = __byte_perm(w2, w3, 0x7632);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const uint32_t A[4] = {vcode2(xl1, mt), vcode2(xh1, mt), vcode2(xl2, mt), vcode2(xh2, mt)};
+        mma_f16(s.o[mt], A, pb);
+        if (NHS == 2) mma_f16(s.o[mt], A, pbl);
+      }
+    } else {
+      const uint2* vw = reinterpret_cast<const uint2*>(vc);
+      const uint2 u0 = vw[ta * 8 + g], u1 = vw[(ta + 8) * 8 + g];
+      const uint2 u2 = vw[(ta + 4) * 8 + g], u3 = vw[(ta + 12) * 8 + g];
+#pragma unroll
+      for (int ws = 0; ws < 2; ++ws) {
+        const uint32_t a0 = ws ? u0.y : u0.x, a1 = ws ? u1.y : u1.x;
+        const uint32_t a2 = ws ? u2.y : u2.x, a3 = ws ? u3.y : u3.x;
+        const uint32_t xl1 = __byte_perm(a0, a1, 0x5410), xh1 = __byte_perm(a0, a1, 0x7632);
+        const uint32_t xl2 = __byte_perm(a2, a3, 0x5410), xh2 = __byte_perm(a2, a3, 0x7632);
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi) {
+          const uint32_t A[4] = {vcode4(xl1, mi), vcode4(xh1, mi), vcode4(xl2, mi), vcode4(xh2, mi)};
+          mma_f16(s.o[4 * ws + mi], A, pb);
+          if (NHS == 2) mma_f16(s.o[4 * ws + mi], A, pbl);
+        }
+      }
+    }
+  }
+}
+
+// fp16 window positions [wbeg, wend) of a unit, positions wbeg + warp, + 4, ...: exact
+// scalar path (lane = 4 dims), written to the window pseudo-warp slots of the merge area.
+template <int G>
+__device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, int n_sink, int r0, int warp,
+                             int lane, Merge* mg, float* wpv) {
+  float qv[G][4];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    const float4 t = *reinterpret_cast<const float4*>(a.qprime + ((size_t)unit * G + hh) * kHeadDim + 4 * lane);
+    qv[hh][0] = t.x;
+    qv[hh][1] = t.y;
+    qv[hh][2] = t.z;
+    qv[hh][3] = t.w;
+  }
+  float m[G], l[G], o[G][4];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    m[hh] = -CUDART_INF_F;
+    l[hh] = 0.f;
+    o[hh][0] = o[hh][1] = o[hh][2] = o[hh][3] = 0.f;
+  }
+  for (int it = wbeg + warp; it < wend; it += kConsumers) {
+    const __half *kr, *vr;
+    if (it < n_sink) {
+      kr = a.k_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
+      vr = a.v_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
+    } else {
+      const int p = r0 + (it - n_sink);
+      kr = a.k_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
+      vr = a.v_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
+    }
+    const uint2 kraw = *reinterpret_cast<const uint2*>(kr + 4 * lane);
+    const uint2 vraw = *reinterpret_cast<const uint2*>(vr + 4 * lane);
+    const float2 k01 = __half22float2(u32_as_h2(kraw.x)), k23 = __half22float2(u32_as_h2(kraw.y));
+    const float2 v01 = __half22float2(u32_as_h2(vraw.x)), v23 = __half22float2(u32_as_h2(vraw.y));
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      float xx = qv[hh][0] * k01.x;
+      xx = fmaf(qv[hh][1], k01.y, xx);
+      xx = fmaf(qv[hh][2], k23.x, xx);
+      xx = fmaf(qv[hh][3], k23.y, xx);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) xx += __shfl_xor_sync(0xffffffffu, xx, off);
+      const float mn = fmaxf(m[hh], xx);
+      const float al = exp2f(m[hh] - mn);
+      const float p = exp2f(xx - mn);
+      l[hh] = fmaf(l[hh], al, p);
+      o[hh][0] = fmaf(o[hh][0], al, p * v01.x);
+      o[hh][1] = fmaf(o[hh][1], al, p * v01.y);
+      o[hh][2] = fmaf(o[hh][2], al, p * v23.x);
+      o[hh][3] = fmaf(o[hh][3], al, p * v23.y);
+      m[hh] = mn;
+    }
+  }
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    if (lane == 0) {
+      mg->m[kConsumers + warp][hh] = m[hh];
+      mg->l[kConsumers + warp][hh] = l[hh];
+      mg->bias[kConsumers + warp][hh] = 0.f;
+    }
+    float* dst = wpv + ((size_t)warp * G + hh) * kHeadDim + 4 * lane;
+    dst[0] = o[hh][0];
+    dst[1] = o[hh][1];
+    dst[2] = o[hh][2];
+    dst[3] = o[hh][3];
+  }
+}
+
+template <int BITS, int G>
+__global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_kernel(const DecodeArgs a) {
   using C = Cfg<BITS>;
+  using SM = Shared<BITS, G>;
   constexpr int NT = GCfg<G>::NT, NHS = GCfg<G>::NHS;
   constexpr int CB = C::CB;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::NSTAGE * C::STAGE);
+  float* pv = reinterpret_cast<float*>(smem);  // [4][G][128], written once the stages are drained
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kArena);
   uint64_t* empty = full + C::NSTAGE;
-  WarpMerge* wm = reinterpret_cast<WarpMerge*>(empty + C::NSTAGE);
-  float* pv = reinterpret_cast<float*>(wm + 1);          // [4][G][128]
-  float* wts = pv + 4 * G * kHeadDim;                     // [nitems][G] (last item only)
+  Merge* mg = reinterpret_cast<Merge*>(empty + C::NSTAGE);
+  float* wpv = reinterpret_cast<float*>(mg + 1);   // window path [4][G][128]
+  float* wts = wpv + kConsumers * G * kHeadDim;    // [nitems][G] (last item only)
   __shared__ uint32_t s_last;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t4 = lane & 3;
   const int unit = blockIdx.y, item = blockIdx.x;
-  const int nitems = a.n_split + 1;
+  const int nitems = a.n_split;
   int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
   if (S < 0 || S > a.cap_alloc || Sq < 0 || Sq > S) {  // never read outside the buffers
     if (tid == 0 && item == 0) atomicOr(a.status, kStatusBadState);
     S = 0;
     Sq = 0;
   }
+  // quantized positions of this item: [lo, hi) within [qlo, qhi)
+  const int qlo = a.s_sink;
+  const int qhi = Sq > a.s_sink ? Sq : a.s_sink;
+  const int ibeg = item * a.split_tokens, iend = ibeg + a.split_tokens;
+  const int lo = max(ibeg, qlo), hi = min(iend, qhi);
+  const int tile0 = lo < hi ? (lo / kTileTokens) * kTileTokens : 0;
+  const int ntiles = lo < hi ? (hi - tile0 + kTileTokens - 1) / kTileTokens : 0;
+  // fp16 window positions of the unit: sink [0, n_sink) then recent [r0, S); this item's share
+  const int n_sink = min(a.s_sink, S);
+  const int r0 = max(Sq, a.s_sink);
+  const int n_win = n_sink + (S > r0 ? S - r0 : 0);
+  const int wper = (n_win + nitems - 1) / nitems;
+  const int wbeg = min(item * wper, n_win), wend = min(wbeg + wper, n_win);
 
-  if (item == 0) {
-    // ======================= fp16 windows: sink [0, n_sink) and recent [r0, S)
-    if (warp < 4) {
-      const int n_sink = min(a.s_sink, S);
-      const int r0 = max(Sq, a.s_sink);
-      const int n_rec = S > r0 ? S - r0 : 0;
-      float qv[G][4];
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float4 t = *reinterpret_cast<const float4*>(a.qprime + ((size_t)unit * G + hh) * kHeadDim + 4 * lane);
-        qv[hh][0] = t.x; qv[hh][1] = t.y; qv[hh][2] = t.z; qv[hh][3] = t.w;
-      }
-      float m[G], l[G], o[G][4];
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        m[hh] = -CUDART_INF_F;
-        l[hh] = 0.f;
-        o[hh][0] = o[hh][1] = o[hh][2] = o[hh][3] = 0.f;
-      }
-      for (int it = warp; it < n_sink + n_rec; it += 4) {
-        const __half *kr, *vr;
-        if (it < n_sink) {
-          kr = a.k_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
-          vr = a.v_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
-        } else {
-          const int p = r0 + (it - n_sink);
-          kr = a.k_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
-          vr = a.v_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
-        }
-        const uint2 kraw = *reinterpret_cast<const uint2*>(kr + 4 * lane);
-        const uint2 vraw = *reinterpret_cast<const uint2*>(vr + 4 * lane);
-        const float2 k01 = __half22float2(u32_as_h2(kraw.x)), k23 = __half22float2(u32_as_h2(kraw.y));
-        const float2 v01 = __half22float2(u32_as_h2(vraw.x)), v23 = __half22float2(u32_as_h2(vraw.y));
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          float x = qv[hh][0] * k01.x;
-          x = fmaf(qv[hh][1], k01.y, x);
-          x = fmaf(qv[hh][2], k23.x, x);
-          x = fmaf(qv[hh][3], k23.y, x);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-          const float mn = fmaxf(m[hh], x);
-          const float alpha = exp2f(m[hh] - mn);
-          const float p = exp2f(x - mn);
-          l[hh] = fmaf(l[hh], alpha, p);
-          o[hh][0] = fmaf(o[hh][0], alpha, p * v01.x);
-          o[hh][1] = fmaf(o[hh][1], alpha, p * v01.y);
-          o[hh][2] = fmaf(o[hh][2], alpha, p * v23.x);
-          o[hh][3] = fmaf(o[hh][3], alpha, p * v23.y);
-          m[hh] = mn;
-        }
-      }
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        if (lane == 0) {
-          wm->m[warp][hh] = m[hh];
-          wm->l[warp][hh] = l[hh];
-          wm->bias[warp][hh] = 0.f;
-        }
-        float* dst = pv + ((size_t)warp * G + hh) * kHeadDim + 4 * lane;
-        dst[0] = o[hh][0]; dst[1] = o[hh][1]; dst[2] = o[hh][2]; dst[3] = o[hh][3];
-      }
+  if (tid == 0) {
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers);
     }
-  } else {
-    // ======================= quantized positions [qlo, qhi) within this item's range
-    const int qlo = a.s_sink;
-    const int qhi = Sq > a.s_sink ? Sq : a.s_sink;
-    const int ibeg = (item - 1) * a.split_tokens;
-    const int lo = max(ibeg, qlo), hi = min(ibeg + a.split_tokens, qhi);
-    const int tile0 = lo < hi ? (lo / kTileTokens) * kTileTokens : 0;
-    const int ntiles = lo < hi ? (hi - tile0 + kTileTokens - 1) / kTileTokens : 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
 
-    if (tid == 0) {
-      for (int s = 0; s < C::NSTAGE; ++s) {
-        mbar_init(&full[s], 1);
-        mbar_init(&empty[s], 4);
-      }
-      fence_mbar_init();
-    }
-    __syncthreads();
+  QState<NHS> qs;
+  bool hvalid[NHS];
+#pragma unroll
+  for (int hs = 0; hs < NHS; ++hs) {
+    hvalid[hs] = t4 + 4 * hs < G;
+    qs.m[hs] = -CUDART_INF_F;
+    qs.l[hs] = 0.f;
+    qs.bias[hs] = 0.f;
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) qs.o[mt][0] = qs.o[mt][1] = qs.o[mt][2] = qs.o[mt][3] = 0.f;
+  qs.kacc = 64;
 
-    if (warp == 4) {
-      // ---------------- producer
-      if (lane == 0 && ntiles > 0) {
-        int issued = 0;
-        for (int t = 0; t < ntiles; ++t) {
-          const int s = t % C::NSTAGE;
-          if (t >= C::NSTAGE && !mbar_wait(&empty[s], ((t / C::NSTAGE) - 1) & 1, a.status)) break;
-          uint8_t* st = stages + s * C::STAGE;
-          const size_t rec = (size_t)unit * a.cap_alloc + tile0 + (size_t)t * kTileTokens;
-          mbar_expect_tx(&full[s], C::STAGE);
-          bulk_g2s(st, a.k_codes + rec * CB, kTileTokens * CB, &full[s]);
-          bulk_g2s(st + kTileTokens * CB, a.v_codes + rec * CB, kTileTokens * CB, &full[s]);
-          bulk_g2s(st + 2 * kTileTokens * CB, a.k_params + rec, kTileTokens * 4, &full[s]);
-          bulk_g2s(st + 2 * kTileTokens * CB + kTileTokens * 4, a.v_params + rec, kTileTokens * 4, &full[s]);
-          issued = t + 1;
-        }
-        // every issued copy has landed before the CTA may leave
-        for (int t = max(0, issued - C::NSTAGE); t < issued; ++t)
-          mbar_wait(&full[t % C::NSTAGE], (t / C::NSTAGE) & 1, a.status);
-      }
-    } else {
-      // ---------------- consumers
-      uint32_t bq[4][NT][2];
-      {
-        const uint2* src = reinterpret_cast<const uint2*>(a.qfrag + (size_t)unit * kFragWords);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const uint2 u = src[(j * NT + nt) * 32 + lane];
-            bq[j][nt][0] = u.x;
-            bq[j][nt][1] = u.y;
-          }
-      }
-      float Ah[NHS], Bh[NHS], m_run[NHS], l_run[NHS], bias[NHS];
-      bool hvalid[NHS];
-#pragma unroll
-      for (int hs = 0; hs < NHS; ++hs) {
-        const int hh = t4 + 4 * hs;
-        hvalid[hs] = hh < G;
-        Ah[hs] = hvalid[hs] ? a.hconst[((size_t)unit * 8 + hh) * 2 + 0] : 0.f;
-        Bh[hs] = hvalid[hs] ? a.hconst[((size_t)unit * 8 + hh) * 2 + 1] : 0.f;
-        m_run[hs] = -CUDART_INF_F;
-        l_run[hs] = 0.f;
-        bias[hs] = 0.f;
-      }
-      float o[8][4];
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-      // p*s enters the PV product scaled by 2^kacc so that the largest weight of a slice sits
-      // near 2^13..2^14 and small weights stay in fp16's normal range; kacc only decreases
-      int kacc = 64;
-
-      const int r0 = 16 * warp + g, r1 = r0 + 8;
+  if (warp == kConsumers) {
+    // ---------------- producer: streams the item's tiles; needs nothing from the prologue
+    if (lane == 0 && ntiles > 0) {
+      int issued = 0;
       for (int t = 0; t < ntiles; ++t) {
         const int s = t % C::NSTAGE;
-        if (!mbar_wait(&full[s], (t / C::NSTAGE) & 1, a.status)) break;
-        const uint8_t* st = stages + s * C::STAGE;
-        const uint8_t* kc = st;
-        const uint8_t* vc = st + kTileTokens * CB;
-        const uint32_t* kpar = reinterpret_cast<const uint32_t*>(st + 2 * kTileTokens * CB);
-        const uint32_t* vpar = kpar + kTileTokens;
-        const int tpos = tile0 + t * kTileTokens;
-
-        // ---- QK^T: exact integer dot products of codes with the query limbs
-        int acc[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
-        if (BITS == 2) {
-          const uint2 ka = *reinterpret_cast<const uint2*>(kc + r0 * CB + 8 * t4);
-          const uint2 kb = *reinterpret_cast<const uint2*>(kc + r1 * CB + 8 * t4);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t mk = 0x03030303u << (2 * j);
-            const uint32_t A[4] = {ka.x & mk, kb.x & mk, ka.y & mk, kb.y & mk};
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[nt], A, bq[j][nt]);
-          }
-        } else {
-          const uint4 ka = *reinterpret_cast<const uint4*>(kc + r0 * CB + 16 * t4);
-          const uint4 kb = *reinterpret_cast<const uint4*>(kc + r1 * CB + 16 * t4);
-          const uint32_t kaw[4] = {ka.x, ka.y, ka.z, ka.w};
-          const uint32_t kbw[4] = {kb.x, kb.y, kb.z, kb.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t mk = (j & 1) ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
-            const int wa = 2 * (j >> 1);
-            const uint32_t A[4] = {kaw[wa] & mk, kbw[wa] & mk, kaw[wa + 1] & mk, kbw[wa + 1] & mk};
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[nt], A, bq[j][nt]);
-          }
-        }
-
-        // ---- logits (base 2), rows r0 / r1
-        const float2 ksz0 = __half22float2(u32_as_h2(kpar[r0]));
-        const float2 ksz1 = __half22float2(u32_as_h2(kpar[r1]));
-        const float2 vsz0 = __half22float2(u32_as_h2(vpar[r0]));
-        const float2 vsz1 = __half22float2(u32_as_h2(vpar[r1]));
-        const bool val0 = (tpos + r0 >= qlo) && (tpos + r0 < qhi) && (tpos + r0 >= ibeg) &&
-                          (tpos + r0 < ibeg + a.split_tokens);
-        const bool val1 = (tpos + r1 >= qlo) && (tpos + r1 < qhi) && (tpos + r1 >= ibeg) &&
-                          (tpos + r1 < ibeg + a.split_tokens);
-        float x0[NHS], x1[NHS], alpha[NHS];
-        bool grow = false;
-#pragma unroll
-        for (int hs = 0; hs < NHS; ++hs) {
-          // q'.c / sigma = sum_l 256^l D_l; pairs of limbs combine exactly in int32
-          const int d01a = acc[hs][0] + 256 * acc[hs][1];
-          const int d01b = acc[hs][2] + 256 * acc[hs][3];
-          const int d23a = acc[NHS + hs][0] + 256 * acc[NHS + hs][1];
-          const int d23b = acc[NHS + hs][2] + 256 * acc[NHS + hs][3];
-          const float fa = fmaf(65536.0f, (float)d23a, (float)d01a);
-          const float fb = fmaf(65536.0f, (float)d23b, (float)d01b);
-          x0[hs] = (val0 && hvalid[hs]) ? fmaf(Bh[hs] * ksz0.x, fa, Ah[hs] * ksz0.y) : -CUDART_INF_F;
-          x1[hs] = (val1 && hvalid[hs]) ? fmaf(Bh[hs] * ksz1.x, fb, Ah[hs] * ksz1.y) : -CUDART_INF_F;
-          float mx = fmaxf(x0[hs], x1[hs]);
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-          const float mn = fmaxf(m_run[hs], mx);
-          alpha[hs] = 1.0f;
-          if (mn > m_run[hs]) {
-            alpha[hs] = exp2f(m_run[hs] - mn);
-            grow = true;
-          }
-          m_run[hs] = mn;
-        }
-        if (__any_sync(0xffffffffu, grow)) {
-          // o columns are heads 2t4, 2t4+1; their alpha lives in lanes 4g + (head & 3)
-          float ac0 = __shfl_sync(0xffffffffu, alpha[0], 4 * g + ((2 * t4) & 3));
-          float ac1 = __shfl_sync(0xffffffffu, alpha[0], 4 * g + ((2 * t4 + 1) & 3));
-          if (NHS == 2) {
-            const float bc0 = __shfl_sync(0xffffffffu, alpha[NHS - 1], 4 * g + ((2 * t4) & 3));
-            const float bc1 = __shfl_sync(0xffffffffu, alpha[NHS - 1], 4 * g + ((2 * t4 + 1) & 3));
-            if (t4 >= 2) {
-              ac0 = bc0;
-              ac1 = bc1;
-            }
-          }
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            o[mt][0] *= ac0;
-            o[mt][1] *= ac1;
-            o[mt][2] *= ac0;
-            o[mt][3] *= ac1;
-          }
-#pragma unroll
-          for (int hs = 0; hs < NHS; ++hs) {
-            l_run[hs] *= alpha[hs];
-            bias[hs] *= alpha[hs];
-          }
-        }
-        {
-          float smax = fmaxf(val0 ? vsz0.x : 0.f, val1 ? vsz1.x : 0.f);
-          smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
-          smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
-          smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
-          if (smax > 0.f) {
-            const int e = ((__float_as_int(smax) >> 23) & 255) - 127;  // smax < 2^(e+1)
-            const int k = 13 - e;
-            if (k < kacc) {  // warp-uniform
-              const float f = pow2i(max(k - kacc, -126));
-#pragma unroll
-              for (int mt = 0; mt < 8; ++mt) {
-                o[mt][0] *= f;
-                o[mt][1] *= f;
-                o[mt][2] *= f;
-                o[mt][3] *= f;
-              }
-              kacc = k;
-            }
-          }
-        }
-        const float wscale = pow2i(kacc);
-        // p*s as an fp16 pair hi + lo (hi = fp16(p*s), lo = fp16(p*s - hi)): the PV product
-        // then carries ~22 bits of p*s, matching the fp32 l it is normalised by
-        uint32_t pk[NHS], pkl[NHS];
-#pragma unroll
-        for (int hs = 0; hs < NHS; ++hs) {
-          const float ms = m_run[hs] == -CUDART_INF_F ? 0.f : m_run[hs];
-          const float p0 = exp2f(x0[hs] - ms);
-          const float p1 = exp2f(x1[hs] - ms);
-          l_run[hs] += p0 + p1;
-          // masked positions may hold any bits in (s, z): never multiply them
-          const float w0 = val0 ? p0 * vsz0.x * wscale : 0.f, w1 = val1 ? p1 * vsz1.x * wscale : 0.f;
-          const float b0 = val0 ? p0 * vsz0.y : 0.f, b1 = val1 ? p1 * vsz1.y : 0.f;
-          bias[hs] += b0 + b1;
-          const __half2 hi2 = __floats2half2_rn(w0, w1);
-          const float2 hif = __half22float2(hi2);
-          pk[hs] = h2_as_u32(hi2);
-          pkl[hs] = h2_as_u32(__floats2half2_rn(w0 - hif.x, w1 - hif.y));
-        }
-        // ---- P (B operand of PV): rows k=2t4,2t4+1 <- tokens t4, t4+8; k=2t4+8,+9 <- t4+4, t4+12
-        // column n = head n (n < 4 or g == 8); for g <= 4, columns 4..7 carry the lo parts
-        const int src0 = 4 * t4 + (g & 3), src1 = 4 * (t4 + 4) + (g & 3);
-        uint32_t pb[2], pbl[2];
-        {
-          const uint32_t h0 = __shfl_sync(0xffffffffu, pk[0], src0);
-          const uint32_t h1 = __shfl_sync(0xffffffffu, pk[0], src1);
-          const uint32_t l0 = __shfl_sync(0xffffffffu, pkl[0], src0);
-          const uint32_t l1 = __shfl_sync(0xffffffffu, pkl[0], src1);
-          if (NHS == 2) {
-            const uint32_t h2 = __shfl_sync(0xffffffffu, pk[NHS - 1], src0);
-            const uint32_t h3 = __shfl_sync(0xffffffffu, pk[NHS - 1], src1);
-            const uint32_t l2 = __shfl_sync(0xffffffffu, pkl[NHS - 1], src0);
-            const uint32_t l3 = __shfl_sync(0xffffffffu, pkl[NHS - 1], src1);
-            pb[0] = g < 4 ? h0 : h2;
-            pb[1] = g < 4 ? h1 : h3;
-            pbl[0] = g < 4 ? l0 : l2;
-            pbl[1] = g < 4 ? l1 : l3;
-          } else {
-            pb[0] = g < 4 ? h0 : l0;
-            pb[1] = g < 4 ? h1 : l1;
-          }
-        }
-
-        // ---- PV: fp16-subnormal codes x fp16 (p*s)
-        const int ta = 16 * warp + t4;
-        if (BITS == 2) {
-          const uint32_t* vw = reinterpret_cast<const uint32_t*>(vc);
-          const uint32_t w0 = vw[(ta)*8 + g], w1 = vw[(ta + 8) * 8 + g];
-          const uint32_t w2 = vw[(ta + 4) * 8 + g], w3 = vw[(ta + 12) * 8 + g];
-          const uint32_t xl1 = __byte_perm(w0, w1, 0x5410), xh1 = __byte_perm(w0, w1, 0x7632);
-          const uint32_t xl2 = __byte_perm(w2, w3, 0x5410), xh2 = __byte_perm(w2, w3, 0x7632);
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            const uint32_t A[4] = {vcode2(xl1, mt), vcode2(xh1, mt), vcode2(xl2, mt), vcode2(xh2, mt)};
-            mma_f16(o[mt], A, pb);
-            if (NHS == 2) mma_f16(o[mt], A, pbl);
-          }
-        } else {
-          const uint2* vw = reinterpret_cast<const uint2*>(vc);
-          const uint2 u0 = vw[(ta)*8 + g], u1 = vw[(ta + 8) * 8 + g];
-          const uint2 u2 = vw[(ta + 4) * 8 + g], u3 = vw[(ta + 12) * 8 + g];
-#pragma unroll
-          for (int ws = 0; ws < 2; ++ws) {
-            const uint32_t a0 = ws ? u0.y : u0.x, a1 = ws ? u1.y : u1.x;
-            const uint32_t a2 = ws ? u2.y : u2.x, a3 = ws ? u3.y : u3.x;
-            const uint32_t xl1 = __byte_perm(a0, a1, 0x5410), xh1 = __byte_perm(a0, a1, 0x7632);
-            const uint32_t xl2 = __byte_perm(a2, a3, 0x5410), xh2 = __byte_perm(a2, a3, 0x7632);
-#pragma unroll
-            for (int mi = 0; mi < 4; ++mi) {
-              const uint32_t A[4] = {vcode4(xl1, mi), vcode4(xh1, mi), vcode4(xl2, mi), vcode4(xh2, mi)};
-              mma_f16(o[4 * ws + mi], A, pb);
-              if (NHS == 2) mma_f16(o[4 * ws + mi], A, pbl);
-            }
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        if (t >= C::NSTAGE && !mbar_wait(&empty[s], ((t / C::NSTAGE) - 1) & 1, a.status)) break;
+        uint8_t* st = stages + s * C::STAGE;
+        const size_t rec = (size_t)unit * a.cap_alloc + tile0 + (size_t)t * kTileTokens;
+        mbar_expect_tx(&full[s], C::STAGE);
+        bulk_g2s(st, a.k_codes + rec * CB, kTileTokens * CB, &full[s]);
+        bulk_g2s(st + kTileTokens * CB, a.v_codes + rec * CB, kTileTokens * CB, &full[s]);
+        bulk_g2s(st + 2 * kTileTokens * CB, a.k_params + rec, kTileTokens * 4, &full[s]);
+        bulk_g2s(st + 2 * kTileTokens * CB + kTileTokens * 4, a.v_params + rec, kTileTokens * 4, &full[s]);
+        issued = t + 1;
       }
+      // every issued copy has landed before the CTA may leave
+      for (int t = max(0, issued - C::NSTAGE); t < issued; ++t)
+        mbar_wait(&full[t % C::NSTAGE], (t / C::NSTAGE) & 1, a.status);
+    }
+  } else {
+    // ---------------- consumers
+    griddep_wait();  // q' fragments, constants and the ticket reset come from the prologue
+    // (a) this warp's share of the fp16 window, while the first tiles are in flight
+    window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, mg, wpv);
+    // (b) quantized positions
+    uint32_t bq[4][NT][2];
+    {
+      const uint2* src = reinterpret_cast<const uint2*>(a.qfrag + (size_t)unit * kFragWords);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint2 u = src[(j * NT + nt) * 32 + lane];
+          bq[j][nt][0] = u.x;
+          bq[j][nt][1] = u.y;
+        }
+    }
+    float Ah[NHS], Bh[NHS];
+#pragma unroll
+    for (int hs = 0; hs < NHS; ++hs) {
+      const int hh = t4 + 4 * hs;
+      Ah[hs] = hvalid[hs] ? a.hconst[((size_t)unit * 8 + hh) * 2 + 0] : 0.f;
+      Bh[hs] = hvalid[hs] ? a.hconst[((size_t)unit * 8 + hh) * 2 + 1] : 0.f;
+    }
+    const int base = kSlice * warp;
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t % C::NSTAGE;
+      if (!mbar_wait(&full[s], (t / C::NSTAGE) & 1, a.status)) break;
+      const uint8_t* st = stages + s * C::STAGE;
+      const int tpos = tile0 + t * kTileTokens;
+      if (tpos + base >= lo && tpos + base + kSlice <= hi)
+        slice<BITS, G, true>(st, base, tpos, lo, hi, bq, Ah, Bh, hvalid, qs, g, t4);
+      else if (tpos + base + kSlice > lo && tpos + base < hi)
+        slice<BITS, G, false>(st, base, tpos, lo, hi, bq, Ah, Bh, hvalid, qs, g, t4);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // l and bias summed over the 8 lane groups
+#pragma unroll
+    for (int hs = 0; hs < NHS; ++hs) {
+      float lv = qs.l[hs], bv = qs.bias[hs];
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        lv += __shfl_xor_sync(0xffffffffu, lv, off);
+        bv += __shfl_xor_sync(0xffffffffu, bv, off);
+      }
+      if (g == 0 && hvalid[hs]) {
+        mg->m[warp][t4 + 4 * hs] = qs.m[hs];
+        mg->l[warp][t4 + 4 * hs] = lv;
+        mg->bias[warp][t4 + 4 * hs] = bv;
+      }
+    }
+    if (NHS == 1) {  // columns 4..7 (lanes t4 = 2, 3) hold the lo parts of heads 0..3
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) qs.o[mt][c] += __shfl_down_sync(0xffffffffu, qs.o[mt][c], 2);
+    }
+  }
+  __syncthreads();  // every stage consumed and every copy landed: pv may reuse the stages
 
-      // ---- per-warp results: l, bias summed over the 8 lane groups
+  if (warp < kConsumers) {
 #pragma unroll
-      for (int hs = 0; hs < NHS; ++hs) {
-        float lv = l_run[hs], bv = bias[hs];
+    for (int mt = 0; mt < 8; ++mt) {
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          lv += __shfl_xor_sync(0xffffffffu, lv, off);
-          bv += __shfl_xor_sync(0xffffffffu, bv, off);
-        }
-        if (g == 0 && hvalid[hs]) {
-          wm->m[warp][t4 + 4 * hs] = m_run[hs];
-          wm->l[warp][t4 + 4 * hs] = lv;
-          wm->bias[warp][t4 + 4 * hs] = bv;
-        }
-      }
-      if (NHS == 1) {  // columns 4..7 (lanes t4 = 2, 3) hold the lo parts of heads 0..3
+      for (int hi2 = 0; hi2 < 2; ++hi2) {
+        int dim, l2s;
+        value_row<BITS>(mt, g, hi2, dim, l2s);
+        const float unscale = pow2i(24 - l2s - qs.kacc);
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) o[mt][c] += __shfl_down_sync(0xffffffffu, o[mt][c], 2);
-      }
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-#pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-          int dim, l2s;
-          value_row<BITS>(mt, g, hi, dim, l2s);
-          const float unscale = pow2i(24 - l2s - kacc);
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int hh = 2 * t4 + c;
-            if (hh < G) pv[((size_t)warp * G + hh) * kHeadDim + dim] = o[mt][2 * hi + c] * unscale;
-          }
+        for (int c = 0; c < 2; ++c) {
+          const int hh = 2 * t4 + c;
+          if (hh < G) pv[((size_t)warp * G + hh) * kHeadDim + dim] = qs.o[mt][2 * hi2 + c] * unscale;
         }
       }
     }
   }
   __syncthreads();
 
-  // ======================= merge the 4 warps, write this item's partial
+  // ======================= merge the 8 pseudo-warps, write this item's partial
   float* part = a.partials + ((size_t)unit * nitems + item) * G * kPartStride;
   for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
     const int hh = idx / kHeadDim, d = idx % kHeadDim;
     float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, wm->m[w][hh]);
+    for (int w = 0; w < 2 * kConsumers; ++w) M = fmaxf(M, mg->m[w][hh]);
     float O = 0.f, L = 0.f;
     if (M != -CUDART_INF_F) {
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float e = exp2f(wm->m[w][hh] - M);
-        O = fmaf(e, pv[((size_t)w * G + hh) * kHeadDim + d] + wm->bias[w][hh], O);
-        L = fmaf(e, wm->l[w][hh], L);
+      for (int w = 0; w < 2 * kConsumers; ++w) {
+        const float e = exp2f(mg->m[w][hh] - M);
+        const float ov = w < kConsumers ? pv[((size_t)w * G + hh) * kHeadDim + d]
+                                        : wpv[((size_t)(w - kConsumers) * G + hh) * kHeadDim + d];
+        O = fmaf(e, ov + mg->bias[w][hh], O);
+        L = fmaf(e, mg->l[w][hh], L);
       }
     }
     part[hh * kPartStride + 4 + d] = O;
@@ -673,24 +772,32 @@ __global__ void __launch_bounds__(kThreads) decode_main_kernel(const DecodeArgs 
 }
 
 template <int BITS, int G>
-size_t main_smem_bytes(int nitems) {
-  using C = Cfg<BITS>;
-  return (size_t)C::NSTAGE * C::STAGE + 2 * C::NSTAGE * sizeof(uint64_t) + sizeof(WarpMerge) +
-         (size_t)4 * G * kHeadDim * sizeof(float) + (size_t)nitems * G * sizeof(float);
-}
-
-template <int BITS, int G>
 cudaError_t launch_decode_t(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
-  decode_prologue_kernel<BITS, G><<<d.units, 128, 0, st>>>(a);
+  decode_prologue_kernel<BITS, G><<<d.units, 256, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int nitems = d.n_split + 1;
-  const size_t smem = main_smem_bytes<BITS, G>(nitems);
-  e = ensure_smem_attr(decode_main_kernel<BITS, G>, (int)smem);
+  const size_t smem = Shared<BITS, G>::bytes(d.n_split);
+  e = ensure_smem_attr<decode_main_kernel<BITS, G>>((int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(nitems, d.units);
-  decode_main_kernel<BITS, G><<<grid, kThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  // programmatic dependent launch: the main kernel may start before the prologue ends; its
+  // consumers wait (griddepcontrol.wait) for the prologue's results, its producer does not
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(d.n_split, d.units);
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  e = cudaLaunchKernelEx(&lc, decode_main_kernel<BITS, G>, a);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    decode_main_kernel<BITS, G><<<lc.gridDim, kThreads, smem, st>>>(a);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 template <int BITS>

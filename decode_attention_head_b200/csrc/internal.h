@@ -9,9 +9,11 @@
 namespace wushkv {
 
 constexpr int kHeadDim = 128;
-constexpr int kTileTokens = 64;       // positions per decode pipeline stage (and cap_alloc granule)
+constexpr int kTileTokens = 128;      // positions per decode pipeline stage (and cap_alloc granule)
 constexpr int kB200SMs = 148;         // split policy sizes the decode grid for this many SMs
-constexpr int kDecodeCtasPerSM = 3;   // resident decode CTAs per SM the policy aims at
+// Resident decode CTAs per SM the split policy aims at (the kernel's launch bounds hold its
+// registers to this): 8 query heads per KV head need more registers than the others.
+constexpr int decode_ctas_per_sm(int group) { return group == 8 ? 3 : 4; }
 constexpr int kMaxSplits = 255;       // quantized work items per (sequence, KV head)
 
 struct Derived {
@@ -79,14 +81,15 @@ struct DecodeArgs {
 
 // Raise a kernel's dynamic shared-memory limit once per device (a function attribute,
 // not a stream operation, so it is kept out of the launch path and of graph capture).
-template <typename F>
-cudaError_t ensure_smem_attr(F* fn, int bytes) {
+// One flag set per kernel (the template argument is the kernel itself).
+template <auto Kernel>
+cudaError_t ensure_smem_attr(int bytes) {
   static int done[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 64 && done[dev] >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = bytes;
   return e;
 }
