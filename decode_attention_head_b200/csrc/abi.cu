@@ -63,10 +63,6 @@ int derive(const wushkv_config* cfg, Derived* d) {
   size_t off = 0;
   d->ws_tickets = off;
   off = round_up(off + U * 4, 256);
-  d->ws_qfrag = off;
-  off = round_up(off + U * 4 * 4 * 64 * 4, 256);
-  d->ws_hconst = off;
-  off = round_up(off + U * 8 * 2 * 4, 256);
   d->ws_qprime = off;
   off = round_up(off + U * g * kHeadDim * 4, 256);
   d->ws_partials = off;
@@ -225,8 +221,6 @@ extern "C" int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* 
   a.out_fp16 = out_fp16;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.tickets = reinterpret_cast<uint32_t*>(ws + d.ws_tickets);
-  a.qfrag = reinterpret_cast<uint32_t*>(ws + d.ws_qfrag);
-  a.hconst = reinterpret_cast<float*>(ws + d.ws_hconst);
   a.qprime = reinterpret_cast<float*>(ws + d.ws_qprime);
   a.partials = reinterpret_cast<float*>(ws + d.ws_partials);
   const cudaError_t e = launch_decode(d, cfg->bits, a, static_cast<cudaStream_t>(stream));

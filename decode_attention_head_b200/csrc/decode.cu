@@ -4,11 +4,12 @@
 // §4.4 fp16 sink / recent windows around the quantized middle region).
 //
 // Two launches per call:
-//  1. decode_prologue (one CTA per (sequence, KV head)): q'_j = T_K^{-T} q_j for its g
-//     query heads (fp32), q' re-expressed as a 31-bit fixed-point integer split into
-//     four signed 8-bit limbs laid out as mma.sync B fragments, and the per-unit
+//  1. decode_prologue (four CTAs per (sequence, KV head), a quarter of the dimensions
+//     each): q'_j = T_K^{-T} q_j for its g query heads in fp32, and the per-unit
 //     completion ticket reset.  It releases the main kernel at once (programmatic
-//     dependent launch), so the main kernel's KV stream starts while it runs.
+//     dependent launch), so the main kernel's KV stream starts while it runs; each
+//     consumer warp then re-expresses q' as a 31-bit fixed-point integer split into
+//     four signed 8-bit limbs, directly in the mma.sync B-fragment registers it needs.
 //  2. decode_main: grid (n_split, units).  Item s of a unit attends over positions
 //     [sL, (s+1)L) of the quantized region [S_sink, S_quant) and over its share of the
 //     unit's fp16 window positions (sink [0, S_sink) and recent [S_quant, S)).
@@ -27,12 +28,12 @@
 // 0x03030303 << 2j leaves, in each byte, one code times 4^j -- an exact u8 operand.
 // The key-side scale 4^j is divided out of the query's integer representation.  On
 // the value side, pairs of 16-bit code chunks (one per token) are shifted so that one
-// code sits at bits 6..9 of each half and masked: the half is then the fp16 subnormal
-// c * 2^(b-24) (b = 6 or 8, the code's lowest bit), an exact operand whose power-of-two
-// scale is undone once per output row.  Codes are kept high in the subnormal range on
-// purpose: the tensor core aligns a product by the operand's nominal exponent (-14 for
-// every subnormal), so each leading zero bit of a subnormal costs one bit of the
-// product's precision inside the MMA; at bits 6..9 at most 4 of 24 bits are lost.
+// code sits at bits 4..9 of each half and masked: the half is then the fp16 subnormal
+// c * 2^(b-24) (b = 4, 6 or 8, the code's lowest bit), an exact operand whose
+// power-of-two scale is undone once per output row.  Codes are kept high in the
+// subnormal range on purpose: the tensor core aligns a product by the operand's nominal
+// exponent (-14 for every subnormal), so each leading zero bit of a subnormal costs one
+// bit of the product's precision inside the MMA; at bits 4..9 at most 6 of 24 are lost.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -44,7 +45,6 @@ namespace wushkv {
 namespace {
 
 constexpr float kQMax = 1073741824.0f;  // |fixed-point query| <= 2^30; four signed 8-bit limbs hold +-2.1e9
-constexpr int kFragWords = 4 * 4 * 64;   // per unit: [kstep 4][n-tile <= 4][lane 32][2] words
 constexpr int kThreads = 160;            // 4 consumer warps + 1 producer warp
 constexpr int kConsumers = 4;
 constexpr int kSlice = 32;               // positions per consumer warp per stage
@@ -53,6 +53,12 @@ static_assert(kTileTokens == kConsumers * kSlice, "a stage holds one slice per c
 
 // 2^n as an fp32 bit pattern, exact for -126 <= n <= 127.
 __device__ __forceinline__ float pow2i(int n) { return __int_as_float((n + 127) << 23); }
+
+__device__ __forceinline__ float ex2(float x) {  // 2^x (hardware approximation, 2^-inf = 0)
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
@@ -99,8 +105,9 @@ __host__ __device__ __forceinline__ void key_slot(int dim, int& kstep, int& t4, 
 template <int BITS>
 __device__ __forceinline__ void value_row(int mt, int g, int hi, int& dim, int& log2scale) {
   if (BITS == 2) {
-    dim = 16 * g + 8 * hi + mt;               // code mt of the chunk
-    log2scale = (mt & 1) && mt != 7 ? 6 : 8;  // placed at bits 6..7 or 8..9
+    constexpr int kPos[8] = {4, 6, 4, 6, 8, 4, 6, 8};  // bit position code mt is moved to
+    dim = 16 * g + 8 * hi + mt;                        // code mt of the chunk
+    log2scale = kPos[mt];
   } else {
     const int ws = mt >> 2, mi = mt & 3;
     dim = 16 * g + 8 * ws + 4 * hi + mi;
@@ -110,15 +117,15 @@ __device__ __forceinline__ void value_row(int mt, int g, int hi, int& dim, int& 
 
 // One value-side A register: code `mt` of both 16-bit halves of x (2-bit codes).
 __device__ __forceinline__ uint32_t vcode2(uint32_t x, int mt) {
-  constexpr uint32_t M89 = 0x03000300u, M67 = 0x00C000C0u;
+  constexpr uint32_t M45 = 0x00300030u, M67 = 0x00C000C0u, M89 = 0x03000300u;
   switch (mt) {
-    case 0: return (x << 8) & M89;
+    case 0: return (x << 4) & M45;
     case 1: return (x << 4) & M67;
-    case 2: return (x << 4) & M89;
+    case 2: return x & M45;
     case 3: return x & M67;
     case 4: return x & M89;
-    case 5: return (x >> 4) & M67;
-    case 6: return (x >> 4) & M89;
+    case 5: return (x >> 6) & M45;
+    case 6: return (x >> 6) & M67;
     default: return (x >> 6) & M89;
   }
 }
@@ -135,100 +142,130 @@ __device__ __forceinline__ uint32_t vcode4(uint32_t x, int mi) {
 }
 
 // ---------------------------------------------------------------------------------
-// Prologue: 256 threads; thread (half, j) sums half of q'[j] = sum_i Tinv[i][j] q[i].
-template <int BITS, int G>
-__global__ void __launch_bounds__(256) decode_prologue_kernel(const DecodeArgs a) {
-  constexpr int NT = GCfg<G>::NT;
+// Prologue: CTA (unit, quarter c), 128 threads; thread (part, jj) sums 32 of the 128 terms
+// of q'[j] = sum_i Tinv[i][j] q[i] for j = 32c + jj.
+template <int G>
+__global__ void __launch_bounds__(128) decode_prologue_kernel(const DecodeArgs a) {
   __shared__ float qs[G][kHeadDim];
-  __shared__ float part[G][kHeadDim];
-  __shared__ uint32_t frag[4][NT][32][2];
-  __shared__ float red_max[G][4], red_sum[G][4];
+  __shared__ float part[4][G][32];
   griddep_launch();
-  const int unit = blockIdx.x;
+  const int unit = blockIdx.x, c = blockIdx.y;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
-  const int tid = threadIdx.x, j = tid & 127, half = tid >> 7;
-  const int warp = j >> 5, lane = j & 31;
-
-  for (int i = tid; i < G * kHeadDim; i += 256) {
-    const int hh = i / kHeadDim, c = i % kHeadDim;
-    qs[hh][c] = __half2float(a.q[((size_t)b * a.Hq + h * G + hh) * kHeadDim + c]);
+  const int tid = threadIdx.x, jj = tid & 31, pt = tid >> 5;
+  for (int i = tid; i < G * kHeadDim; i += 128) {
+    const int hh = i / kHeadDim, cc = i % kHeadDim;
+    qs[hh][cc] = __half2float(a.q[((size_t)b * a.Hq + h * G + hh) * kHeadDim + cc]);
   }
-  uint32_t* fz = &frag[0][0][0][0];
-  for (int i = tid; i < 4 * NT * 64; i += 256) fz[i] = 0u;
   __syncthreads();
-
+  const int j = 32 * c + jj;
+  const float* Ti = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim + (size_t)(32 * pt) * kHeadDim + j;
   float qp[G];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) qp[hh] = 0.f;
-  const float* Ti = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim + (size_t)(64 * half) * kHeadDim + j;
-  for (int i0 = 0; i0 < 64; i0 += 16) {
+#pragma unroll
+  for (int i0 = 0; i0 < 32; i0 += 16) {
     float t[16];
 #pragma unroll
     for (int u = 0; u < 16; ++u) t[u] = __ldg(Ti + (size_t)(i0 + u) * kHeadDim);
 #pragma unroll
     for (int u = 0; u < 16; ++u)
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) qp[hh] = fmaf(t[u], qs[hh][64 * half + i0 + u], qp[hh]);
+      for (int hh = 0; hh < G; ++hh) qp[hh] = fmaf(t[u], qs[hh][32 * pt + i0 + u], qp[hh]);
   }
-  if (half == 1) {
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) part[hh][j] = qp[hh];
-  }
+  for (int hh = 0; hh < G; ++hh) part[pt][hh][jj] = qp[hh];
   __syncthreads();
-  int kstep, t4, r, byte, l2s;
-  key_slot<BITS>(j, kstep, t4, r, byte, l2s);
-  const float inv_scale = 1.0f / float(1 << l2s);
-  if (half == 0) {
+  for (int i = tid; i < G * 32; i += 128) {
+    const int hh = i / 32, q = i % 32;
+    a.qprime[((size_t)unit * G + hh) * kHeadDim + 32 * c + q] =
+        (part[0][hh][q] + part[1][hh][q]) + (part[2][hh][q] + part[3][hh][q]);
+  }
+  if (c == 0 && tid == 0) a.tickets[unit] = 0u;
+}
+
+// The query-side B fragments of one lane, built in registers from q' (fp32, in global
+// memory): lane (g, t4) holds, for k-step j, n-tile nt and register r, four bytes = limb
+// l = 2*(nt / NHS) + (g & 1) of the fixed-point Q of head 4*(nt % NHS) + (g >> 1) at the
+// four dimensions key_slot maps (j, t4, r, byte) to.  Q_d = rint(q'_d / (sigma * scale_d)),
+// sigma = max_d |q'_d| / scale_d / 2^30 per head (scale_d = the power of two that masking
+// leaves on dimension d's codes).  Also returns, for the lane's logit head t4 + 4*hs, the
+// constants log2e*scale*sum(q') (zero-point term) and log2e*scale*sigma.
+template <int BITS, int G>
+__device__ __forceinline__ void build_query(const DecodeArgs& a, int unit, int g, int t4,
+                                            uint32_t (&bq)[4][GCfg<G>::NT][2], float (&Ah)[GCfg<G>::NHS],
+                                            float (&Bh)[GCfg<G>::NHS]) {
+  constexpr int NHS = GCfg<G>::NHS;
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      qp[hh] += part[hh][j];
-      a.qprime[((size_t)unit * G + hh) * kHeadDim + j] = qp[hh] * a.scale_log2;
-      float m = fabsf(qp[hh]) * inv_scale, s = qp[hh];
+  for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        s += __shfl_xor_sync(0xffffffffu, s, o);
+    for (int nt = 0; nt < GCfg<G>::NT; ++nt) bq[j][nt][0] = bq[j][nt][1] = 0u;
+#pragma unroll
+  for (int hs = 0; hs < NHS; ++hs) {
+    const int hh = 4 * hs + (g >> 1);
+    float qv[32];
+    if (hh < G) {
+      const float4* src = reinterpret_cast<const float4*>(a.qprime + ((size_t)unit * G + hh) * kHeadDim + 32 * t4);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const float4 f = src[v];
+        qv[4 * v] = f.x;
+        qv[4 * v + 1] = f.y;
+        qv[4 * v + 2] = f.z;
+        qv[4 * v + 3] = f.w;
       }
-      if (lane == 0) {
-        red_max[hh][warp] = m;
-        red_sum[hh][warp] = s;
-      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) qv[k] = 0.f;
     }
-  }
-  __syncthreads();
-  if (half == 0) {
-    uint8_t* fb = reinterpret_cast<uint8_t*>(&frag[0][0][0][0]);
+    // dimension 32*t4 + k: its masking scale 2^l2s(k)
+    float amax = 0.f, sum = 0.f;
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      const float amax = fmaxf(fmaxf(red_max[hh][0], red_max[hh][1]), fmaxf(red_max[hh][2], red_max[hh][3]));
-      const float sum = (red_sum[hh][0] + red_sum[hh][1]) + (red_sum[hh][2] + red_sum[hh][3]);
-      const float sigma = amax > 0.f ? amax / kQMax : 1.0f;
-      // balanced base-256 digits of Q, each in [-128, 127]
-      long long Q = __float2ll_rn(qp[hh] * inv_scale / sigma);
-      int limbs[4];
-#pragma unroll
-      for (int l = 0; l < 4; ++l) {
-        const long long d = ((Q + 128) & 255) - 128;
-        limbs[l] = (int)d;
-        Q = (Q - d) >> 8;
-      }
-#pragma unroll
-      for (int l = 0; l < 4; ++l) {
-        const int nt = (l >> 1) * GCfg<G>::NHS + (hh >> 2);
-        const int col = 2 * (hh & 3) + (l & 1);
-        const int ln = 4 * col + t4;
-        fb[(((kstep * NT + nt) * 32 + ln) * 2 + r) * 4 + byte] = static_cast<uint8_t>(limbs[l] & 255);
-      }
-      if (j == 0) {
-        a.hconst[((size_t)unit * 8 + hh) * 2 + 0] = a.scale_log2 * sum;
-        a.hconst[((size_t)unit * 8 + hh) * 2 + 1] = a.scale_log2 * sigma;
-      }
+    for (int k = 0; k < 32; ++k) {
+      const int l2s = BITS == 2 ? 2 * (k & 3) : 4 * (k & 1);
+      amax = fmaxf(amax, fabsf(qv[k]) * (1.0f / float(1 << l2s)));
+      sum += qv[k];
     }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    const float sigma = amax > 0.f ? amax / kQMax : 1.0f;
+    const float rs = 1.0f / sigma;
+    const int lp = g & 1;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      int j, r, i, l2s;
+      if (BITS == 2) {
+        r = k >> 4;
+        i = (k & 15) >> 2;
+        j = k & 3;
+        l2s = 2 * j;
+      } else {
+        const int wl = k >> 3;
+        r = wl & 1;
+        i = (k & 7) >> 1;
+        j = 2 * (wl >> 1) + (k & 1);
+        l2s = 4 * (k & 1);
+      }
+      const int Q = __float2int_rn(qv[k] * (rs / float(1 << l2s)));
+      // balanced base-256 digits, each in [-128, 127]
+      const int L0 = ((Q + 128) & 255) - 128;
+      const int Q1 = (Q - L0) >> 8;
+      const int L1 = ((Q1 + 128) & 255) - 128;
+      const int Q2 = (Q1 - L1) >> 8;
+      const int L2 = ((Q2 + 128) & 255) - 128;
+      const int L3 = (Q2 - L2) >> 8;
+      const uint32_t lo = (uint32_t)((lp ? L1 : L0) & 255), hi = (uint32_t)((lp ? L3 : L2) & 255);
+      bq[j][hs][r] |= lo << (8 * i);
+      bq[j][NHS + hs][r] |= hi << (8 * i);
+    }
+    // the lane's logit head is t4 + 4*hs: its totals live in lanes with g = 2*t4
+    const float sum_t = __shfl_sync(0xffffffffu, sum, 8 * t4);
+    const float sig_t = __shfl_sync(0xffffffffu, sigma, 8 * t4);
+    const bool ok = t4 + 4 * hs < G;
+    Ah[hs] = ok ? a.scale_log2 * sum_t : 0.f;
+    Bh[hs] = ok ? a.scale_log2 * sig_t : 0.f;
   }
-  __syncthreads();
-  uint32_t* dst = a.qfrag + (size_t)unit * kFragWords;
-  for (int i = tid; i < 4 * NT * 64; i += 256) dst[i] = fz[i];
-  if (tid == 0) a.tickets[unit] = 0u;
 }
 
 // ---------------------------------------------------------------------------------
@@ -252,6 +289,7 @@ struct QState {
   float m[NHS], l[NHS], bias[NHS];
   float o[8][4];
   int kacc;
+  float s_lim;
 };
 
 // One consumer warp's 32-position slice of a stage.  FULL: every position is in range.
@@ -337,27 +375,36 @@ __device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, 
     const float mn = fmaxf(s.m[hs], mx);
     alpha[hs] = 1.0f;
     if (mn > s.m[hs]) {
-      alpha[hs] = exp2f(s.m[hs] - mn);
+      alpha[hs] = ex2(s.m[hs] - mn);
       grow = true;
     }
     s.m[hs] = mn;
   }
-  // ---- p*s enters the PV product scaled by 2^kacc: the largest weight of a slice sits near
-  // 2^13..2^14 and small weights stay in fp16's normal range; kacc only decreases
-  float smax = 0.f;
+  // ---- p*s enters the PV product scaled by 2^kacc: the largest weight of a slice sits below
+  // 2^14 and small weights stay in fp16's normal range; kacc only decreases, and only a
+  // position whose s reaches s_lim = 2^(14 - kacc) forces a (warp-wide) recomputation
+  bool over = false;
 #pragma unroll
   for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int u = 0; u < 2; ++u) smax = fmaxf(smax, val[i][u] ? vsz[i][u].x : 0.f);
-  smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
-  smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
-  smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
+    for (int u = 0; u < 2; ++u) over |= val[i][u] && vsz[i][u].x >= s.s_lim;
   float fk = 1.0f;
-  if (smax > 0.f) {
-    const int k = 13 - (((__float_as_int(smax) >> 23) & 255) - 127);  // smax * 2^k < 2^14
-    if (k < s.kacc) {  // warp-uniform
-      fk = pow2i(max(k - s.kacc, -126));
-      s.kacc = k;
+  if (__any_sync(0xffffffffu, over)) {
+    float smax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) smax = fmaxf(smax, val[i][u] ? vsz[i][u].x : 0.f);
+    smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
+    smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
+    smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
+    if (smax > 0.f) {
+      const int k = 13 - (((__float_as_int(smax) >> 23) & 255) - 127);  // smax * 2^k < 2^14
+      if (k < s.kacc) {
+        fk = pow2i(max(k - s.kacc, -126));
+        s.kacc = k;
+        s.s_lim = pow2i(14 - k);
+      }
     }
   }
   if (__any_sync(0xffffffffu, grow) || fk != 1.0f) {
@@ -399,8 +446,8 @@ __device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, 
 #pragma unroll
     for (int hs = 0; hs < NHS; ++hs) {
       const float ms = s.m[hs] == -CUDART_INF_F ? 0.f : s.m[hs];
-      const float p0 = exp2f(x[i][0][hs] - ms);
-      const float p1 = exp2f(x[i][1][hs] - ms);
+      const float p0 = ex2(x[i][0][hs] - ms);
+      const float p1 = ex2(x[i][1][hs] - ms);
       s.l[hs] += p0 + p1;
       // masked positions may hold any bits in (s, z): never multiply them
       const float w0 = val[i][0] ? p0 * vsz[i][0].x * wscale : 0.f;
@@ -480,10 +527,10 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
     const float4 t = *reinterpret_cast<const float4*>(a.qprime + ((size_t)unit * G + hh) * kHeadDim + 4 * lane);
-    qv[hh][0] = t.x;
-    qv[hh][1] = t.y;
-    qv[hh][2] = t.z;
-    qv[hh][3] = t.w;
+    qv[hh][0] = t.x * a.scale_log2;
+    qv[hh][1] = t.y * a.scale_log2;
+    qv[hh][2] = t.z * a.scale_log2;
+    qv[hh][3] = t.w * a.scale_log2;
   }
   float m[G], l[G], o[G][4];
 #pragma unroll
@@ -492,20 +539,32 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
     l[hh] = 0.f;
     o[hh][0] = o[hh][1] = o[hh][2] = o[hh][3] = 0.f;
   }
-  for (int it = wbeg + warp; it < wend; it += kConsumers) {
-    const __half *kr, *vr;
-    if (it < n_sink) {
-      kr = a.k_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
-      vr = a.v_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
-    } else {
-      const int p = r0 + (it - n_sink);
-      kr = a.k_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
-      vr = a.v_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
+  constexpr int kBatch = 8;  // positions whose loads are all in flight before any math
+  for (int it0 = wbeg + warp; it0 < wend; it0 += kBatch * kConsumers) {
+    uint2 kraw[kBatch], vraw[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int it = it0 + u * kConsumers;
+      kraw[u] = vraw[u] = make_uint2(0u, 0u);
+      if (it < wend) {
+        const __half *kr, *vr;
+        if (it < n_sink) {
+          kr = a.k_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
+          vr = a.v_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
+        } else {
+          const int p = r0 + (it - n_sink);
+          kr = a.k_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
+          vr = a.v_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
+        }
+        kraw[u] = *reinterpret_cast<const uint2*>(kr + 4 * lane);
+        vraw[u] = *reinterpret_cast<const uint2*>(vr + 4 * lane);
+      }
     }
-    const uint2 kraw = *reinterpret_cast<const uint2*>(kr + 4 * lane);
-    const uint2 vraw = *reinterpret_cast<const uint2*>(vr + 4 * lane);
-    const float2 k01 = __half22float2(u32_as_h2(kraw.x)), k23 = __half22float2(u32_as_h2(kraw.y));
-    const float2 v01 = __half22float2(u32_as_h2(vraw.x)), v23 = __half22float2(u32_as_h2(vraw.y));
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+    if (it0 + u * kConsumers >= wend) break;
+    const float2 k01 = __half22float2(u32_as_h2(kraw[u].x)), k23 = __half22float2(u32_as_h2(kraw[u].y));
+    const float2 v01 = __half22float2(u32_as_h2(vraw[u].x)), v23 = __half22float2(u32_as_h2(vraw[u].y));
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
       float xx = qv[hh][0] * k01.x;
@@ -515,14 +574,15 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) xx += __shfl_xor_sync(0xffffffffu, xx, off);
       const float mn = fmaxf(m[hh], xx);
-      const float al = exp2f(m[hh] - mn);
-      const float p = exp2f(xx - mn);
+      const float al = ex2(m[hh] - mn);
+      const float p = ex2(xx - mn);
       l[hh] = fmaf(l[hh], al, p);
       o[hh][0] = fmaf(o[hh][0], al, p * v01.x);
       o[hh][1] = fmaf(o[hh][1], al, p * v01.y);
       o[hh][2] = fmaf(o[hh][2], al, p * v23.x);
       o[hh][3] = fmaf(o[hh][3], al, p * v23.y);
       m[hh] = mn;
+    }
     }
   }
 #pragma unroll
@@ -601,6 +661,7 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) qs.o[mt][0] = qs.o[mt][1] = qs.o[mt][2] = qs.o[mt][3] = 0.f;
   qs.kacc = 64;
+  qs.s_lim = 0.f;  // the first position with s > 0 sets kacc
 
   if (warp == kConsumers) {
     // ---------------- producer: streams the item's tiles; needs nothing from the prologue
@@ -629,24 +690,8 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, mg, wpv);
     // (b) quantized positions
     uint32_t bq[4][NT][2];
-    {
-      const uint2* src = reinterpret_cast<const uint2*>(a.qfrag + (size_t)unit * kFragWords);
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const uint2 u = src[(j * NT + nt) * 32 + lane];
-          bq[j][nt][0] = u.x;
-          bq[j][nt][1] = u.y;
-        }
-    }
     float Ah[NHS], Bh[NHS];
-#pragma unroll
-    for (int hs = 0; hs < NHS; ++hs) {
-      const int hh = t4 + 4 * hs;
-      Ah[hs] = hvalid[hs] ? a.hconst[((size_t)unit * 8 + hh) * 2 + 0] : 0.f;
-      Bh[hs] = hvalid[hs] ? a.hconst[((size_t)unit * 8 + hh) * 2 + 1] : 0.f;
-    }
+    build_query<BITS, G>(a, unit, g, t4, bq, Ah, Bh);
     const int base = kSlice * warp;
     for (int t = 0; t < ntiles; ++t) {
       const int s = t % C::NSTAGE;
@@ -773,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
 
 template <int BITS, int G>
 cudaError_t launch_decode_t(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
-  decode_prologue_kernel<BITS, G><<<d.units, 256, 0, st>>>(a);
+  decode_prologue_kernel<G><<<dim3(d.units, 4), 128, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = Shared<BITS, G>::bytes(d.n_split);

@@ -28,7 +28,7 @@ struct Derived {
   float f_lo, f_hi;
   int n_split, split_tokens;
   // workspace offsets (bytes)
-  size_t ws_tickets, ws_qfrag, ws_hconst, ws_qprime, ws_partials, ws_total;
+  size_t ws_tickets, ws_qprime, ws_partials, ws_total;
   // cache buffer sizes (bytes)
   size_t codes_bytes, params_bytes, sink_bytes, ring_bytes, state_bytes;
 };
@@ -73,8 +73,6 @@ struct DecodeArgs {
   void* out;
   int out_fp16;
   uint32_t* tickets;
-  uint32_t* qfrag;
-  float* hconst;
   float* qprime;
   float* partials;
 };
