@@ -49,6 +49,7 @@ constexpr int kThreads = 160;            // 4 consumer warps + 1 producer warp
 constexpr int kConsumers = 4;
 constexpr int kSlice = 32;               // positions per consumer warp per stage
 constexpr int kPartStride = 132;         // floats per (item, head) partial: m, l, pad, pad, o[128]
+constexpr int kTau = 8;                  // log2 headroom of the stale running max
 static_assert(kTileTokens == kConsumers * kSlice, "a stage holds one slice per consumer warp");
 
 // 2^n as an fp32 bit pattern, exact for -126 <= n <= 127.
@@ -202,28 +203,20 @@ __device__ __forceinline__ void build_query(const DecodeArgs& a, int unit, int g
 #pragma unroll
   for (int hs = 0; hs < NHS; ++hs) {
     const int hh = 4 * hs + (g >> 1);
-    float qv[32];
-    if (hh < G) {
-      const float4* src = reinterpret_cast<const float4*>(a.qprime + ((size_t)unit * G + hh) * kHeadDim + 32 * t4);
-#pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        const float4 f = src[v];
-        qv[4 * v] = f.x;
-        qv[4 * v + 1] = f.y;
-        qv[4 * v + 2] = f.z;
-        qv[4 * v + 3] = f.w;
-      }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 32; ++k) qv[k] = 0.f;
-    }
-    // dimension 32*t4 + k: its masking scale 2^l2s(k)
+    const float4* src = reinterpret_cast<const float4*>(a.qprime + ((size_t)unit * G + hh) * kHeadDim + 32 * t4);
+    // dimension 32*t4 + k: its masking scale is 2^l2s(k); pass 1: max and sum
     float amax = 0.f, sum = 0.f;
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const int l2s = BITS == 2 ? 2 * (k & 3) : 4 * (k & 1);
-      amax = fmaxf(amax, fabsf(qv[k]) * (1.0f / float(1 << l2s)));
-      sum += qv[k];
+    for (int v = 0; v < 8; ++v) {
+      const float4 f = hh < G ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k = 4 * v + e;
+        const int l2s = BITS == 2 ? 2 * (k & 3) : 4 * (k & 1);
+        amax = fmaxf(amax, fabsf(fv[e]) * (1.0f / float(1 << l2s)));
+        sum += fv[e];
+      }
     }
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
@@ -232,32 +225,39 @@ __device__ __forceinline__ void build_query(const DecodeArgs& a, int unit, int g
     const float sigma = amax > 0.f ? amax / kQMax : 1.0f;
     const float rs = 1.0f / sigma;
     const int lp = g & 1;
+    // pass 2 (values re-read from L1/L2): fixed-point digits into the fragment bytes
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      int j, r, i, l2s;
-      if (BITS == 2) {
-        r = k >> 4;
-        i = (k & 15) >> 2;
-        j = k & 3;
-        l2s = 2 * j;
-      } else {
-        const int wl = k >> 3;
-        r = wl & 1;
-        i = (k & 7) >> 1;
-        j = 2 * (wl >> 1) + (k & 1);
-        l2s = 4 * (k & 1);
+    for (int v = 0; v < 8; ++v) {
+      const float4 f = hh < G ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k = 4 * v + e;
+        int j, r, i, l2s;
+        if (BITS == 2) {
+          r = k >> 4;
+          i = (k & 15) >> 2;
+          j = k & 3;
+          l2s = 2 * j;
+        } else {
+          const int wl = k >> 3;
+          r = wl & 1;
+          i = (k & 7) >> 1;
+          j = 2 * (wl >> 1) + (k & 1);
+          l2s = 4 * (k & 1);
+        }
+        const int Q = __float2int_rn(fv[e] * (rs / float(1 << l2s)));
+        // balanced base-256 digits, each in [-128, 127]
+        const int L0 = ((Q + 128) & 255) - 128;
+        const int Q1 = (Q - L0) >> 8;
+        const int L1 = ((Q1 + 128) & 255) - 128;
+        const int Q2 = (Q1 - L1) >> 8;
+        const int L2 = ((Q2 + 128) & 255) - 128;
+        const int L3 = (Q2 - L2) >> 8;
+        const uint32_t lo = (uint32_t)((lp ? L1 : L0) & 255), hi = (uint32_t)((lp ? L3 : L2) & 255);
+        bq[j][hs][r] |= lo << (8 * i);
+        bq[j][NHS + hs][r] |= hi << (8 * i);
       }
-      const int Q = __float2int_rn(qv[k] * (rs / float(1 << l2s)));
-      // balanced base-256 digits, each in [-128, 127]
-      const int L0 = ((Q + 128) & 255) - 128;
-      const int Q1 = (Q - L0) >> 8;
-      const int L1 = ((Q1 + 128) & 255) - 128;
-      const int Q2 = (Q1 - L1) >> 8;
-      const int L2 = ((Q2 + 128) & 255) - 128;
-      const int L3 = (Q2 - L2) >> 8;
-      const uint32_t lo = (uint32_t)((lp ? L1 : L0) & 255), hi = (uint32_t)((lp ? L3 : L2) & 255);
-      bq[j][hs][r] |= lo << (8 * i);
-      bq[j][NHS + hs][r] |= hi << (8 * i);
     }
     // the lane's logit head is t4 + 4*hs: its totals live in lanes with g = 2*t4
     const float sum_t = __shfl_sync(0xffffffffu, sum, 8 * t4);
@@ -352,8 +352,10 @@ __device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, 
       vsz[i][u] = __half22float2(u32_as_h2(vpar[r]));
       val[i][u] = FULL || (tpos + r >= vlo && tpos + r < vhi);
     }
+  // The running max is kept stale: p = 2^(x - mref) may reach 2^kTau, and only a logit above
+  // mref + kTau (a warp vote) triggers the rescale, so the common path has no reduction.
   float x[2][2][NHS], alpha[NHS];
-  bool grow = false;
+  bool hit = false;
 #pragma unroll
   for (int hs = 0; hs < NHS; ++hs) {
     float mx = -CUDART_INF_F;
@@ -369,20 +371,25 @@ __device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, 
         x[i][u][hs] = (val[i][u] && hvalid[hs]) ? xv : -CUDART_INF_F;
         mx = fmaxf(mx, x[i][u][hs]);
       }
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    const float mn = fmaxf(s.m[hs], mx);
-    alpha[hs] = 1.0f;
-    if (mn > s.m[hs]) {
-      alpha[hs] = ex2(s.m[hs] - mn);
-      grow = true;
+    alpha[hs] = mx;  // lane maximum, reused below
+    hit |= mx > s.m[hs] + kTau;
+  }
+  const bool any_hit = __any_sync(0xffffffffu, hit);
+  if (any_hit) {
+#pragma unroll
+    for (int hs = 0; hs < NHS; ++hs) {
+      float mx = alpha[hs];
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float mn = fmaxf(s.m[hs], mx);
+      alpha[hs] = mn > s.m[hs] ? ex2(s.m[hs] - mn) : 1.0f;
+      s.m[hs] = mn;
     }
-    s.m[hs] = mn;
   }
   // ---- p*s enters the PV product scaled by 2^kacc: the largest weight of a slice sits below
   // 2^14 and small weights stay in fp16's normal range; kacc only decreases, and only a
-  // position whose s reaches s_lim = 2^(14 - kacc) forces a (warp-wide) recomputation
+  // position whose s reaches s_lim = 2^(14 - kTau - kacc) forces a (warp-wide) recomputation
   bool over = false;
 #pragma unroll
   for (int i = 0; i < 2; ++i)
@@ -399,15 +406,20 @@ __device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, 
     smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
     smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
     if (smax > 0.f) {
-      const int k = 13 - (((__float_as_int(smax) >> 23) & 255) - 127);  // smax * 2^k < 2^14
+      // p <= 2^kTau, so smax * 2^k < 2^(14 - kTau) keeps p*s*2^k below 2^14
+      const int k = 13 - kTau - (((__float_as_int(smax) >> 23) & 255) - 127);
       if (k < s.kacc) {
         fk = pow2i(max(k - s.kacc, -126));
         s.kacc = k;
-        s.s_lim = pow2i(14 - k);
+        s.s_lim = pow2i(14 - kTau - k);
       }
     }
   }
-  if (__any_sync(0xffffffffu, grow) || fk != 1.0f) {
+  if (any_hit || fk != 1.0f) {
+    if (!any_hit) {
+#pragma unroll
+      for (int hs = 0; hs < NHS; ++hs) alpha[hs] = 1.0f;
+    }
     // o columns are heads 2t4, 2t4+1 (lo parts in 4..7 when g <= 4); their alpha lives in
     // lanes 4g + (head & 3)
     float ac0 = __shfl_sync(0xffffffffu, alpha[0], 4 * g + ((2 * t4) & 3));
@@ -539,7 +551,7 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
     l[hh] = 0.f;
     o[hh][0] = o[hh][1] = o[hh][2] = o[hh][3] = 0.f;
   }
-  constexpr int kBatch = 8;  // positions whose loads are all in flight before any math
+  constexpr int kBatch = G >= 8 ? 2 : (G >= 4 ? 4 : 8);  // positions whose loads are in flight at once
   for (int it0 = wbeg + warp; it0 < wend; it0 += kBatch * kConsumers) {
     uint2 kraw[kBatch], vraw[kBatch];
 #pragma unroll
@@ -653,13 +665,11 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   bool hvalid[NHS];
 #pragma unroll
   for (int hs = 0; hs < NHS; ++hs) {
-    hvalid[hs] = t4 + 4 * hs < G;
+    hvalid[hs] = (G % 4 == 0) || t4 + 4 * hs < G;
     qs.m[hs] = -CUDART_INF_F;
     qs.l[hs] = 0.f;
     qs.bias[hs] = 0.f;
   }
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt) qs.o[mt][0] = qs.o[mt][1] = qs.o[mt][2] = qs.o[mt][3] = 0.f;
   qs.kacc = 64;
   qs.s_lim = 0.f;  // the first position with s > 0 sets kacc
 
@@ -688,6 +698,8 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     griddep_wait();  // q' fragments, constants and the ticket reset come from the prologue
     // (a) this warp's share of the fp16 window, while the first tiles are in flight
     window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, mg, wpv);
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) qs.o[mt][0] = qs.o[mt][1] = qs.o[mt][2] = qs.o[mt][3] = 0.f;
     // (b) quantized positions
     uint32_t bq[4][NT][2];
     float Ah[NHS], Bh[NHS];
