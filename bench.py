@@ -68,7 +68,7 @@ class StateMirror:
         wl = self.wl
         units = wl.batch * wl.n_kv_heads
         cb = 16 * wl.bits
-        lo0, nf = flush_plan(self.Sq, self.S, self.S, wl.s_sink, wl.s_keep, wl.s_flush)
+        lo0, nf = flush_plan(self.S, self.Sq, self.S, wl.s_sink, wl.s_keep, wl.s_flush)
         if nf:
             self.Sq = lo0 + nf
         self.S += n
@@ -83,6 +83,30 @@ class StateMirror:
         nw = min(wl.s_sink, self.S) + max(self.S - max(self.Sq, wl.s_sink), 0)
         per_unit = nq * 2 * (cb + 4) + nw * 512 + wl.group * (256 + 512)
         return units * per_unit + wl.n_kv_heads * 128 * 128 * 4
+
+
+def layer_config(wl, bnd, steps=32000, warmup=64, layers=32, e2e=True):
+    """Library config of one layer cache as the benchmark sizes it: capacity = context plus
+    the tokens the warm-up, timed and end-to-end steps append to each layer."""
+    per_layer = math.ceil((steps + warmup + (steps if e2e else 0) + 8) / layers)
+    return bnd.config_for_workload(wl, extra_capacity=per_layer + 64)
+
+
+def max_over_ranks(values, device, world):
+    """Element-wise max of per-rank floats over all ranks (one all-reduce; identity at world 1)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world, bytes_per_rank, seconds_max):
+    """Whole-job GB/s of `world` replicas that each moved `bytes_per_rank` in at most
+    `seconds_max` (the slowest rank's device time)."""
+    return world * bytes_per_rank / seconds_max / 1e9
 
 
 def measured_peaks():
@@ -242,8 +266,7 @@ def run_gpu(args, rank, world, local_rank):
     L = args.layers
     K, W = args.steps, args.warmup
     e2e_steps = 0 if args.no_e2e else K
-    per_layer = math.ceil((K + W + e2e_steps + 8) / L)
-    cfg = bnd.config_for_workload(wl, extra_capacity=per_layer + 64)
+    cfg = layer_config(wl, bnd, K, W, L, e2e=not args.no_e2e)
     scale = synth.default_softmax_scale(wl.head_dim)
 
     # ---- caches, prefilled to context - 1 with the bulk append path
@@ -351,13 +374,7 @@ def run_gpu(args, rank, world, local_rank):
     status = [cch.status() for cch in caches]
     assert all(s == 0 for s in status), status
 
-    t_total = t_total_ms / 1e3
-    if world > 1:
-        tt = torch.tensor([t_total, sum(dec_ms) / 1e3], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_total, dec_total = float(tt[0]), float(tt[1])
-    else:
-        dec_total = sum(dec_ms) / 1e3
+    t_total, dec_total = max_over_ranks([t_total_ms / 1e3, sum(dec_ms) / 1e3], dev, world)
 
     # ---- end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
@@ -391,12 +408,8 @@ def run_gpu(args, rank, world, local_rank):
         for j in range(e2e_steps):
             c = (first_e + j) % L
             e2e_bytes += mirrors[c].append_bytes(1) + mirrors[c].decode_bytes()
-        t_e2e = e0.elapsed_time(e1) / 1e3
-        if world > 1:
-            tt = torch.tensor([t_e2e], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            t_e2e = float(tt[0])
-        e2e = {"value": world * e2e_bytes / t_e2e / 1e9, "unit": "GB/s",
+        (t_e2e,) = max_over_ranks([e0.elapsed_time(e1) / 1e3], dev, world)
+        e2e = {"value": round(job_throughput(world, e2e_bytes, t_e2e), 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(dk.numel() * 2 + dv.numel() * 2 + dq.numel() * 2),
                "d2h_bytes_per_step": int(hout.numel() * 4)}
 
@@ -405,7 +418,7 @@ def run_gpu(args, rank, world, local_rank):
     dec_bytes_per_launch = step_dec_bytes / K
     achieved = dec_bytes_per_launch / dec_launch_s / 1e9
     total_bytes = step_app_bytes + step_dec_bytes
-    value = world * total_bytes / t_total / 1e9
+    value = job_throughput(world, total_bytes, t_total)
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -442,7 +455,7 @@ def run_gpu(args, rank, world, local_rank):
             "frac": round(achieved / peak, 4), "traffic": profile_traffic("decode_main_llama3-8b-layer.md"),
             "kernel": "wushkv_decode_attn (decode_prologue + decode_main)", "peak_kind": peak_kind,
         },
-        "gpu_launches": 3 * K,
+        "gpu_launches": 3 * K,  # per step: append_small, decode_prologue, decode_main
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -111,7 +111,7 @@ class KVCache:
         self.k_ring = torch.zeros(L.ring_bytes // 2, dtype=torch.float16, device=device)
         self.v_ring = torch.zeros(L.ring_bytes // 2, dtype=torch.float16, device=device)
         self.state = torch.zeros(L.state_bytes // 4, dtype=torch.int32, device=device)
-        self.workspace = torch.empty(L.workspace_bytes, **u8)
+        self.workspace = torch.zeros(L.workspace_bytes, **u8)
         self.bufs = CacheBufs(*(t.data_ptr() for t in (self.k_codes, self.v_codes, self.k_params, self.v_params,
                                                         self.k_sink, self.v_sink, self.k_ring, self.v_ring,
                                                         self.state)))

@@ -45,14 +45,28 @@ int derive(const wushkv_config* cfg, Derived* d) {
   if (d->nsel < 2) d->nsel = 2;
   if (d->nsel > 4) return WUSHKV_EUNSUPPORTED;
 
-  // decode work split: at most one wave of items over all units
-  int per_unit = (kB200SMs * decode_ctas_per_sm(g)) / d->units;
-  if (per_unit < 1) per_unit = 1;
-  if (per_unit > kMaxSplits) per_unit = kMaxSplits;
-  int L = ceil_div(ceil_div(d->cap_alloc, per_unit), kTileTokens) * kTileTokens;
-  if (L < kTileTokens) L = kTileTokens;
-  d->split_tokens = L;
-  d->n_split = ceil_div(d->cap_alloc, L);
+  // decode work split: n_split items per unit, chosen so that units * n_split fills whole
+  // waves of the GPU's CTA slots (the kernel divides each unit's current quantized region
+  // evenly among its items at run time); split_tokens is the per-item bound at capacity
+  {
+    const int slots = kB200SMs * decode_ctas_per_sm(g);
+    int n0 = slots / d->units;
+    if (n0 < 1) n0 = 1;
+    int best = n0;
+    double best_eff = 0.0;
+    for (int n = n0; n <= n0 + 3 && n <= kMaxSplits; ++n) {
+      const long long items = (long long)d->units * n;
+      const long long waves = (items + slots - 1) / slots;
+      const double eff = (double)items / (double)(waves * slots);
+      if (eff > best_eff + 1e-9) {
+        best_eff = eff;
+        best = n;
+      }
+    }
+    d->n_split = best > kMaxSplits ? kMaxSplits : best;
+    const int tiles = ceil_div(d->cap_alloc, kTileTokens);
+    d->split_tokens = ceil_div(tiles, d->n_split) * kTileTokens;
+  }
 
   const size_t U = (size_t)d->units;
   d->codes_bytes = U * d->cap_alloc * d->code_bytes;

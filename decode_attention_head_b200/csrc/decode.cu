@@ -153,26 +153,24 @@ __global__ void __launch_bounds__(128) decode_prologue_kernel(const DecodeArgs a
   const int unit = blockIdx.x, c = blockIdx.y;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
   const int tid = threadIdx.x, jj = tid & 31, pt = tid >> 5;
+  const int j = 32 * c + jj;
+  const float* Ti = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim + (size_t)(32 * pt) * kHeadDim + j;
+  // all 32 of this thread's T_K^{-1} loads are in flight before q is staged: one round trip
+  float t[32];
+#pragma unroll
+  for (int u = 0; u < 32; ++u) t[u] = __ldg(Ti + (size_t)u * kHeadDim);
   for (int i = tid; i < G * kHeadDim; i += 128) {
     const int hh = i / kHeadDim, cc = i % kHeadDim;
     qs[hh][cc] = __half2float(a.q[((size_t)b * a.Hq + h * G + hh) * kHeadDim + cc]);
   }
   __syncthreads();
-  const int j = 32 * c + jj;
-  const float* Ti = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim + (size_t)(32 * pt) * kHeadDim + j;
   float qp[G];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) qp[hh] = 0.f;
 #pragma unroll
-  for (int i0 = 0; i0 < 32; i0 += 16) {
-    float t[16];
+  for (int u = 0; u < 32; ++u)
 #pragma unroll
-    for (int u = 0; u < 16; ++u) t[u] = __ldg(Ti + (size_t)(i0 + u) * kHeadDim);
-#pragma unroll
-    for (int u = 0; u < 16; ++u)
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) qp[hh] = fmaf(t[u], qs[hh][32 * pt + i0 + u], qp[hh]);
-  }
+    for (int hh = 0; hh < G; ++hh) qp[hh] = fmaf(t[u], qs[hh][32 * pt + u], qp[hh]);
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) part[pt][hh][jj] = qp[hh];
   __syncthreads();
@@ -638,10 +636,15 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     S = 0;
     Sq = 0;
   }
-  // quantized positions of this item: [lo, hi) within [qlo, qhi)
+  // quantized positions of this item: [lo, hi) within [qlo, qhi).  The items split the
+  // region as it stands now (not the capacity), in whole 128-position stages counted from
+  // the stage that holds qlo, so every item but the last streams the same number of stages.
   const int qlo = a.s_sink;
   const int qhi = Sq > a.s_sink ? Sq : a.s_sink;
-  const int ibeg = item * a.split_tokens, iend = ibeg + a.split_tokens;
+  const int qbase = (qlo / kTileTokens) * kTileTokens;
+  const int tiles_all = qhi > qlo ? (qhi - qbase + kTileTokens - 1) / kTileTokens : 0;
+  const int per = (tiles_all + nitems - 1) / nitems * kTileTokens;
+  const int ibeg = qbase + item * per, iend = ibeg + per;
   const int lo = max(ibeg, qlo), hi = min(iend, qhi);
   const int tile0 = lo < hi ? (lo / kTileTokens) * kTileTokens : 0;
   const int ntiles = lo < hi ? (hi - tile0 + kTileTokens - 1) / kTileTokens : 0;

@@ -50,6 +50,7 @@ extern "C" {
 #define WUSHKV_ECUDA (-3)        /* a CUDA launch or query failed */
 #define WUSHKV_ESINGULAR (-4)    /* wushkv_compensation: T_K is singular */
 
+
 /* Bits of the device status word (state buffer, int32 index 2*batch*n_kv_heads). */
 #define WUSHKV_STATUS_OVERFLOW 1u /* an append would exceed `capacity`: that sequence was skipped */
 #define WUSHKV_STATUS_EMPTY 2u    /* decode of a sequence with S == 0: its output rows are zero */
@@ -84,11 +85,13 @@ typedef struct wushkv_layout {
   size_t state_bytes;     /* int32 [B*H_kv][2] = (S, S_quant) per (sequence, KV head), then the
                              status word; zero it to start from an empty cache */
   size_t workspace_bytes; /* wushkv_decode_attn scratch; no initialisation needed */
-  int32_t cap_alloc;      /* capacity rounded up to a multiple of 64 */
+  int32_t cap_alloc;      /* capacity rounded up to a multiple of 128 */
   int32_t ring_slots;     /* s_keep + s_flush - 1 + chunk_max; position p lives in slot p % ring_slots */
   int32_t code_bytes;     /* 128 * bits / 8 bytes of packed codes per token and head */
   int32_t n_splits;       /* decode work items per (sequence, KV head) over the quantized region */
-  int32_t split_tokens;   /* positions per decode work item (multiple of 64) */
+  int32_t split_tokens;   /* most positions one decode work item streams (at full capacity; the
+                             kernel splits each sequence's current length evenly among the
+                             n_splits items, in whole multiples of 128) */
   int32_t reserved;
 } wushkv_layout;
 
@@ -151,7 +154,8 @@ int wushkv_append(const wushkv_config* cfg, const wushkv_cache* cache, const voi
  * t_k_inv:  device fp32 [H_kv][128][128], T_K^{-1} row-major (see wushkv_compensation).
  * softmax_scale: logits are softmax_scale * q.k (1/sqrt(128) for standard attention).
  * out_fp16: 0 -> out is fp32 [B][H_q][128]; 1 -> fp16.
- * workspace: device scratch of layout.workspace_bytes (no initialisation needed).
+ * workspace: device scratch of layout.workspace_bytes (no initialisation needed; calls that
+ *   share one workspace must not overlap in time).
  * out[b][j] = sum_p softmax_p(softmax_scale * q'_j . khat_p) vhat_p over p < S, with
  *   q'_j = T_K^{-T} q_j, khat_p / vhat_p the stored fp16 k'/v in the windows and
  *   z + s*code in the quantized region.  S == 0 gives zeros and WUSHKV_STATUS_EMPTY.

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(bnd):
 def test_layout_sizes(bnd):
     cfg = bnd.make_config(8, 8, 32, 2, 32768 + 1000, 4, 128, 16, 1)
     L = bnd.pack_layout(cfg)
-    assert L.cap_alloc == 33792 and L.cap_alloc % 64 == 0
+    assert L.cap_alloc == 33792 and L.cap_alloc % 128 == 0
     assert L.code_bytes == 32
     assert L.ring_slots == 128 + 16 - 1 + 1
     assert L.codes_bytes == 64 * 33792 * 32
@@ -43,7 +43,7 @@ def test_layout_sizes(bnd):
     assert L.sink_bytes == 64 * 4 * 128 * 2
     assert L.ring_bytes == 64 * 144 * 128 * 2
     assert L.state_bytes >= (2 * 64 + 1) * 4
-    assert L.split_tokens % 64 == 0 and L.n_splits * L.split_tokens >= L.cap_alloc
+    assert L.split_tokens % 128 == 0 and L.n_splits * L.split_tokens >= L.cap_alloc
     assert L.workspace_bytes > 0
     cfg4 = bnd.make_config(64, 32, 32, 4, 8192, 4, 64, 16, 1, 0.5, 99.5)
     L4 = bnd.pack_layout(cfg4)

@@ -1,0 +1,80 @@
+"""Host-side logic of bench.py that needs no GPU: the multi-rank reduction (world size 2
+over gloo on CPU), the whole-job throughput, and the algorithmic byte accounting of a
+step, checked against the oracle cache's own Algorithm-2 bookkeeping."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+from decode_attention_head_b200 import synth
+from oracle import cache as ocache
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # rank r saw device times (r + 1, 10 - r) seconds: the job takes the slowest
+        got = bench.max_over_ranks([rank + 1.0, 10.0 - rank], "cpu", world)
+        q.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[0] == res[1] == [2.0, 10.0]
+
+
+def test_max_over_ranks_single_process_is_identity():
+    assert bench.max_over_ranks([3.0, 4.5], "cpu", 1) == [3.0, 4.5]
+
+
+def test_job_throughput_counts_every_replica():
+    # 4 replicas of 155.4 MB in 25 us (slowest rank): 4 * 6.216 TB/s
+    assert bench.job_throughput(4, 155.4e6, 25e-6) == pytest.approx(4 * 6216.0)
+
+
+@pytest.mark.parametrize("sink,keep,flush", [(4, 32, 16), (0, 8, 1), (4, 128, 16), (2, 5, 7)])
+def test_state_mirror_tracks_the_oracle_flush(sink, keep, flush):
+    """The byte accounting's (S, S_quant) mirror follows the oracle's Algorithm-2 state
+    step for step through decode-style single-token appends."""
+    wl = synth.scaled(synth.WORKLOADS["tiny"], batch=1, n_kv_heads=1, n_q_heads=4, s_sink=sink, s_keep=keep,
+                      s_flush=flush)
+    oc = ocache.Cache(1, 1, 128, 2, 1.0, 99.0, sink, keep, flush, capacity=400, chunk_max=1)
+    T = np.eye(128, dtype=np.float16)[None]
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((1, 300, 1, 128)).astype(np.float16)
+    oc.append(x[:, :100], x[:, :100], T)
+    m = bench.StateMirror(wl, int(oc.S[0]), int(oc.S_quant[0]))
+    for p in range(100, 300):
+        sq_before = int(oc.S_quant[0])
+        oc.append(x[:, p:p + 1], x[:, p:p + 1], T)
+        nbytes = m.append_bytes(1)
+        assert (m.S, m.Sq) == (int(oc.S[0]), int(oc.S_quant[0]))
+        nf = int(oc.S_quant[0]) - max(sq_before, sink) if int(oc.S_quant[0]) > sq_before else 0
+        assert nbytes == nf * (512 + 2 * 36) + 1024 + 128 * 128 * 2
+        nq = max(m.Sq - sink, 0)
+        assert m.decode_bytes() == nq * 72 + (m.S - nq) * 512 + 4 * 768 + 128 * 128 * 4
