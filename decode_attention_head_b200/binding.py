@@ -14,11 +14,13 @@ import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwushkv.so")
 
-OK, EINVAL, EUNSUPPORTED, ECUDA, ESINGULAR = 0, -1, -2, -3, -4
+OK, EINVAL, EUNSUPPORTED, ECUDA, ESINGULAR, ESCRATCH = 0, -1, -2, -3, -4, -5
+STATIC_SCRATCH_BYTES = 8 << 20  # WUSHKV_STATIC_SCRATCH_BYTES
 STATUS_OVERFLOW, STATUS_EMPTY, STATUS_TIMEOUT, STATUS_BADSTATE = 1, 2, 4, 8
 _ERR = {EINVAL: "invalid argument", EUNSUPPORTED: "unsupported configuration", ECUDA: "CUDA launch failed",
-        ESINGULAR: "singular key transform"}
-SYMBOLS = ("wushkv_pack_layout", "wushkv_compensation", "wushkv_append", "wushkv_decode_attn")
+        ESINGULAR: "singular key transform", ESCRATCH: "needs more than the static scratch array holds"}
+SYMBOLS = ("wushkv_pack_layout", "wushkv_compensation", "wushkv_append", "wushkv_decode_attn",
+           "wushkv_decode_attn_static")
 
 
 class Config(ctypes.Structure):
@@ -56,6 +58,9 @@ def _load() -> ctypes.CDLL:
     lib.wushkv_decode_attn.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
                                        ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
                                        ctypes.c_void_p, ctypes.c_void_p]
+    lib.wushkv_decode_attn_static.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
+                                              ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
+                                              ctypes.c_void_p]
     for name in SYMBOLS:
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -146,6 +151,17 @@ class KVCache:
                                       t_k_inv.data_ptr(), float(softmax_scale), 1 if out.dtype == torch.float16 else 0,
                                       out.data_ptr(), self.workspace.data_ptr(), _stream_ptr(stream)),
                "wushkv_decode_attn")
+        return out
+
+    def decode_attn_static(self, q: torch.Tensor, t_k_inv: torch.Tensor, softmax_scale: float,
+                           out: torch.Tensor, stream=None) -> torch.Tensor:
+        """decode_attn through wushkv_decode_attn_static: scratch in the library's own device
+        array, `out` supplied by the caller (fp32 or fp16), nothing allocated."""
+        _check(lib.wushkv_decode_attn_static(ctypes.byref(self.cfg), ctypes.byref(self.bufs), q.data_ptr(),
+                                             t_k_inv.data_ptr(), float(softmax_scale),
+                                             1 if out.dtype == torch.float16 else 0, out.data_ptr(),
+                                             _stream_ptr(stream)),
+               "wushkv_decode_attn_static")
         return out
 
     # -- typed views of the buffers (for tests and tools) ------------------------

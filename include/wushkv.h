@@ -22,8 +22,8 @@
  *     the first (lower address) element in the low half.
  *   - All device buffers are allocated and owned by the caller (sizes from
  *     wushkv_pack_layout), must be 16-byte aligned, and stay valid until the work
- *     queued on `stream` has finished.  The library allocates nothing and keeps no
- *     global state.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *     queued on `stream` has finished.  The library allocates nothing; its only
+ *     global state is the fixed scratch array of wushkv_decode_attn_static.  `stream` is a cudaStream_t (NULL = legacy default stream).
  *   - Calls are asynchronous: a zero return means the work was validated and
  *     queued.  Conditions only the device can see (capacity overflow, decode of an
  *     empty sequence, a bounded wait that gave up) are OR-ed into the cache's
@@ -49,7 +49,11 @@ extern "C" {
                                     needing more than the 4 extreme order statistics */
 #define WUSHKV_ECUDA (-3)        /* a CUDA launch or query failed */
 #define WUSHKV_ESINGULAR (-4)    /* wushkv_compensation: T_K is singular */
+#define WUSHKV_ESCRATCH (-5)     /* wushkv_decode_attn_static: the configuration needs more scratch
+                                    than WUSHKV_STATIC_SCRATCH_BYTES */
 
+/* Size of the library-owned device scratch array behind wushkv_decode_attn_static. */
+#define WUSHKV_STATIC_SCRATCH_BYTES (8u << 20)
 
 /* Bits of the device status word (state buffer, int32 index 2*batch*n_kv_heads). */
 #define WUSHKV_STATUS_OVERFLOW 1u /* an append would exceed `capacity`: that sequence was skipped */
@@ -163,6 +167,26 @@ int wushkv_append(const wushkv_config* cfg, const wushkv_cache* cache, const voi
 int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* cache, const void* q,
                        const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
                        void* workspace, void* stream);
+
+/* wushkv_decode_attn with library-owned scratch instead of a caller-allocated workspace.
+ * The method has no counterpart of this call: it serves callers that cannot allocate
+ * device memory when they decode (a runtime without an allocator, a step that must not
+ * enter a caching allocator, a host program that owns every buffer it hands over).
+ * Arguments, layouts, results and return codes are those of wushkv_decode_attn, minus
+ * `workspace`; it allocates nothing.
+ * Scratch: a file-scope device array of WUSHKV_STATIC_SCRATCH_BYTES that every GPU
+ *   loading the library holds until the process exits.  A configuration whose
+ *   layout.workspace_bytes exceeds it returns WUSHKV_ESCRATCH and queues nothing.
+ * Set-up: the first call made with a given device current looks up the array's device
+ *   address (cudaGetSymbolAddress) and caches it; make that first call before any
+ *   stream capture on that device.
+ * Sharing: all calls on a device share the one array, which keeps what the last call
+ *   left; each call clears the part that must start at zero (a memset queued on
+ *   `stream` ahead of the kernels).  Calls whose work overlaps in time (different
+ *   streams, or threads without ordering) race on the array: serialise them. */
+int wushkv_decode_attn_static(const wushkv_config* cfg, const wushkv_cache* cache, const void* q,
+                              const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
+                              void* stream);
 
 #ifdef __cplusplus
 }

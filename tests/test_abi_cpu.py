@@ -69,7 +69,22 @@ def test_bad_pointers_rejected_before_device_work(bnd):
     rc = bnd.lib.wushkv_decode_attn(ctypes.byref(cfg), ctypes.byref(bufs), None, None, ctypes.c_float(0.1), 0,
                                     None, None, None)
     assert rc == bnd.EINVAL
+    rc = bnd.lib.wushkv_decode_attn_static(ctypes.byref(cfg), ctypes.byref(bufs), None, None, ctypes.c_float(0.1),
+                                           0, None, None)
+    assert rc == bnd.EINVAL
     assert bnd.lib.wushkv_pack_layout(None, None) == bnd.EINVAL
+
+
+def test_static_scratch_limit_checked_on_the_host(bnd):
+    """A configuration needing more scratch than the library's array is refused before any
+    CUDA call (the pointers are never dereferenced: the check comes first)."""
+    cfg = bnd.make_config(512, 8, 64, 2, 128, 4, 32, 16, 1)
+    assert bnd.pack_layout(cfg).workspace_bytes > bnd.STATIC_SCRATCH_BYTES
+    fake = 1 << 20  # aligned, never touched
+    bufs = bnd.CacheBufs(*([fake] * 9))
+    rc = bnd.lib.wushkv_decode_attn_static(ctypes.byref(cfg), ctypes.byref(bufs), fake, fake, ctypes.c_float(0.1),
+                                           0, fake, None)
+    assert rc == bnd.ESCRATCH
 
 
 def test_compensation_inverts_fp16_transform(bnd):
