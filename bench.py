@@ -47,6 +47,9 @@ def parse_args():
     p.add_argument("--layers", type=int, default=32)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--prefill-only", action="store_true",
+                   help="only the prefill workload's bulk append + decode measurement (one JSON line)")
     return p.parse_args()
 
 
@@ -87,8 +90,8 @@ class StateMirror:
 
 def layer_config(wl, bnd, steps=32000, warmup=64, layers=32, e2e=True):
     """Library config of one layer cache as the benchmark sizes it: capacity = context plus
-    the tokens the warm-up, timed and end-to-end steps append to each layer."""
-    per_layer = math.ceil((steps + warmup + (steps if e2e else 0) + 8) / layers)
+    the tokens the warm-up, timed, per-kernel-timing and end-to-end steps append to each layer."""
+    per_layer = math.ceil((steps + warmup + min(steps, 4000) + (steps if e2e else 0) + 8) / layers)
     return bnd.config_for_workload(wl, extra_capacity=per_layer + 64)
 
 
@@ -119,19 +122,30 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def code_sha256(path):
+    """sha256 of a C++/CUDA source with // comments and blank lines removed: it changes when
+    the code changes, not when only its comments do."""
+    lines = []
+    for line in open(path, encoding="utf-8"):
+        code = line.split("//", 1)[0].rstrip()
+        if code.strip():
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
 def profile_traffic(kernel_file):
     """DRAM bytes per launch of the decode kernel from the committed ncu summary, if that
-    summary was taken on the current kernel source (its sha256 is recorded there)."""
+    summary was taken on the current kernel code (its code sha256 is recorded there)."""
     src = os.path.join(ROOT, "decode_attention_head_b200", "csrc", "decode.cu")
     path = os.path.join(ROOT, "profiles", kernel_file)
     try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        sha = code_sha256(src)
         info = {}
         for line in open(path):
             if ":" in line and line.strip().startswith("- "):
                 k, v = line.strip()[2:].split(":", 1)
                 info[k.strip()] = v.strip().strip("`")
-        if info.get("decode.cu sha256") != sha:
+        if info.get("decode.cu code sha256") != sha:
             return None
         return float(info["dram bytes per launch (full workload)"])
     except Exception:
@@ -314,39 +328,46 @@ def run_gpu(args, rank, world, local_rank):
             bytes_dec.append(mirrors[i % L].decode_bytes())
     stream.synchronize()
 
-    # ---- CUDA graphs: one (append) and one (decode) graph per layer
-    g_app, g_dec = [], []
+    # ---- CUDA graphs per layer: the fused step (wushkv_step: append + decode, the timed
+    # path) and, for the per-kernel roofline, append and decode as separate calls
+    g_step, g_app, g_dec = [], [], []
     for c in range(L):
-        ga, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        gs, ga, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gs, stream=stream):
+            caches[c].step(k_pool[c % P], v_pool[c % P], tks[c], q_pool[c % P], tinvs[c], scale, out=outs[c],
+                           stream=stream)
         with torch.cuda.graph(ga, stream=stream):
             caches[c].append(k_pool[c % P], v_pool[c % P], tks[c], stream=stream)
         with torch.cuda.graph(gd, stream=stream):
             caches[c].decode_attn(q_pool[c % P], tinvs[c], scale, out=outs[c], stream=stream)
+        g_step.append(gs)
         g_app.append(ga)
         g_dec.append(gd)
     # capture does not execute; the state mirrors stay in step with the device state
 
-    def graph_steps(n, first, evs=None):
+    def step_graphs(n, first):
+        for j in range(n):
+            g_step[(first + j) % L].replay()
+
+    def split_graphs(n, first, evs):
         for j in range(n):
             c = (first + j) % L
-            if evs is not None:
-                evs[2 * j].record(stream)
+            evs[2 * j].record(stream)
             g_app[c].replay()
-            if evs is not None:
-                evs[2 * j + 1].record(stream)
+            evs[2 * j + 1].record(stream)
             g_dec[c].replay()
+        evs[2 * n].record(stream)
 
     with torch.cuda.stream(stream):
-        graph_steps(W, L)
+        step_graphs(W, L)
     for j in range(W):
-        c = (L + j) % L
-        mirrors[c].append_bytes(1)
+        mirrors[(L + j) % L].append_bytes(1)
     stream.synchronize()
     if world > 1:
         dist.barrier()
 
-    # ---- timed region (device): exactly K steps
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K + 1)]
+    # ---- timed region (device): exactly K fused steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
     try:
         uuid = torch.cuda.get_device_properties(dev).uuid
@@ -358,23 +379,40 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     first = L + W
     with torch.cuda.stream(stream):
-        graph_steps(K, first, evs)
-        evs[2 * K].record(stream)
+        ev0.record(stream)
+        step_graphs(K, first)
+        ev1.record(stream)
     stream.synchronize()
     torch.cuda.synchronize()
-    clocks = sampler.stop()
-    t_total_ms = evs[0].elapsed_time(evs[2 * K])
-    dec_ms = [evs[2 * j + 1].elapsed_time(evs[2 * j + 2]) for j in range(K)]
-    app_ms = [evs[2 * j].elapsed_time(evs[2 * j + 1]) for j in range(K)]
+    t_total_ms = ev0.elapsed_time(ev1)
     step_app_bytes, step_dec_bytes = 0, 0
     for j in range(K):
         c = (first + j) % L
         step_app_bytes += mirrors[c].append_bytes(1)
         step_dec_bytes += mirrors[c].decode_bytes()
+
+    # ---- per-kernel timing (same workload, separate calls): events around each append and
+    # each decode call give the decode kernel's launch duration for the roofline
+    K2 = min(K, 4000)
+    first2 = first + K
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K2 + 1)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        split_graphs(K2, first2, evs)
+    stream.synchronize()
+    clocks = sampler.stop()
+    dec_ms = [evs[2 * j + 1].elapsed_time(evs[2 * j + 2]) for j in range(K2)]
+    app_ms = [evs[2 * j].elapsed_time(evs[2 * j + 1]) for j in range(K2)]
+    k2_app_bytes, k2_dec_bytes = 0, 0
+    for j in range(K2):
+        c = (first2 + j) % L
+        k2_app_bytes += mirrors[c].append_bytes(1)
+        k2_dec_bytes += mirrors[c].decode_bytes()
     status = [cch.status() for cch in caches]
     assert all(s == 0 for s in status), status
 
-    t_total, dec_total = max_over_ranks([t_total_ms / 1e3, sum(dec_ms) / 1e3], dev, world)
+    t_total, dec_total, app_total = max_over_ranks([t_total_ms / 1e3, sum(dec_ms) / 1e3, sum(app_ms) / 1e3], dev,
+                                                   world)
 
     # ---- end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
@@ -386,7 +424,7 @@ def run_gpu(args, rank, world, local_rank):
         dk = torch.empty_like(k_pool[0])
         dv = torch.empty_like(v_pool[0])
         dq = torch.empty_like(q_pool[0])
-        first_e = first + K
+        first_e = first2 + K2
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
@@ -400,8 +438,7 @@ def run_gpu(args, rank, world, local_rank):
                 dk.copy_(hk[i % P], non_blocking=True)
                 dv.copy_(hv[i % P], non_blocking=True)
                 dq.copy_(hq[i % P], non_blocking=True)
-                caches[c].append(dk, dv, tks[c], stream=stream)
-                caches[c].decode_attn(dq, tinvs[c], scale, out=outs[c], stream=stream)
+                caches[c].step(dk, dv, tks[c], dq, tinvs[c], scale, out=outs[c], stream=stream)
                 hout.copy_(outs[c], non_blocking=True)
             e1.record(stream)
         stream.synchronize()
@@ -414,8 +451,8 @@ def run_gpu(args, rank, world, local_rank):
                "d2h_bytes_per_step": int(hout.numel() * 4)}
 
     peak, peak_kind = measured_peaks()
-    dec_launch_s = dec_total / K
-    dec_bytes_per_launch = step_dec_bytes / K
+    dec_launch_s = dec_total / K2
+    dec_bytes_per_launch = k2_dec_bytes / K2
     achieved = dec_bytes_per_launch / dec_launch_s / 1e9
     total_bytes = step_app_bytes + step_dec_bytes
     value = job_throughput(world, total_bytes, t_total)
@@ -440,28 +477,103 @@ def run_gpu(args, rank, world, local_rank):
             "layers_rotated": L,
             "l2": f"inputs larger than L2: {L} rotating layer caches, "
                   f"{L * (bnd.pack_layout(cfg).codes_bytes * 2 + bnd.pack_layout(cfg).params_bytes * 2) / 1e9:.1f} GB",
-            "launch": "per-layer CUDA graphs (append, decode)",
+            "launch": "per-layer CUDA graphs of wushkv_step (append fused with decode)",
+            "per_kernel_timing": "append and decode as separate calls, events per launch, "
+                                 "min(K, 4000) more steps of the same workload",
             "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
         },
         "decode_attn_gbs": round(achieved, 2),
         "decode_pct_of_measured_hbm": round(100 * achieved / peak, 2),
         "decode_pct_of_8tbps": round(100 * achieved / NOMINAL_HBM_GBS, 2),
         "decode_us_per_launch": round(dec_launch_s * 1e6, 3),
-        "append_gbs": round(step_app_bytes / (sum(app_ms) / 1e3) / 1e9, 2),
-        "append_us_per_launch": round(sum(app_ms) / K * 1e3, 3),
+        "append_gbs": round(k2_app_bytes / app_total / 1e9, 2),
+        "append_us_per_launch": round(app_total / K2 * 1e6, 3),
         "layer_tokens_per_s": round(world * wl.batch * K / t_total, 1),
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": profile_traffic("decode_main_llama3-8b-layer.md"),
             "kernel": "wushkv_decode_attn (decode_prologue + decode_main)", "peak_kind": peak_kind,
         },
-        "gpu_launches": 3 * K,  # per step: append_small, decode_prologue, decode_main
+        "gpu_launches": 2 * K,  # per timed step: fused append_small + decode_main
         "clocks": clocks,
         "e2e": e2e,
     }
     # release graphs before the process group goes away
-    del g_app, g_dec
+    del g_step, g_app, g_dec
+    if not args.no_prefill:
+        del caches, outs
+        torch.cuda.empty_cache()
+        result["prefill_append"] = measure_prefill(bnd, synth, dev)
     return result, wl
+
+
+def bulk_append_bytes(wl, S, Sq, n):
+    """Algorithmic bytes of one n-token bulk append to every (sequence, KV head) of `wl` at
+    state (S, S_quant): fp16 k / v in, T_K, ring entries the flush re-reads, codes and
+    (s, z) of the newly quantized positions, fp16 ring writes of the new tokens kept."""
+    units = wl.batch * wl.n_kv_heads
+    cb = 16 * wl.bits
+    lo0, nf = flush_plan(S, Sq, S + n, wl.s_sink, wl.s_keep, wl.s_flush)
+    from_ring = max(0, min(lo0 + nf, S) - lo0)
+    kept_new = S + n - max(lo0 + nf, S)
+    per_unit = n * 2 * 256 + from_ring * 2 * 256 + nf * 2 * (cb + 4) + kept_new * 2 * 256
+    return units * per_unit + wl.n_kv_heads * 128 * 128 * 2
+
+
+def measure_prefill(bnd, synth, dev, reps=5):
+    """The prefill workload's append: one bulk append of its chunk (16,384 tokens per
+    sequence) into a 114,688-token cache, then its decode at 131,072.  The append is
+    repeated from the same state (state words and fp16 ring restored, so every repetition
+    does the same work and writes the same codes), each timed with CUDA events."""
+    import torch
+    wl = synth.WORKLOADS["prefill-append-decode"]
+    n = wl.prefill_chunk
+    base = wl.context - n
+    cfg = bnd.config_for_workload(wl, extra_capacity=64)
+    c = bnd.KVCache(cfg, device=dev)
+    T = synth.key_transforms(wl, 0)
+    tk, tinv = T.to(dev), bnd.compensation(T).to(dev)
+    for s0 in range(0, base, 4096):
+        m = min(4096, base - s0)
+        c.append(synth.bulk_tokens(wl, 0, s0, m, device=dev, which="k"),
+                 synth.bulk_tokens(wl, 0, s0, m, device=dev, which="v"), tk)
+    kk = synth.bulk_tokens(wl, 0, base, n, device=dev, which="k")
+    vv = synth.bulk_tokens(wl, 0, base, n, device=dev, which="v")
+    q = synth.bulk_queries(wl, 0, wl.context, device=dev)
+    out = torch.empty(wl.batch, wl.n_q_heads, wl.head_dim, device=dev)
+    torch.cuda.synchronize()
+    state0, kring0, vring0 = c.state.clone(), c.k_ring.clone(), c.v_ring.clone()
+    S0, Sq0 = (int(t[0, 0].item()) for t in c.lengths())
+    scale = synth.default_softmax_scale(wl.head_dim)
+    app_ms, dec_ms = [], []
+    for r in range(reps + 1):
+        c.state.copy_(state0)
+        c.k_ring.copy_(kring0)
+        c.v_ring.copy_(vring0)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        torch.cuda.synchronize()
+        e0.record()
+        c.append(kk, vv, tk)
+        e1.record()
+        c.decode_attn(q, tinv, scale, out=out)
+        e2.record()
+        torch.cuda.synchronize()
+        if r:
+            app_ms.append(e0.elapsed_time(e1))
+            dec_ms.append(e1.elapsed_time(e2))
+    assert c.status() == 0
+    app_s = sum(app_ms) / len(app_ms) / 1e3
+    dec_s = sum(dec_ms) / len(dec_ms) / 1e3
+    nbytes = bulk_append_bytes(wl, S0, Sq0, n)
+    S1, Sq1 = (int(t[0, 0].item()) for t in c.lengths())
+    dec_bytes = StateMirror(wl, S1, Sq1).decode_bytes()
+    flop = 2.0 * wl.batch * wl.n_kv_heads * n * 128 * 128
+    return {"workload": wl.name, "chunk_tokens": n, "cached_before": S0,
+            "append_us": round(app_s * 1e6, 2), "append_gbs": round(nbytes / app_s / 1e9, 2),
+            "append_bytes": nbytes, "transform_tflops": round(flop / app_s / 1e12, 2),
+            "decode_us_at_131072": round(dec_s * 1e6, 2), "decode_gbs": round(dec_bytes / dec_s / 1e9, 2),
+            "launch": "eager, 3 append launches (flush_ring, append_bulk, advance_state) + 2 decode launches",
+            "reps": reps}
 
 
 def main():
@@ -494,6 +606,15 @@ def main():
 
     import torch
     import torch.distributed as dist
+    if args.prefill_only:
+        from decode_attention_head_b200 import binding as bnd
+        from decode_attention_head_b200 import build as _build
+        from decode_attention_head_b200 import synth
+        _build.build()
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        print(json.dumps(measure_prefill(bnd, synth, dev)))
+        return 0
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))

@@ -20,7 +20,7 @@ STATUS_OVERFLOW, STATUS_EMPTY, STATUS_TIMEOUT, STATUS_BADSTATE = 1, 2, 4, 8
 _ERR = {EINVAL: "invalid argument", EUNSUPPORTED: "unsupported configuration", ECUDA: "CUDA launch failed",
         ESINGULAR: "singular key transform", ESCRATCH: "needs more than the static scratch array holds"}
 SYMBOLS = ("wushkv_pack_layout", "wushkv_compensation", "wushkv_append", "wushkv_decode_attn",
-           "wushkv_decode_attn_static")
+           "wushkv_step", "wushkv_decode_attn_static")
 
 
 class Config(ctypes.Structure):
@@ -58,6 +58,9 @@ def _load() -> ctypes.CDLL:
     lib.wushkv_decode_attn.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
                                        ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
                                        ctypes.c_void_p, ctypes.c_void_p]
+    lib.wushkv_step.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p, ctypes.c_void_p,
+                                ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     lib.wushkv_decode_attn_static.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
                                               ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
                                               ctypes.c_void_p]
@@ -151,6 +154,19 @@ class KVCache:
                                       t_k_inv.data_ptr(), float(softmax_scale), 1 if out.dtype == torch.float16 else 0,
                                       out.data_ptr(), self.workspace.data_ptr(), _stream_ptr(stream)),
                "wushkv_decode_attn")
+        return out
+
+    def step(self, k_new: torch.Tensor, v_new: torch.Tensor, t_k: torch.Tensor, q: torch.Tensor,
+             t_k_inv: torch.Tensor, softmax_scale: float, out: Optional[torch.Tensor] = None,
+             out_fp16: bool = False, stream=None) -> torch.Tensor:
+        """append(k_new, v_new) then decode_attn(q) in one call (wushkv_step)."""
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float16 if out_fp16 else torch.float32, device=q.device)
+        _check(lib.wushkv_step(ctypes.byref(self.cfg), ctypes.byref(self.bufs), k_new.data_ptr(), v_new.data_ptr(),
+                               k_new.shape[1], t_k.data_ptr(), q.data_ptr(), t_k_inv.data_ptr(), float(softmax_scale),
+                               1 if out.dtype == torch.float16 else 0, out.data_ptr(), self.workspace.data_ptr(),
+                               _stream_ptr(stream)),
+               "wushkv_step")
         return out
 
     def decode_attn_static(self, q: torch.Tensor, t_k_inv: torch.Tensor, softmax_scale: float,

@@ -75,12 +75,15 @@ int derive(const wushkv_config* cfg, Derived* d) {
   d->ring_bytes = U * (size_t)d->ring * kHeadDim * 2;
   d->state_bytes = round_up((2 * U + 1) * 4, 16);
   size_t off = 0;
-  d->ws_tickets = off;
-  off = round_up(off + U * 4, 256);
+  d->ws_tickets = off;  // unit counters, then group counters
+  off = round_up(off + U * 4 * (1 + (size_t)ceil_div(d->n_split, kMergeGroup)), 256);
   d->ws_qprime = off;
   off = round_up(off + U * g * kHeadDim * 4, 256);
   d->ws_partials = off;
   off = round_up(off + U * (size_t)d->n_split * g * 132 * 4, 256);
+  const size_t ngroups = (size_t)ceil_div(d->n_split, kMergeGroup);
+  d->ws_gpartials = off;
+  off = round_up(off + U * ngroups * g * 132 * 4, 256);
   d->ws_total = off;
   return WUSHKV_OK;
 }
@@ -159,41 +162,101 @@ extern "C" int wushkv_compensation(const uint16_t* t_k, int32_t n_kv_heads, floa
   return WUSHKV_OK;
 }
 
+static void fill_append(const wushkv_config* cfg, const Derived& d, const wushkv_cache* cache, const void* k_new,
+                        const void* v_new, int32_t n_new, const void* t_k, AppendArgs* a) {
+  std::memset(a, 0, sizeof(*a));
+  a->B = cfg->batch;
+  a->Hkv = cfg->n_kv_heads;
+  a->cap = cfg->capacity;
+  a->cap_alloc = d.cap_alloc;
+  a->s_sink = cfg->s_sink;
+  a->s_keep = cfg->s_keep;
+  a->s_flush = cfg->s_flush;
+  a->R = d.ring;
+  a->sink_dim = d.sink_dim;
+  a->n_new = n_new;
+  a->k_codes = static_cast<uint8_t*>(cache->k_codes);
+  a->v_codes = static_cast<uint8_t*>(cache->v_codes);
+  a->k_params = static_cast<uint32_t*>(cache->k_params);
+  a->v_params = static_cast<uint32_t*>(cache->v_params);
+  a->k_sink = static_cast<__half*>(cache->k_sink);
+  a->v_sink = static_cast<__half*>(cache->v_sink);
+  a->k_ring = static_cast<__half*>(cache->k_ring);
+  a->v_ring = static_cast<__half*>(cache->v_ring);
+  a->state = cache->state;
+  a->status = reinterpret_cast<uint32_t*>(cache->state + 2 * (size_t)d.units);
+  a->k_new = static_cast<const __half*>(k_new);
+  a->v_new = static_cast<const __half*>(v_new);
+  a->t_k = static_cast<const __half*>(t_k);
+  a->i_lo = d.i_lo;
+  a->i_hi = d.i_hi;
+  a->f_lo = d.f_lo;
+  a->f_hi = d.f_hi;
+  a->Hq = cfg->n_q_heads;
+  a->ngroups = ceil_div(d.n_split, kMergeGroup);
+}
+
+static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv_cache* cache, const void* q,
+                        const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out, void* workspace,
+                        DecodeArgs* a) {
+  std::memset(a, 0, sizeof(*a));
+  a->B = cfg->batch;
+  a->Hkv = cfg->n_kv_heads;
+  a->Hq = cfg->n_q_heads;
+  a->cap_alloc = d.cap_alloc;
+  a->s_sink = cfg->s_sink;
+  a->R = d.ring;
+  a->sink_dim = d.sink_dim;
+  a->n_split = d.n_split;
+  a->split_tokens = d.split_tokens;
+  a->k_codes = static_cast<const uint8_t*>(cache->k_codes);
+  a->v_codes = static_cast<const uint8_t*>(cache->v_codes);
+  a->k_params = static_cast<const uint32_t*>(cache->k_params);
+  a->v_params = static_cast<const uint32_t*>(cache->v_params);
+  a->k_sink = static_cast<const __half*>(cache->k_sink);
+  a->v_sink = static_cast<const __half*>(cache->v_sink);
+  a->k_ring = static_cast<const __half*>(cache->k_ring);
+  a->v_ring = static_cast<const __half*>(cache->v_ring);
+  a->state = cache->state;
+  a->status = reinterpret_cast<uint32_t*>(cache->state + 2 * (size_t)d.units);
+  a->q = static_cast<const __half*>(q);
+  a->t_k_inv = t_k_inv;
+  a->scale_log2 = softmax_scale * 1.4426950408889634f;
+  a->out = out;
+  a->out_fp16 = out_fp16;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a->tickets = reinterpret_cast<uint32_t*>(ws + d.ws_tickets);
+  a->qprime = reinterpret_cast<float*>(ws + d.ws_qprime);
+  a->partials = reinterpret_cast<float*>(ws + d.ws_partials);
+  a->gpartials = reinterpret_cast<float*>(ws + d.ws_gpartials);
+  a->units = d.units;
+  a->wait_all = 0;
+}
+
+static int check_append(const wushkv_cache* cache, const void* k_new, const void* v_new, int32_t n_new,
+                        const void* t_k) {
+  if (!cache_ok(cache) || n_new < 0 || !aligned16(t_k)) return WUSHKV_EINVAL;
+  if (n_new > 0 && (!aligned16(k_new) || !aligned16(v_new))) return WUSHKV_EINVAL;
+  return WUSHKV_OK;
+}
+
+static int check_decode(const wushkv_cache* cache, const void* q, const float* t_k_inv, float softmax_scale,
+                        int32_t out_fp16, const void* out, const void* workspace) {
+  if (!cache_ok(cache) || !aligned16(q) || !aligned16(t_k_inv) || !aligned16(out) || !aligned16(workspace))
+    return WUSHKV_EINVAL;
+  if (!std::isfinite(softmax_scale) || (out_fp16 != 0 && out_fp16 != 1)) return WUSHKV_EINVAL;
+  return WUSHKV_OK;
+}
+
 extern "C" int wushkv_append(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new,
                              const void* v_new, int32_t n_new, const void* t_k, void* stream) {
   Derived d;
-  const int rc = derive(cfg, &d);
+  int rc = derive(cfg, &d);
   if (rc != WUSHKV_OK) return rc;
-  if (!cache_ok(cache) || n_new < 0 || !aligned16(t_k)) return WUSHKV_EINVAL;
-  if (n_new > 0 && (!aligned16(k_new) || !aligned16(v_new))) return WUSHKV_EINVAL;
+  rc = check_append(cache, k_new, v_new, n_new, t_k);
+  if (rc != WUSHKV_OK) return rc;
   AppendArgs a;
-  a.B = cfg->batch;
-  a.Hkv = cfg->n_kv_heads;
-  a.cap = cfg->capacity;
-  a.cap_alloc = d.cap_alloc;
-  a.s_sink = cfg->s_sink;
-  a.s_keep = cfg->s_keep;
-  a.s_flush = cfg->s_flush;
-  a.R = d.ring;
-  a.sink_dim = d.sink_dim;
-  a.n_new = n_new;
-  a.k_codes = static_cast<uint8_t*>(cache->k_codes);
-  a.v_codes = static_cast<uint8_t*>(cache->v_codes);
-  a.k_params = static_cast<uint32_t*>(cache->k_params);
-  a.v_params = static_cast<uint32_t*>(cache->v_params);
-  a.k_sink = static_cast<__half*>(cache->k_sink);
-  a.v_sink = static_cast<__half*>(cache->v_sink);
-  a.k_ring = static_cast<__half*>(cache->k_ring);
-  a.v_ring = static_cast<__half*>(cache->v_ring);
-  a.state = cache->state;
-  a.status = reinterpret_cast<uint32_t*>(cache->state + 2 * (size_t)d.units);
-  a.k_new = static_cast<const __half*>(k_new);
-  a.v_new = static_cast<const __half*>(v_new);
-  a.t_k = static_cast<const __half*>(t_k);
-  a.i_lo = d.i_lo;
-  a.i_hi = d.i_hi;
-  a.f_lo = d.f_lo;
-  a.f_hi = d.f_hi;
+  fill_append(cfg, d, cache, k_new, v_new, n_new, t_k, &a);
   const bool small = n_new <= cfg->chunk_max;
   const cudaError_t e = launch_append(d, cfg->bits, small, a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA;
@@ -203,40 +266,47 @@ extern "C" int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* 
                                   const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
                                   void* workspace, void* stream) {
   Derived d;
-  const int rc = derive(cfg, &d);
+  int rc = derive(cfg, &d);
   if (rc != WUSHKV_OK) return rc;
-  if (!cache_ok(cache) || !aligned16(q) || !aligned16(t_k_inv) || !aligned16(out) || !aligned16(workspace))
-    return WUSHKV_EINVAL;
-  if (!std::isfinite(softmax_scale) || (out_fp16 != 0 && out_fp16 != 1)) return WUSHKV_EINVAL;
+  rc = check_decode(cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace);
+  if (rc != WUSHKV_OK) return rc;
   DecodeArgs a;
-  a.B = cfg->batch;
-  a.Hkv = cfg->n_kv_heads;
-  a.Hq = cfg->n_q_heads;
-  a.cap_alloc = d.cap_alloc;
-  a.s_sink = cfg->s_sink;
-  a.R = d.ring;
-  a.sink_dim = d.sink_dim;
-  a.n_split = d.n_split;
-  a.split_tokens = d.split_tokens;
-  a.k_codes = static_cast<const uint8_t*>(cache->k_codes);
-  a.v_codes = static_cast<const uint8_t*>(cache->v_codes);
-  a.k_params = static_cast<const uint32_t*>(cache->k_params);
-  a.v_params = static_cast<const uint32_t*>(cache->v_params);
-  a.k_sink = static_cast<const __half*>(cache->k_sink);
-  a.v_sink = static_cast<const __half*>(cache->v_sink);
-  a.k_ring = static_cast<const __half*>(cache->k_ring);
-  a.v_ring = static_cast<const __half*>(cache->v_ring);
-  a.state = cache->state;
-  a.status = reinterpret_cast<uint32_t*>(cache->state + 2 * (size_t)d.units);
-  a.q = static_cast<const __half*>(q);
-  a.t_k_inv = t_k_inv;
-  a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  a.out = out;
-  a.out_fp16 = out_fp16;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  a.tickets = reinterpret_cast<uint32_t*>(ws + d.ws_tickets);
-  a.qprime = reinterpret_cast<float*>(ws + d.ws_qprime);
-  a.partials = reinterpret_cast<float*>(ws + d.ws_partials);
+  fill_decode(cfg, d, cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace, &a);
   const cudaError_t e = launch_decode(d, cfg->bits, a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA;
+}
+
+extern "C" int wushkv_step(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
+                           int32_t n_new, const void* t_k, const void* q, const float* t_k_inv, float softmax_scale,
+                           int32_t out_fp16, void* out, void* workspace, void* stream) {
+  Derived d;
+  int rc = derive(cfg, &d);
+  if (rc != WUSHKV_OK) return rc;
+  rc = check_append(cache, k_new, v_new, n_new, t_k);
+  if (rc != WUSHKV_OK) return rc;
+  rc = check_decode(cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace);
+  if (rc != WUSHKV_OK) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AppendArgs aa;
+  fill_append(cfg, d, cache, k_new, v_new, n_new, t_k, &aa);
+  DecodeArgs da;
+  fill_decode(cfg, d, cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace, &da);
+  cudaError_t e;
+  if (n_new <= cfg->chunk_max) {
+    // one kernel appends and prepares the decode (q', counters); the main decode kernel
+    // is its programmatic dependent and waits for it before reading the cache
+    aa.q = da.q;
+    aa.t_k_inv = da.t_k_inv;
+    aa.qprime = da.qprime;
+    aa.tickets = da.tickets;
+    e = launch_append_fused(d, cfg->bits, aa, st);
+    if (e == cudaSuccess) {
+      da.wait_all = 1;
+      e = launch_decode_main(d, cfg->bits, da, st);
+    }
+  } else {
+    e = launch_append(d, cfg->bits, false, aa, st);
+    if (e == cudaSuccess) e = launch_decode(d, cfg->bits, da, st);
+  }
   return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA;
 }

@@ -51,14 +51,17 @@ __device__ __forceinline__ QuantSpec spec_of(const AppendArgs& a) {
   return q;
 }
 
-// Quantize ring positions [p_begin, p_end) of `unit` (K and V), threads of the CTA in turn.
+// Quantize ring positions [p_begin, p_end) of `unit` (K and V): each row is split over four
+// adjacent threads (quantize_row_part), nthreads / 4 rows at a time.
 template <int BITS, int NSEL>
-__device__ void quantize_ring_range(const AppendArgs& a, int unit, int p_begin, int p_end) {
+__device__ void quantize_ring_range(const AppendArgs& a, int unit, int p_begin, int p_end, int tid = threadIdx.x,
+                                    int nthreads = blockDim.x) {
   const int n = p_end - p_begin;
   if (n <= 0) return;
   constexpr int CB = 16 * BITS;
+  constexpr int P = 4;
   const QuantSpec qs = spec_of(a);
-  for (int item = threadIdx.x; item < 2 * n; item += blockDim.x) {
+  for (int item = tid / P; item < 2 * n; item += nthreads / P) {
     const int kind = item / n;  // 0 = K, 1 = V
     const int p = p_begin + item % n;
     const __half* ring = kind ? a.v_ring : a.k_ring;
@@ -66,33 +69,91 @@ __device__ void quantize_ring_range(const AppendArgs& a, int unit, int p_begin, 
     const size_t rec = (size_t)unit * a.cap_alloc + p;
     uint8_t* codes = (kind ? a.v_codes : a.k_codes) + rec * CB;
     uint32_t* params = (kind ? a.v_params : a.k_params) + rec;
-    quantize_row<BITS, NSEL>(row, codes, params, qs);
+    quantize_row_part<BITS, NSEL, P>(row, tid % P, codes, params, qs);
   }
 }
 
 // ---------------------------------------------------------------------------------
-// Small append: one CTA (128 threads) per (sequence, KV head).
-template <int BITS, int NSEL>
-__global__ void __launch_bounds__(128) append_small_kernel(const AppendArgs a) {
+// q'_j = T_K^{-T} q_j (fp32) of the unit's G query heads into the decode workspace, by the
+// CTA's 128 threads: warp w sums rows [32w, 32w+32) of T_K^{-1} for the four dimensions
+// 4*lane .. 4*lane+3 (all 32 float4 loads in flight at once), the warps' partial sums meet
+// in shared memory.  Also resets the unit's decode completion counters.
+template <int G>
+__device__ void prepare_query(const AppendArgs& a, int unit, int tid) {
+  __shared__ float qs[G][kHeadDim];
+  __shared__ float red[4][G][kHeadDim];
+  const int b = unit / a.Hkv, h = unit % a.Hkv;
+  const int warp = tid >> 5, lane = tid & 31;
+  const float4* Ti =
+      reinterpret_cast<const float4*>(a.t_k_inv + ((size_t)h * kHeadDim + 32 * warp) * kHeadDim) + lane;
+  float4 t[32];
+#pragma unroll
+  for (int u = 0; u < 32; ++u) t[u] = __ldg(Ti + (size_t)u * (kHeadDim / 4));
+  for (int i = tid; i < G * kHeadDim; i += 128)
+    qs[i / kHeadDim][i % kHeadDim] = __half2float(a.q[((size_t)b * a.Hq + h * G) * kHeadDim + i]);
+  bar_sync(2, 128);
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const float qv = qs[hh][32 * warp + u];
+      acc.x = fmaf(t[u].x, qv, acc.x);
+      acc.y = fmaf(t[u].y, qv, acc.y);
+      acc.z = fmaf(t[u].z, qv, acc.z);
+      acc.w = fmaf(t[u].w, qv, acc.w);
+    }
+    reinterpret_cast<float4*>(red[warp][hh])[lane] = acc;
+  }
+  bar_sync(2, 128);
+  for (int i = tid; i < G * kHeadDim; i += 128) {
+    const int hh = i / kHeadDim, j = i % kHeadDim;
+    a.qprime[(size_t)unit * G * kHeadDim + i] = (red[0][hh][j] + red[1][hh][j]) + (red[2][hh][j] + red[3][hh][j]);
+  }
+  for (int i = tid; i < a.ngroups; i += 128) a.tickets[a.B * a.Hkv + (size_t)unit * a.ngroups + i] = 0u;
+  if (tid == 0) a.tickets[unit] = 0u;
+}
+
+// Small append: one CTA per (sequence, KV head); threads 0..127 append.  G > 0: the fused
+// step (wushkv_step) also prepares the decode that follows (q' and its counters) on
+// threads 128..255, in parallel with the append and for every unit, including one whose
+// append is refused (its cache is decoded as it stands).  The two halves synchronise on
+// separate named barriers (1: append, 2: decode preparation).
+template <int BITS, int NSEL, int G>
+__global__ void __launch_bounds__(G > 0 ? 256 : 128) append_small_kernel(const AppendArgs a) {
+  if (G > 0) {
+    griddep_launch();  // the decode kernel may launch now; it waits for this whole grid
+    if (threadIdx.x >= 128) {
+      prepare_query<(G > 0 ? G : 1)>(a, blockIdx.x, threadIdx.x - 128);
+      return;
+    }
+  }
   const int unit = blockIdx.x;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
   const int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
+  bool fits = true;
   if (!state_ok(S, Sq, a)) {
     if (threadIdx.x == 0) atomicOr(a.status, kStatusBadState);
-    return;
-  }
-  if (S + a.n_new > a.cap) {
+    fits = false;
+  } else if (S + a.n_new > a.cap) {
     if (threadIdx.x == 0) atomicOr(a.status, kStatusOverflow);
-    return;
+    fits = false;
   }
+  if (!fits) return;
   // 1. the flush that closes the previous chunk (entries still in the ring)
   const FlushPlan fp = flush_plan(Sq, S, a);
-  quantize_ring_range<BITS, NSEL>(a, unit, fp.lo0, fp.lo0 + fp.nf);
-  __syncthreads();  // ring slots are read above before new tokens may reuse them below
+  quantize_ring_range<BITS, NSEL>(a, unit, fp.lo0, fp.lo0 + fp.nf, threadIdx.x, 128);
+  bar_sync(1, 128);  // ring slots are read above before new tokens may reuse them below
 
-  // 2. new tokens: k' = fp16_rn(T_K k) (fp32 accumulation), v as given
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const __half* T = a.t_k + (size_t)h * kHeadDim * kHeadDim;
+  // 2. new tokens: k' = fp16_rn(T_K k) (fp32 accumulation), v as given.  Thread r owns
+  // output row r: its 256-byte row of T_K is loaded once (16 x 16 B in flight), the
+  // token's key is staged in shared memory as fp32.
+  __shared__ float ks[kHeadDim];
+  const int r = threadIdx.x;
+  const uint4* Trow = reinterpret_cast<const uint4*>(a.t_k + ((size_t)h * kHeadDim + r) * kHeadDim);
+  uint4 tr[kHeadDim / 8];
+#pragma unroll
+  for (int i = 0; i < kHeadDim / 8; ++i) tr[i] = Trow[i];
   for (int t = 0; t < a.n_new; ++t) {
     const int p = S + t;
     const size_t src = (((size_t)b * a.n_new + t) * a.Hkv + h) * kHeadDim;
@@ -105,30 +166,24 @@ __global__ void __launch_bounds__(128) append_small_kernel(const AppendArgs a) {
       kdst = a.k_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
       vdst = a.v_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
     }
-    // lane holds k[4*lane .. 4*lane+3]
-    const uint2 kraw = *reinterpret_cast<const uint2*>(a.k_new + src + 4 * lane);
-    const float2 k01 = __half22float2(u32_as_h2(kraw.x));
-    const float2 k23 = __half22float2(u32_as_h2(kraw.y));
-    float mine = 0.f;
-    for (int j = 0; j < 32; ++j) {
-      const int r = 32 * warp + j;
-      const uint2 traw = *reinterpret_cast<const uint2*>(T + (size_t)r * kHeadDim + 4 * lane);
-      const float2 t01 = __half22float2(u32_as_h2(traw.x));
-      const float2 t23 = __half22float2(u32_as_h2(traw.y));
-      float acc = t01.x * k01.x;
-      acc = fmaf(t01.y, k01.y, acc);
-      acc = fmaf(t23.x, k23.x, acc);
-      acc = fmaf(t23.y, k23.y, acc);
+    ks[r] = __half2float(a.k_new[src + r]);
+    if (r < kHeadDim / 8)
+      reinterpret_cast<uint4*>(vdst)[r] = reinterpret_cast<const uint4*>(a.v_new + src)[r];
+    bar_sync(1, 128);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four interleaved partial sums, added at the end
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == j) mine = acc;
+    for (int i = 0; i < kHeadDim / 8; ++i) {
+      const uint32_t w[4] = {tr[i].x, tr[i].y, tr[i].z, tr[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 tf = __half22float2(u32_as_h2(w[e]));
+        acc[e] = fmaf(tf.x, ks[8 * i + 2 * e], acc[e]);
+        acc[e] = fmaf(tf.y, ks[8 * i + 2 * e + 1], acc[e]);
+      }
     }
-    kdst[32 * warp + lane] = __float2half_rn(mine);
-    if (threadIdx.x < 32) {
-      reinterpret_cast<uint2*>(vdst)[threadIdx.x] = reinterpret_cast<const uint2*>(a.v_new + src)[threadIdx.x];
-    }
+    kdst[r] = __float2half_rn((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    bar_sync(1, 128);  // ks is rewritten by the next token
   }
-  __syncthreads();
   // 3. state
   if (threadIdx.x == 0) {
     a.state[2 * unit] = S + a.n_new;
@@ -147,16 +202,19 @@ __global__ void __launch_bounds__(128) flush_ring_kernel(const AppendArgs a) {
   quantize_ring_range<BITS, NSEL>(a, unit, fp.lo0, min(fp.lo0 + fp.nf, S));
 }
 
-// Bulk append, launch 2.  CTA = (256-token slab, unit), 4 warps; per 64-token tile:
-// load k / v tiles and T_K into padded shared memory, k' = k T_K^T on tensor cores,
-// fp16 k' back into the k tile, then one thread per token-head quantizes or stores.
+// Bulk append, launch 2.  CTA = (256-token slab, unit), 8 warps; per 64-token tile:
+// load k / v tiles and T_K into padded shared memory, k' = k T_K^T on tensor cores
+// (warp w: tile rows 16*(w%4).., output columns 64*(w/4)..), fp16 k' back into the k tile,
+// then two threads per token-head row quantize it (or store it fp16).
 constexpr int kBulkTile = 64;
 constexpr int kBulkSlab = 256;
 constexpr int kPad = 136;  // halves per padded shared row (272 bytes: conflict-free ldmatrix)
 constexpr size_t kBulkSmem = (size_t)(kHeadDim + 2 * kBulkTile) * kPad * sizeof(__half);
 
+constexpr int kBulkThreads = 256;
+
 template <int BITS, int NSEL>
-__global__ void __launch_bounds__(128) append_bulk_kernel(const AppendArgs a) {
+__global__ void __launch_bounds__(kBulkThreads) append_bulk_kernel(const AppendArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __half* Ts = reinterpret_cast<__half*>(smem_raw);
   __half* ks = Ts + kHeadDim * kPad;
@@ -174,7 +232,7 @@ __global__ void __launch_bounds__(128) append_bulk_kernel(const AppendArgs a) {
 
   // T_K -> shared (row r = output dim, col i = input dim)
   const __half* T = a.t_k + (size_t)h * kHeadDim * kHeadDim;
-  for (int c = tid; c < kHeadDim * 16; c += 128) {
+  for (int c = tid; c < kHeadDim * 16; c += kBulkThreads) {
     const int r = c >> 4, col = (c & 15) * 8;
     *reinterpret_cast<uint4*>(Ts + r * kPad + col) = *reinterpret_cast<const uint4*>(T + r * kHeadDim + col);
   }
@@ -182,7 +240,7 @@ __global__ void __launch_bounds__(128) append_bulk_kernel(const AppendArgs a) {
   const int slab0 = blockIdx.x * kBulkSlab;
   for (int tile0 = slab0; tile0 < min(slab0 + kBulkSlab, a.n_new); tile0 += kBulkTile) {
     __syncthreads();  // previous tile fully consumed (and T_K stored on the first pass)
-    for (int c = tid; c < kBulkTile * 16; c += 128) {
+    for (int c = tid; c < kBulkTile * 16; c += kBulkThreads) {
       const int r = c >> 4, col = (c & 15) * 8;
       const int t = tile0 + r;
       uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
@@ -196,23 +254,25 @@ __global__ void __launch_bounds__(128) append_bulk_kernel(const AppendArgs a) {
     }
     __syncthreads();
 
-    // GEMM: warp w owns tile rows [16w, 16w+16): C[16][128] = K[16][128] * T^T
+    // GEMM: warp w owns tile rows [16*mw, 16*mw+16) and output columns [64*nw, 64*nw+64)
+    // (mw = w % 4, nw = w / 4): C[16][64] = K[16][128] * T^T
     {
-      float acc[16][4];
+      const int mw = warp & 3, nw = warp >> 2;
+      float acc[8][4];
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt)
+      for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-      const int arow = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);
+      const int arow = 16 * mw + (lane & 7) + 8 * ((lane >> 3) & 1);
       const int acol = 8 * (lane >> 4);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         uint32_t A[4];
         ldmatrix_x4(A, ks + arow * kPad + 16 * kk + acol);
 #pragma unroll
-        for (int np = 0; np < 8; ++np) {
+        for (int np = 0; np < 4; ++np) {
           uint32_t Bm[4];
-          const int brow = 8 * (2 * np + (lane >> 4)) + (lane & 7);
+          const int brow = 64 * nw + 8 * (2 * np + (lane >> 4)) + (lane & 7);
           const int bcol = 16 * kk + 8 * ((lane >> 3) & 1);
           ldmatrix_x4(Bm, Ts + brow * kPad + bcol);
           const uint32_t b0[2] = {Bm[0], Bm[1]};
@@ -221,38 +281,40 @@ __global__ void __launch_bounds__(128) append_bulk_kernel(const AppendArgs a) {
           mma_f16(acc[2 * np + 1], A, b1);
         }
       }
-      __syncwarp();
+      // every warp has read its rows of the k tile before any overwrites them with k'
+      __syncthreads();
       const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        const int col = 8 * nt + 2 * t4;
-        *reinterpret_cast<__half2*>(ks + (16 * warp + g) * kPad + col) = __floats2half2_rn(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<__half2*>(ks + (16 * warp + g + 8) * kPad + col) =
+      for (int nt = 0; nt < 8; ++nt) {
+        const int col = 64 * nw + 8 * nt + 2 * t4;
+        *reinterpret_cast<__half2*>(ks + (16 * mw + g) * kPad + col) = __floats2half2_rn(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<__half2*>(ks + (16 * mw + g + 8) * kPad + col) =
             __floats2half2_rn(acc[nt][2], acc[nt][3]);
       }
     }
     __syncthreads();
 
-    // route: threads 0..63 keys, 64..127 values
+    // route: row = tid / 2 (rows 0..63 keys, 64..127 values), two threads per row
     {
-      const int kind = tid >> 6;
-      const int r = tid & 63;
+      const int row = tid >> 1, part = tid & 1;
+      const int kind = row >> 6;
+      const int r = row & 63;
       const int t = tile0 + r;
       if (t < a.n_new) {
         const int p = S + t;
-        const __half* row = (kind ? vs : ks) + r * kPad;
+        const __half* src = (kind ? vs : ks) + r * kPad;
         if (p < a.s_sink) {
           __half* dst = (kind ? a.v_sink : a.k_sink) + ((size_t)unit * a.sink_dim + p) * kHeadDim;
-          for (int i = 0; i < 16; ++i)
-            reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(row)[i];
+          for (int i = 8 * part; i < 8 * part + 8; ++i)
+            reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
         } else if (p < sq_new) {
           const size_t rec = (size_t)unit * a.cap_alloc + p;
-          quantize_row<BITS, NSEL>(row, (kind ? a.v_codes : a.k_codes) + rec * CB,
-                                   (kind ? a.v_params : a.k_params) + rec, qs);
+          quantize_row_part<BITS, NSEL, 2>(src, part, (kind ? a.v_codes : a.k_codes) + rec * CB,
+                                           (kind ? a.v_params : a.k_params) + rec, qs);
         } else {
           __half* dst = (kind ? a.v_ring : a.k_ring) + ((size_t)unit * a.R + p % a.R) * kHeadDim;
-          for (int i = 0; i < 16; ++i)
-            reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(row)[i];
+          for (int i = 8 * part; i < 8 * part + 8; ++i)
+            reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
         }
       }
     }
@@ -280,7 +342,7 @@ __global__ void advance_state_kernel(const AppendArgs a) {
 template <int BITS, int NSEL>
 cudaError_t launch_append_t(const Derived& d, bool small, const AppendArgs& a, cudaStream_t st) {
   if (small) {
-    append_small_kernel<BITS, NSEL><<<d.units, 128, 0, st>>>(a);
+    append_small_kernel<BITS, NSEL, 0><<<d.units, 128, 0, st>>>(a);
     return cudaGetLastError();
   }
   flush_ring_kernel<BITS, NSEL><<<d.units, 128, 0, st>>>(a);
@@ -289,11 +351,31 @@ cudaError_t launch_append_t(const Derived& d, bool small, const AppendArgs& a, c
   e = ensure_smem_attr<append_bulk_kernel<BITS, NSEL>>((int)kBulkSmem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n_new + kBulkSlab - 1) / kBulkSlab, d.units);
-  append_bulk_kernel<BITS, NSEL><<<grid, 128, kBulkSmem, st>>>(a);
+  append_bulk_kernel<BITS, NSEL><<<grid, kBulkThreads, kBulkSmem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   advance_state_kernel<<<(d.units + 127) / 128, 128, 0, st>>>(a);
   return cudaGetLastError();
+}
+
+template <int BITS, int NSEL>
+cudaError_t launch_fused_t(const Derived& d, const AppendArgs& a, cudaStream_t st) {
+  switch (d.group) {
+    case 1: append_small_kernel<BITS, NSEL, 1><<<d.units, 256, 0, st>>>(a); break;
+    case 2: append_small_kernel<BITS, NSEL, 2><<<d.units, 256, 0, st>>>(a); break;
+    case 4: append_small_kernel<BITS, NSEL, 4><<<d.units, 256, 0, st>>>(a); break;
+    default: append_small_kernel<BITS, NSEL, 8><<<d.units, 256, 0, st>>>(a); break;
+  }
+  return cudaGetLastError();
+}
+
+template <int BITS>
+cudaError_t launch_fused_b(const Derived& d, const AppendArgs& a, cudaStream_t st) {
+  switch (d.nsel) {
+    case 2: return launch_fused_t<BITS, 2>(d, a, st);
+    case 3: return launch_fused_t<BITS, 3>(d, a, st);
+    default: return launch_fused_t<BITS, 4>(d, a, st);
+  }
 }
 
 template <int BITS>
@@ -309,6 +391,10 @@ cudaError_t launch_append_b(const Derived& d, bool small, const AppendArgs& a, c
 
 cudaError_t launch_append(const Derived& d, int bits, bool small, const AppendArgs& a, cudaStream_t st) {
   return bits == 2 ? launch_append_b<2>(d, small, a, st) : launch_append_b<4>(d, small, a, st);
+}
+
+cudaError_t launch_append_fused(const Derived& d, int bits, const AppendArgs& a, cudaStream_t st) {
+  return bits == 2 ? launch_fused_b<2>(d, a, st) : launch_fused_b<4>(d, a, st);
 }
 
 }  // namespace wushkv

@@ -5,24 +5,27 @@
 //
 // Two launches per call:
 //  1. decode_prologue (four CTAs per (sequence, KV head), a quarter of the dimensions
-//     each): q'_j = T_K^{-T} q_j for its g query heads in fp32, and the per-unit
-//     completion ticket reset.  It releases the main kernel at once (programmatic
-//     dependent launch), so the main kernel's KV stream starts while it runs; each
-//     consumer warp then re-expresses q' as a 31-bit fixed-point integer split into
-//     four signed 8-bit limbs, directly in the mma.sync B-fragment registers it needs.
-//  2. decode_main: grid (n_split, units).  Item s of a unit attends over positions
-//     [sL, (s+1)L) of the quantized region [S_sink, S_quant) and over its share of the
-//     unit's fp16 window positions (sink [0, S_sink) and recent [S_quant, S)).
+//     each): q'_j = T_K^{-T} q_j for its g query heads in fp32, and the reset of the
+//     unit's completion counters.  It releases the main kernel at once (programmatic
+//     dependent launch), so the main kernel's KV stream starts while it runs.  (In a
+//     fused step, wushkv_step, the append kernel does this work instead and the main
+//     kernel waits for it before reading anything.)
+//  2. decode_main: grid (n_split, units).  Work item s of a unit takes the s-th share of
+//     the unit's current quantized region [S_sink, S_quant) (whole 128-position stages)
+//     and of its fp16 window positions (sink [0, S_sink) and recent [S_quant, S)).
 //     The quantized positions stream through shared memory in 128-position stages
 //     (K codes, V codes, K and V (s, z)) via bulk copies on an mbarrier ring: one
-//     producer warp, four consumer warps, 32 positions per consumer warp per stage:
+//     producer warp, four consumer warps, 32 positions per consumer warp per stage.
+//     Each consumer warp re-expresses q' as a 31-bit fixed-point integer split into four
+//     signed 8-bit limbs, directly in the mma.sync B-fragment registers it needs:
 //       QK  : u8 codes x s8 query limbs on tensor cores (mma m16n8k32, exact int32),
 //             logit = log2e*scale*(z*sum(q') + s*sigma*D)  (dequantization folded);
-//       softmax: online, base 2, the running max rescales only when it grows;
+//       softmax: online, base 2, with a running max that may go stale by 2^8;
 //       PV  : fp16 codes x fp16 (p*s as hi + lo) on tensor cores (mma m16n8k16,
 //             fp32 accumulate), plus sum(p*z) for the zero-point term.
-//     Each item merges its warps and writes (m, l, o); the last item of a unit to
-//     finish (atomic ticket, no waiting) merges all items and writes the output.
+//     Each item merges its warps and writes (m, l, o); the last item of each group of
+//     items merges the group, the last group merges the groups and writes the output
+//     (atomic counters, nobody waits).
 //
 // Code unpacking needs no shifts on the key side: masking a packed 32-bit word with
 // 0x03030303 << 2j leaves, in each byte, one code times 4^j -- an exact u8 operand.
@@ -61,8 +64,6 @@ __device__ __forceinline__ float ex2(float x) {  // 2^x (hardware approximation,
   return y;
 }
 
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 template <int BITS>
 struct Cfg {
@@ -179,7 +180,11 @@ __global__ void __launch_bounds__(128) decode_prologue_kernel(const DecodeArgs a
     a.qprime[((size_t)unit * G + hh) * kHeadDim + 32 * c + q] =
         (part[0][hh][q] + part[1][hh][q]) + (part[2][hh][q] + part[3][hh][q]);
   }
-  if (c == 0 && tid == 0) a.tickets[unit] = 0u;
+  if (c == 0) {  // completion counters of the unit: its group counters, then the unit counter
+    const int ngroups = (a.n_split + kMergeGroup - 1) / kMergeGroup;
+    for (int i = tid; i < ngroups; i += 128) a.tickets[a.units + (size_t)unit * ngroups + i] = 0u;
+    if (tid == 0) a.tickets[unit] = 0u;
+  }
 }
 
 // The query-side B fragments of one lane, built in registers from q' (fp32, in global
@@ -530,9 +535,42 @@ __device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, 
 
 // fp16 window positions [wbeg, wend) of a unit, positions wbeg + warp, + 4, ...: exact
 // scalar path (lane = 4 dims), written to the window pseudo-warp slots of the merge area.
+// The rows of a batch of positions are loaded together (the first batch before
+// the kernel waits for q'), their G x batch logits are reduced as independent
+// shuffle chains, and the online softmax is updated once per batch.
+template <int G>
+struct WinRows {
+  static constexpr int KB = G >= 8 ? 2 : 4;  // positions per batch (registers bound it at G = 8)
+  uint2 k[KB], v[KB];
+};
+
+template <int G>
+__device__ __forceinline__ void window_load(const DecodeArgs& a, int unit, int it0, int wend, int n_sink, int r0,
+                                            int lane, WinRows<G>& w) {
+#pragma unroll
+  for (int u = 0; u < WinRows<G>::KB; ++u) {
+    const int it = it0 + u * kConsumers;
+    w.k[u] = w.v[u] = make_uint2(0u, 0u);
+    if (it < wend) {
+      const __half *kr, *vr;
+      if (it < n_sink) {
+        kr = a.k_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
+        vr = a.v_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
+      } else {
+        const int p = r0 + (it - n_sink);
+        kr = a.k_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
+        vr = a.v_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
+      }
+      w.k[u] = *reinterpret_cast<const uint2*>(kr + 4 * lane);
+      w.v[u] = *reinterpret_cast<const uint2*>(vr + 4 * lane);
+    }
+  }
+}
+
 template <int G>
 __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, int n_sink, int r0, int warp,
-                             int lane, Merge* mg, float* wpv) {
+                             int lane, WinRows<G>& w, Merge* mg, float* wpv) {
+  constexpr int KB = WinRows<G>::KB;
   float qv[G][4];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
@@ -549,50 +587,53 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
     l[hh] = 0.f;
     o[hh][0] = o[hh][1] = o[hh][2] = o[hh][3] = 0.f;
   }
-  constexpr int kBatch = G >= 8 ? 2 : (G >= 4 ? 4 : 8);  // positions whose loads are in flight at once
-  for (int it0 = wbeg + warp; it0 < wend; it0 += kBatch * kConsumers) {
-    uint2 kraw[kBatch], vraw[kBatch];
+  for (int it0 = wbeg + warp; it0 < wend; it0 += KB * kConsumers) {
+    if (it0 != wbeg + warp) window_load<G>(a, unit, it0, wend, n_sink, r0, lane, w);
+    float x[KB][G];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int it = it0 + u * kConsumers;
-      kraw[u] = vraw[u] = make_uint2(0u, 0u);
-      if (it < wend) {
-        const __half *kr, *vr;
-        if (it < n_sink) {
-          kr = a.k_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
-          vr = a.v_sink + ((size_t)unit * a.sink_dim + it) * kHeadDim;
-        } else {
-          const int p = r0 + (it - n_sink);
-          kr = a.k_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
-          vr = a.v_ring + ((size_t)unit * a.R + p % a.R) * kHeadDim;
-        }
-        kraw[u] = *reinterpret_cast<const uint2*>(kr + 4 * lane);
-        vraw[u] = *reinterpret_cast<const uint2*>(vr + 4 * lane);
+    for (int u = 0; u < KB; ++u) {
+      const float2 k01 = __half22float2(u32_as_h2(w.k[u].x)), k23 = __half22float2(u32_as_h2(w.k[u].y));
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        float xx = qv[hh][0] * k01.x;
+        xx = fmaf(qv[hh][1], k01.y, xx);
+        xx = fmaf(qv[hh][2], k23.x, xx);
+        x[u][hh] = fmaf(qv[hh][3], k23.y, xx);
       }
     }
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-    if (it0 + u * kConsumers >= wend) break;
-    const float2 k01 = __half22float2(u32_as_h2(kraw[u].x)), k23 = __half22float2(u32_as_h2(kraw[u].y));
-    const float2 v01 = __half22float2(u32_as_h2(vraw[u].x)), v23 = __half22float2(u32_as_h2(vraw[u].y));
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+      for (int u = 0; u < KB; ++u)
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) x[u][hh] += __shfl_xor_sync(0xffffffffu, x[u][hh], off);
+#pragma unroll
+    for (int u = 0; u < KB; ++u)
+      if (it0 + u * kConsumers >= wend)
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) x[u][hh] = -CUDART_INF_F;
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
-      float xx = qv[hh][0] * k01.x;
-      xx = fmaf(qv[hh][1], k01.y, xx);
-      xx = fmaf(qv[hh][2], k23.x, xx);
-      xx = fmaf(qv[hh][3], k23.y, xx);
+      float mn = m[hh];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) xx += __shfl_xor_sync(0xffffffffu, xx, off);
-      const float mn = fmaxf(m[hh], xx);
-      const float al = ex2(m[hh] - mn);
-      const float p = ex2(xx - mn);
-      l[hh] = fmaf(l[hh], al, p);
-      o[hh][0] = fmaf(o[hh][0], al, p * v01.x);
-      o[hh][1] = fmaf(o[hh][1], al, p * v01.y);
-      o[hh][2] = fmaf(o[hh][2], al, p * v23.x);
-      o[hh][3] = fmaf(o[hh][3], al, p * v23.y);
+      for (int u = 0; u < KB; ++u) mn = fmaxf(mn, x[u][hh]);
+      const float al = ex2(m[hh] - mn);  // 2^-inf = 0 on the first batch
+      l[hh] *= al;
+      o[hh][0] *= al;
+      o[hh][1] *= al;
+      o[hh][2] *= al;
+      o[hh][3] *= al;
+#pragma unroll
+      for (int u = 0; u < KB; ++u) {
+        const float p = ex2(x[u][hh] - mn);
+        const float2 v01 = __half22float2(u32_as_h2(w.v[u].x)), v23 = __half22float2(u32_as_h2(w.v[u].y));
+        l[hh] += p;
+        o[hh][0] = fmaf(p, v01.x, o[hh][0]);
+        o[hh][1] = fmaf(p, v01.y, o[hh][1]);
+        o[hh][2] = fmaf(p, v23.x, o[hh][2]);
+        o[hh][3] = fmaf(p, v23.y, o[hh][3]);
+      }
       m[hh] = mn;
-    }
     }
   }
 #pragma unroll
@@ -607,6 +648,60 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
     dst[1] = o[hh][1];
     dst[2] = o[hh][2];
     dst[3] = o[hh][3];
+  }
+}
+
+// Merge `count` consecutive partials (m, l, pad, pad, o[128] per head, base 2, o not yet
+// normalised) of one unit.  dst != nullptr: write the merged partial there; else write the
+// normalised output rows of the unit's G query heads.  wts: shared [count][G].
+template <int G>
+__device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, int count, float* dst,
+                               float* wts) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int hh = warp; hh < G; hh += kThreads / 32) {
+    float M = -CUDART_INF_F;
+    for (int it = lane; it < count; it += 32) M = fmaxf(M, __ldcg(src + ((size_t)it * G + hh) * kPartStride));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    for (int it = lane; it < count; it += 32) {
+      const float mi = __ldcg(src + ((size_t)it * G + hh) * kPartStride);
+      const float e = (M == -CUDART_INF_F) ? 0.f : exp2f(mi - M);
+      wts[it * G + hh] = e;
+      L = fmaf(e, __ldcg(src + ((size_t)it * G + hh) * kPartStride + 1), L);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    __syncwarp();
+    if (dst) {
+      if (lane == 0) {
+        dst[hh * kPartStride + 0] = M;
+        dst[hh * kPartStride + 1] = L;
+      }
+    } else {
+      const float invL = L > 0.f ? 1.0f / L : 0.f;
+      for (int it = lane; it < count; it += 32) wts[it * G + hh] *= invL;
+      if (lane == 0 && !(L > 0.f)) atomicOr(a.status, kStatusEmpty);
+    }
+  }
+  __syncthreads();
+  const int b = unit / a.Hkv, h = unit % a.Hkv;
+  for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
+    const int hh = idx / kHeadDim, d = idx % kHeadDim;
+    float acc = 0.f;
+    // every partial is finite (an empty one holds o = 0), so no term needs skipping
+#pragma unroll 4
+    for (int it = 0; it < count; ++it)
+      acc = fmaf(wts[it * G + hh], __ldcg(src + ((size_t)it * G + hh) * kPartStride + 4 + d), acc);
+    if (dst) {
+      dst[hh * kPartStride + 4 + d] = acc;
+    } else {
+      const size_t o = ((size_t)b * a.Hq + h * G + hh) * kHeadDim + d;
+      if (a.out_fp16)
+        reinterpret_cast<__half*>(a.out)[o] = __float2half_rn(acc);
+      else
+        reinterpret_cast<float*>(a.out)[o] = acc;
+    }
   }
 }
 
@@ -630,6 +725,7 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   const int g = lane >> 2, t4 = lane & 3;
   const int unit = blockIdx.y, item = blockIdx.x;
   const int nitems = a.n_split;
+  if (a.wait_all) griddep_wait();  // fused step: the append before this kernel writes the cache
   int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
   if (S < 0 || S > a.cap_alloc || Sq < 0 || Sq > S) {  // never read outside the buffers
     if (tid == 0 && item == 0) atomicOr(a.status, kStatusBadState);
@@ -698,9 +794,12 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     }
   } else {
     // ---------------- consumers
-    griddep_wait();  // q' fragments, constants and the ticket reset come from the prologue
-    // (a) this warp's share of the fp16 window, while the first tiles are in flight
-    window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, mg, wpv);
+    // (a) this warp's share of the fp16 window: the first rows are loaded before the wait
+    // for the prologue (they do not depend on it), the rest while the first tiles land
+    WinRows<G> wr;
+    window_load<G>(a, unit, wbeg + warp, wend, n_sink, r0, lane, wr);
+    griddep_wait();  // q', its constants and the counter resets come from the prologue
+    window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, wr, mg, wpv);
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) qs.o[mt][0] = qs.o[mt][1] = qs.o[mt][2] = qs.o[mt][3] = 0.f;
     // (b) quantized positions
@@ -786,61 +885,44 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
       part[hh * kPartStride + 1] = L;
     }
   }
+  // ======================= two-level merge: the last item of each group of kMergeGroup
+  // items merges the group; the last group to finish merges the groups and writes the
+  // output (atomic counters, nobody waits).  Neither level reads more than a few partials.
+  const int ngroups = (nitems + kMergeGroup - 1) / kMergeGroup;
+  const int grp = item / kMergeGroup;
+  const int g0 = grp * kMergeGroup, gn = min(kMergeGroup, nitems - g0);
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&a.tickets[unit], 1u) == (uint32_t)(nitems - 1)) ? 1u : 0u;
+  if (tid == 0) {
+    uint32_t* gt = a.tickets + a.units + (size_t)unit * ngroups + grp;
+    s_last = (atomicAdd(gt, 1u) == (uint32_t)(gn - 1)) ? 1u : 0u;
+  }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-
-  // ======================= last item of the unit: merge all items, write the output
-  const float* up = a.partials + (size_t)unit * nitems * G * kPartStride;
-  for (int hh = warp; hh < G; hh += kThreads / 32) {
-    float M = -CUDART_INF_F;
-    for (int it = lane; it < nitems; it += 32) M = fmaxf(M, __ldcg(up + ((size_t)it * G + hh) * kPartStride));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
-    for (int it = lane; it < nitems; it += 32) {
-      const float mi = __ldcg(up + ((size_t)it * G + hh) * kPartStride);
-      const float e = (M == -CUDART_INF_F) ? 0.f : exp2f(mi - M);
-      wts[it * G + hh] = e;
-      L = fmaf(e, __ldcg(up + ((size_t)it * G + hh) * kPartStride + 1), L);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    __syncwarp();
-    const float invL = L > 0.f ? 1.0f / L : 0.f;
-    for (int it = lane; it < nitems; it += 32) wts[it * G + hh] *= invL;
-    if (lane == 0 && !(L > 0.f)) atomicOr(a.status, kStatusEmpty);
+  const float* up = a.partials + ((size_t)unit * nitems + g0) * G * kPartStride;
+  if (ngroups == 1) {
+    merge_partials<G>(a, unit, up, gn, nullptr, wts);
+    return;
   }
+  float* gp = a.gpartials + ((size_t)unit * ngroups + grp) * G * kPartStride;
+  merge_partials<G>(a, unit, up, gn, gp, wts);
+  __threadfence();
   __syncthreads();
-  const int b = unit / a.Hkv, h = unit % a.Hkv;
-  for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
-    const int hh = idx / kHeadDim, d = idx % kHeadDim;
-    float acc = 0.f;
-    for (int it = 0; it < nitems; ++it) {
-      const float w = wts[it * G + hh];
-      if (w != 0.f) acc = fmaf(w, __ldcg(up + ((size_t)it * G + hh) * kPartStride + 4 + d), acc);
-    }
-    const size_t o = ((size_t)b * a.Hq + h * G + hh) * kHeadDim + d;
-    if (a.out_fp16)
-      reinterpret_cast<__half*>(a.out)[o] = __float2half_rn(acc);
-    else
-      reinterpret_cast<float*>(a.out)[o] = acc;
-  }
+  if (tid == 0) s_last = (atomicAdd(&a.tickets[unit], 1u) == (uint32_t)(ngroups - 1)) ? 1u : 0u;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  merge_partials<G>(a, unit, a.gpartials + (size_t)unit * ngroups * G * kPartStride, ngroups, nullptr, wts);
 }
 
+// The main kernel as the programmatic dependent of the kernel before it in the stream: it
+// may start before that kernel ends; whatever it reads from it is behind griddepcontrol.wait.
 template <int BITS, int G>
-cudaError_t launch_decode_t(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
-  decode_prologue_kernel<G><<<dim3(d.units, 4), 128, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+cudaError_t launch_main_t(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = Shared<BITS, G>::bytes(d.n_split);
-  e = ensure_smem_attr<decode_main_kernel<BITS, G>>((int)smem);
+  cudaError_t e = ensure_smem_attr<decode_main_kernel<BITS, G>>((int)smem);
   if (e != cudaSuccess) return e;
-  // programmatic dependent launch: the main kernel may start before the prologue ends; its
-  // consumers wait (griddepcontrol.wait) for the prologue's results, its producer does not
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(d.n_split, d.units);
   lc.blockDim = dim3(kThreads);
@@ -852,12 +934,32 @@ cudaError_t launch_decode_t(const Derived& d, const DecodeArgs& a, cudaStream_t 
   lc.attrs = attr;
   lc.numAttrs = 1;
   e = cudaLaunchKernelEx(&lc, decode_main_kernel<BITS, G>, a);
-  if (e != cudaSuccess) {
+  if (e != cudaSuccess) {  // without the attribute: plain stream order
     (void)cudaGetLastError();
     decode_main_kernel<BITS, G><<<lc.gridDim, kThreads, smem, st>>>(a);
     e = cudaGetLastError();
   }
   return e;
+}
+
+template <int BITS, int G>
+cudaError_t launch_decode_t(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
+  decode_prologue_kernel<G><<<dim3(d.units, 4), 128, 0, st>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the main kernel may start before the prologue ends; its consumers wait
+  // (griddepcontrol.wait) for the prologue's results, its producer does not
+  return launch_main_t<BITS, G>(d, a, st);
+}
+
+template <int BITS>
+cudaError_t launch_main_b(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
+  switch (d.group) {
+    case 1: return launch_main_t<BITS, 1>(d, a, st);
+    case 2: return launch_main_t<BITS, 2>(d, a, st);
+    case 4: return launch_main_t<BITS, 4>(d, a, st);
+    default: return launch_main_t<BITS, 8>(d, a, st);
+  }
 }
 
 template <int BITS>
@@ -874,6 +976,10 @@ cudaError_t launch_decode_b(const Derived& d, const DecodeArgs& a, cudaStream_t 
 
 cudaError_t launch_decode(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st) {
   return bits == 2 ? launch_decode_b<2>(d, a, st) : launch_decode_b<4>(d, a, st);
+}
+
+cudaError_t launch_decode_main(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st) {
+  return bits == 2 ? launch_main_b<2>(d, a, st) : launch_main_b<4>(d, a, st);
 }
 
 }  // namespace wushkv

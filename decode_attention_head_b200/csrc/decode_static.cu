@@ -66,7 +66,7 @@ extern "C" int wushkv_decode_attn_static(const wushkv_config* cfg, const wushkv_
   if (scratch_address(&ws) != cudaSuccess) return WUSHKV_ECUDA;
   // The array keeps whatever the previous call (of any configuration) left in it; the
   // completion counters of the split merge must start at zero.
-  if (cudaMemsetAsync(static_cast<unsigned char*>(ws) + d.ws_tickets, 0, (size_t)d.units * sizeof(uint32_t),
+  if (cudaMemsetAsync(static_cast<unsigned char*>(ws) + d.ws_tickets, 0, d.ws_qprime - d.ws_tickets,
                       static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return WUSHKV_ECUDA;
   return wushkv_decode_attn(cfg, cache, q, t_k_inv, softmax_scale, out_fp16, out, ws, stream);

@@ -15,11 +15,12 @@ constexpr int kB200SMs = 148;         // split policy sizes the decode grid for 
 // registers to this): 8 query heads per KV head need more registers than the others.
 constexpr int decode_ctas_per_sm(int group) { return group == 8 ? 3 : 4; }
 constexpr int kMaxSplits = 255;       // quantized work items per (sequence, KV head)
+constexpr int kMergeGroup = 16;       // work items merged together at the first merge level
 
 struct Derived {
   int units;        // B * H_kv
   int group;        // H_q / H_kv
-  int cap_alloc;    // capacity rounded up to 64
+  int cap_alloc;    // capacity rounded up to 128
   int ring;         // ring slots
   int sink_dim;     // max(s_sink, 1)
   int code_bytes;   // 16 * bits
@@ -28,7 +29,7 @@ struct Derived {
   float f_lo, f_hi;
   int n_split, split_tokens;
   // workspace offsets (bytes)
-  size_t ws_tickets, ws_qprime, ws_partials, ws_total;
+  size_t ws_tickets, ws_qprime, ws_partials, ws_gpartials, ws_total;
   // cache buffer sizes (bytes)
   size_t codes_bytes, params_bytes, sink_bytes, ring_bytes, state_bytes;
 };
@@ -53,6 +54,13 @@ struct AppendArgs {
   const __half* t_k;
   int i_lo, i_hi;
   float f_lo, f_hi;
+  // decode preparation fused into a one-token append (wushkv_step): q' = T_K^{-T} q of the
+  // unit's query heads into the decode workspace, and its completion counters reset
+  const __half* q;
+  const float* t_k_inv;
+  float* qprime;
+  uint32_t* tickets;
+  int Hq, ngroups;
 };
 
 struct DecodeArgs {
@@ -72,9 +80,12 @@ struct DecodeArgs {
   float scale_log2;  // softmax_scale * log2(e)
   void* out;
   int out_fp16;
-  uint32_t* tickets;
+  int units;
+  uint32_t* tickets;   // [units] unit counters, then [units][ngroups] group counters
   float* qprime;
-  float* partials;
+  float* partials;     // [units][n_split][G][132]
+  float* gpartials;    // [units][ngroups][G][132]
+  int wait_all;        // 1: the preceding kernel writes the cache (fused step): wait before any read
 };
 
 // Raise a kernel's dynamic shared-memory limit once per device (a function attribute,
@@ -94,5 +105,10 @@ cudaError_t ensure_smem_attr(int bytes) {
 
 cudaError_t launch_append(const Derived& d, int bits, bool small, const AppendArgs& a, cudaStream_t st);
 cudaError_t launch_decode(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st);
+// wushkv_step's one-token path: the small append fused with the decode prologue (it lets
+// its dependents launch early), then the main decode kernel alone, launched as that
+// kernel's programmatic dependent (it waits for it before reading anything).
+cudaError_t launch_append_fused(const Derived& d, int bits, const AppendArgs& a, cudaStream_t st);
+cudaError_t launch_decode_main(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st);
 
 }  // namespace wushkv

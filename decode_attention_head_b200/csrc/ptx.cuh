@@ -57,6 +57,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   return true;
 }
 
+// Named barrier `id` over `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Programmatic dependent launch: a kernel lets the next kernel in its stream start
+// (launch_dependents); the dependent blocks until this grid has completed and its memory
+// operations are visible (wait).  Without a programmatic dependency both are no-ops.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Bulk global -> shared copy completing on an mbarrier (no multicast).  dst, src and
 // bytes must be multiples of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

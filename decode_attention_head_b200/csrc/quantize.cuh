@@ -179,4 +179,110 @@ __device__ __noinline__ void quantize_row(const __half* __restrict__ x, uint8_t*
   *params_out = h2_as_u32(__halves2half2(s_h, z_h));
 }
 
+// The same quantizer with one row split over P adjacent lanes (P = 2 or 4; lanes
+// P*k .. P*k+P-1 of a warp, all active together): lane `part` takes values
+// [part*128/P, (part+1)*128/P), keeps its own NSEL smallest / largest, the lists are merged
+// over log2(P) xor-shuffle rounds (every lane ends with the same order statistics, so
+// every lane computes the same s and z), and each lane quantizes and writes its own
+// slice of the packed codes (16*BITS/P bytes); part 0 writes (s, z).
+template <int BITS, int NSEL, int P>
+__device__ __forceinline__ void quantize_row_part(const __half* __restrict__ x, int part,
+                                                  uint8_t* __restrict__ codes_out,
+                                                  uint32_t* __restrict__ params_out, const QuantSpec qs) {
+  static_assert(P == 2 || P == 4, "two or four lanes per row");
+  constexpr int V = 128 / P;  // values of this lane
+  constexpr int H = V / 2;    // half2 of this lane
+  __half2 v[H];
+  const uint4* src = reinterpret_cast<const uint4*>(x + part * V);
+#pragma unroll
+  for (int i = 0; i < V / 8; ++i) {
+    uint4 u = src[i];
+    v[4 * i + 0] = u32_as_h2(u.x);
+    v[4 * i + 1] = u32_as_h2(u.y);
+    v[4 * i + 2] = u32_as_h2(u.z);
+    v[4 * i + 3] = u32_as_h2(u.w);
+  }
+  const __half2 pinf = __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));
+  const __half2 ninf = __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));
+  __half2 a[NSEL], b[NSEL];
+#pragma unroll
+  for (int j = 0; j < NSEL; ++j) {
+    a[j] = pinf;
+    b[j] = ninf;
+  }
+#pragma unroll
+  for (int i = 0; i < H; ++i) {
+    insert_small<NSEL>(a, v[i]);
+    insert_large<NSEL>(b, v[i]);
+  }
+  float lo_s[NSEL], lo_t[NSEL], hi_s[NSEL], hi_t[NSEL];
+#pragma unroll
+  for (int j = 0; j < NSEL; ++j) {
+    lo_s[j] = __low2float(a[j]);
+    lo_t[j] = __high2float(a[j]);
+    hi_s[j] = __low2float(b[j]);
+    hi_t[j] = __high2float(b[j]);
+  }
+  merge_small<NSEL>(lo_s, lo_t);
+  merge_large<NSEL>(hi_s, hi_t);
+  const int lane = threadIdx.x & 31;
+  const unsigned group = ((1u << P) - 1u) << (lane & ~(P - 1));
+#pragma unroll
+  for (int off = 1; off < P; off <<= 1) {
+#pragma unroll
+    for (int j = 0; j < NSEL; ++j) {
+      lo_t[j] = __shfl_xor_sync(group, lo_s[j], off);
+      hi_t[j] = __shfl_xor_sync(group, hi_s[j], off);
+    }
+    merge_small<NSEL>(lo_s, lo_t);
+    merge_large<NSEL>(hi_s, hi_t);
+  }
+  float slo0 = 0.f, slo1 = 0.f, shi0 = 0.f, shi1 = 0.f;
+  const int jh0 = 127 - qs.i_hi;
+  const int jh1 = 127 - min(qs.i_hi + 1, 127);
+#pragma unroll
+  for (int j = 0; j < NSEL; ++j) {
+    if (j == qs.i_lo) slo0 = lo_s[j];
+    if (j == qs.i_lo + 1) slo1 = lo_s[j];
+    if (j == jh0) shi0 = hi_s[j];
+    if (j == jh1) shi1 = hi_s[j];
+  }
+  const float lo = interp(slo0, slo1, qs.f_lo);
+  const float hi = interp(shi0, shi1, qs.f_hi);
+  const float scale32 = __fdiv_rn(__fsub_rn(hi, lo), float((1 << BITS) - 1));
+  const __half s_h = __float2half_rn(scale32);
+  const __half z_h = __float2half_rn(lo);
+  const float sf = __half2float(s_h);
+  const float zf = __half2float(z_h);
+
+  constexpr int NW = 4 * BITS / P;  // 32-bit words of this lane's packed codes
+  uint32_t w[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) w[i] = 0u;
+  if (sf != 0.0f) {
+    const float rcp = __frcp_rn(sf);
+#pragma unroll
+    for (int k = 0; k < H; ++k) {
+      const float2 f = __half22float2(v[k]);
+      const uint32_t c0 = quantize_one<BITS>(f.x, zf, sf, rcp);
+      const uint32_t c1 = quantize_one<BITS>(f.y, zf, sf, rcp);
+      if (BITS == 2) {
+        w[k / 8] |= (c0 | (c1 << 2)) << (4 * (k % 8));
+      } else {
+        w[k / 4] |= (c0 | (c1 << 4)) << (8 * (k % 4));
+      }
+    }
+  }
+  uint8_t* dst = codes_out + part * (NW * 4);
+  if (NW % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < NW / 4; ++i)
+      reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < NW / 2; ++i) reinterpret_cast<uint2*>(dst)[i] = make_uint2(w[2 * i], w[2 * i + 1]);
+  }
+  if (part == 0) *params_out = h2_as_u32(__halves2half2(s_h, z_h));
+}
+
 }  // namespace wushkv

@@ -168,6 +168,18 @@ int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* cache, cons
                        const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
                        void* workspace, void* stream);
 
+/* One decode step: wushkv_append(k_new, v_new, n_new) followed by wushkv_decode_attn(q) on
+ * the same stream, with the same arguments, buffers and results as those two calls
+ * (§4.4: the new tokens are appended in full precision and serve the step's attention).
+ * With n_new <= chunk_max the append also prepares the decode (the compensated queries and
+ * the workspace's counters) and the decode kernel is launched as its programmatic
+ * dependent, so the step costs two kernel launches instead of three.  The decode of a
+ * sequence whose append is refused (STATUS_OVERFLOW) attends over its cache unchanged.
+ * Returns WUSHKV_OK, WUSHKV_EINVAL, WUSHKV_EUNSUPPORTED or WUSHKV_ECUDA. */
+int wushkv_step(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
+                int32_t n_new, const void* t_k, const void* q, const float* t_k_inv, float softmax_scale,
+                int32_t out_fp16, void* out, void* workspace, void* stream);
+
 /* wushkv_decode_attn with library-owned scratch instead of a caller-allocated workspace.
  * The method has no counterpart of this call: it serves callers that cannot allocate
  * device memory when they decode (a runtime without an allocator, a step that must not

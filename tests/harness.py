@@ -130,6 +130,29 @@ def assert_attention_close(gpu: np.ndarray, ref: np.ndarray, atol=ATOL, rtol=RTO
     return float(err.max()), float(rel.max())
 
 
+def oracle_cache_from_gpu(gc) -> ocache.Cache:
+    """An oracle cache holding exactly the GPU cache's contents (state, codes, (s, z), fp16
+    windows), so that decode parity is measured on an identical cache."""
+    cfg, L = gc.cfg, gc.layout
+    g = download(gc)
+    oc = ocache.Cache(cfg.batch, cfg.n_kv_heads, 128, cfg.bits, cfg.p_lo, cfg.p_hi, cfg.s_sink, cfg.s_keep,
+                      cfg.s_flush, capacity=L.cap_alloc, chunk_max=cfg.chunk_max)
+    for b in range(cfg.batch):
+        S, Sq = int(g["S"][b].max()), int(g["Sq"][b].max())
+        assert (g["S"][b] == S).all() and (g["Sq"][b] == Sq).all()
+        oc.S[b], oc.S_quant[b] = S, Sq
+        for kind in ("k", "v"):
+            getattr(oc, f"{kind}_codes")[b] = g[f"{kind}_codes"][b]
+            getattr(oc, f"{kind}_s")[b] = g[f"{kind}_s"][b]
+            getattr(oc, f"{kind}_z")[b] = g[f"{kind}_z"][b]
+            store = getattr(oc, f"{kind}_store")
+            ns = min(cfg.s_sink, S)
+            store[b, :, :ns] = g[f"{kind}_sink"][b][:, :ns]
+            rpos = np.arange(max(Sq, cfg.s_sink), S)
+            store[b][:, rpos] = g[f"{kind}_ring"][b][:, rpos % L.ring_slots]
+    return oc
+
+
 def oracle_decode(oc, q_np, T_K_np, scale):
     return oatt.decode(oc, q_np, T_K_np, scale)
 

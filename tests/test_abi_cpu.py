@@ -69,6 +69,9 @@ def test_bad_pointers_rejected_before_device_work(bnd):
     rc = bnd.lib.wushkv_decode_attn(ctypes.byref(cfg), ctypes.byref(bufs), None, None, ctypes.c_float(0.1), 0,
                                     None, None, None)
     assert rc == bnd.EINVAL
+    rc = bnd.lib.wushkv_step(ctypes.byref(cfg), ctypes.byref(bufs), None, None, 1, None, None, None,
+                             ctypes.c_float(0.1), 0, None, None, None)
+    assert rc == bnd.EINVAL
     rc = bnd.lib.wushkv_decode_attn_static(ctypes.byref(cfg), ctypes.byref(bufs), None, None, ctypes.c_float(0.1),
                                            0, None, None)
     assert rc == bnd.EINVAL

@@ -78,3 +78,26 @@ def test_state_mirror_tracks_the_oracle_flush(sink, keep, flush):
         assert nbytes == nf * (512 + 2 * 36) + 1024 + 128 * 128 * 2
         nq = max(m.Sq - sink, 0)
         assert m.decode_bytes() == nq * 72 + (m.S - nq) * 512 + 4 * 768 + 128 * 128 * 4
+
+
+@pytest.mark.parametrize("S0,n", [(300, 170), (100, 33), (37, 500)])
+def test_bulk_append_bytes_follow_the_oracle_flush(S0, n):
+    """The prefill byte count's flush (positions quantized, ring entries re-read, tokens kept
+    fp16) matches the oracle cache's state change on the same bulk append."""
+    sink, keep, flush = 4, 32, 16
+    wl = synth.scaled(synth.WORKLOADS["tiny"], batch=1, n_kv_heads=1, n_q_heads=4, s_sink=sink, s_keep=keep,
+                      s_flush=flush)
+    oc = ocache.Cache(1, 1, 128, 2, 1.0, 99.0, sink, keep, flush, capacity=2000, chunk_max=1)
+    T = np.eye(128, dtype=np.float16)[None]
+    x = np.random.default_rng(1).standard_normal((1, S0 + n, 1, 128)).astype(np.float16)
+    for p in range(S0):  # decode-style appends up to S0 (deferred flushes)
+        oc.append(x[:, p:p + 1], x[:, p:p + 1], T)
+    S, Sq = int(oc.S[0]), int(oc.S_quant[0])
+    oc.append(x[:, S0:], x[:, S0:], T)
+    lo0 = max(Sq, sink)
+    nq = int(oc.S_quant[0]) - lo0 if int(oc.S_quant[0]) > Sq else 0
+    from_ring = max(0, min(lo0 + nq, S) - lo0)
+    kept = S + n - max(lo0 + nq, S)
+    expect = n * 512 + from_ring * 512 + nq * 72 + kept * 512 + 128 * 128 * 2
+    assert bench.bulk_append_bytes(wl, S, Sq, n) == expect
+    assert int(oc.S[0]) == S + n
