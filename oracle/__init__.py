@@ -16,8 +16,11 @@ Modules:
   cache      -- the cache with full-precision sink / recent windows (Alg. 2 prose)
   attention  -- query compensation and exact-softmax decode attention
   footprint  -- the pages' cache-size arithmetic
+  rope       -- per-head RMSNorm and rotate-half RoPE of the path's raw inputs
+  transform  -- the normalised Walsh-Hadamard key transform
 
 Parity status: every function is pinned by a ``-m "not gpu"`` test in
-``tests/test_oracle_pins.py``; none is "parity unpinned".
+``tests/test_oracle_pins.py``, ``tests/test_oracle_rope.py`` and
+``tests/test_oracle_transform.py``; none is "parity unpinned".
 """
-from . import quantizer, cache, attention, footprint  # noqa: F401
+from . import quantizer, cache, attention, footprint, rope, transform  # noqa: F401
