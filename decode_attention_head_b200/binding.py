@@ -19,15 +19,24 @@ STATIC_SCRATCH_BYTES = 8 << 20  # WUSHKV_STATIC_SCRATCH_BYTES
 STATUS_OVERFLOW, STATUS_EMPTY, STATUS_TIMEOUT, STATUS_BADSTATE = 1, 2, 4, 8
 _ERR = {EINVAL: "invalid argument", EUNSUPPORTED: "unsupported configuration", ECUDA: "CUDA launch failed",
         ESINGULAR: "singular key transform", ESCRATCH: "needs more than the static scratch array holds"}
-SYMBOLS = ("wushkv_pack_layout", "wushkv_compensation", "wushkv_append", "wushkv_decode_attn",
-           "wushkv_step", "wushkv_decode_attn_static")
+SYMBOLS = ("wushkv_pack_layout", "wushkv_compensation", "wushkv_hadamard", "wushkv_append", "wushkv_decode_attn",
+           "wushkv_step", "wushkv_step_prep", "wushkv_decode_attn_static")
+
+
+class Prep(ctypes.Structure):
+    _fields_ = [("rope_theta", ctypes.c_float), ("q_norm_gain", ctypes.c_void_p), ("k_norm_gain", ctypes.c_void_p),
+                ("norm_eps", ctypes.c_float)]
 
 
 class Config(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("bits", ctypes.c_int32), ("capacity", ctypes.c_int32),
                 ("s_sink", ctypes.c_int32), ("s_keep", ctypes.c_int32), ("s_flush", ctypes.c_int32),
-                ("chunk_max", ctypes.c_int32), ("p_lo", ctypes.c_float), ("p_hi", ctypes.c_float)]
+                ("chunk_max", ctypes.c_int32), ("p_lo", ctypes.c_float), ("p_hi", ctypes.c_float),
+                ("transform", ctypes.c_int32)]
+
+
+TRANSFORM_DENSE, TRANSFORM_HADAMARD = 0, 1
 
 
 class Layout(ctypes.Structure):
@@ -53,6 +62,7 @@ def _load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     lib.wushkv_pack_layout.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Layout)]
     lib.wushkv_compensation.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]
+    lib.wushkv_hadamard.argtypes = [ctypes.c_int32, ctypes.c_void_p]
     lib.wushkv_append.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
                                   ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
     lib.wushkv_decode_attn.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
@@ -61,6 +71,10 @@ def _load() -> ctypes.CDLL:
     lib.wushkv_step.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p, ctypes.c_void_p,
                                 ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                 ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    lib.wushkv_step_prep.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
+                                     ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
+                                     ctypes.c_void_p, ctypes.POINTER(Prep), ctypes.c_void_p]
     lib.wushkv_decode_attn_static.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
                                               ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
                                               ctypes.c_void_p]
@@ -78,9 +92,9 @@ def _check(rc: int, what: str) -> None:
 
 
 def make_config(batch, n_kv_heads, n_q_heads, bits, capacity, s_sink, s_keep, s_flush=16, chunk_max=1,
-                p_lo=1.0, p_hi=99.0, head_dim=128) -> Config:
+                p_lo=1.0, p_hi=99.0, head_dim=128, transform=TRANSFORM_DENSE) -> Config:
     return Config(batch, n_kv_heads, n_q_heads, head_dim, bits, capacity, s_sink, s_keep, s_flush, chunk_max,
-                  p_lo, p_hi)
+                  p_lo, p_hi, transform)
 
 
 def pack_layout(cfg: Config) -> Layout:
@@ -95,6 +109,17 @@ def compensation(t_k: torch.Tensor) -> torch.Tensor:
     out = torch.empty(t.shape, dtype=torch.float32)
     _check(lib.wushkv_compensation(t.data_ptr(), t.shape[0], out.data_ptr()), "wushkv_compensation")
     return out
+
+
+def hadamard_compensation(n_kv_heads: int) -> torch.Tensor:
+    """T_K^{-1} (fp32, host) of the in-kernel Hadamard transform: H itself (wushkv_hadamard)."""
+    out = torch.empty(n_kv_heads, 128, 128, dtype=torch.float32)
+    _check(lib.wushkv_hadamard(n_kv_heads, out.data_ptr()), "wushkv_hadamard")
+    return out
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return t.data_ptr() if t is not None else None
 
 
 def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
@@ -143,7 +168,7 @@ class KVCache:
         """k_new, v_new: fp16 [B, n_new, H_kv, 128] on the device; t_k fp16 [H_kv, 128, 128]."""
         n_new = k_new.shape[1]
         _check(lib.wushkv_append(ctypes.byref(self.cfg), ctypes.byref(self.bufs), k_new.data_ptr(),
-                                 v_new.data_ptr(), n_new, t_k.data_ptr(), _stream_ptr(stream)), "wushkv_append")
+                                 v_new.data_ptr(), n_new, _ptr(t_k), _stream_ptr(stream)), "wushkv_append")
 
     def decode_attn(self, q: torch.Tensor, t_k_inv: torch.Tensor, softmax_scale: float,
                     out: Optional[torch.Tensor] = None, out_fp16: bool = False, stream=None) -> torch.Tensor:
@@ -163,10 +188,29 @@ class KVCache:
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float16 if out_fp16 else torch.float32, device=q.device)
         _check(lib.wushkv_step(ctypes.byref(self.cfg), ctypes.byref(self.bufs), k_new.data_ptr(), v_new.data_ptr(),
-                               k_new.shape[1], t_k.data_ptr(), q.data_ptr(), t_k_inv.data_ptr(), float(softmax_scale),
+                               k_new.shape[1], _ptr(t_k), q.data_ptr(), t_k_inv.data_ptr(), float(softmax_scale),
                                1 if out.dtype == torch.float16 else 0, out.data_ptr(), self.workspace.data_ptr(),
                                _stream_ptr(stream)),
                "wushkv_step")
+        return out
+
+    def step_prep(self, k_raw: torch.Tensor, v_new: torch.Tensor, t_k: torch.Tensor, q_raw: torch.Tensor,
+                  t_k_inv: torch.Tensor, softmax_scale: float, rope_theta: float,
+                  q_norm_gain: Optional[torch.Tensor] = None, k_norm_gain: Optional[torch.Tensor] = None,
+                  norm_eps: float = 1e-6, out: Optional[torch.Tensor] = None, out_fp16: bool = False,
+                  stream=None) -> torch.Tensor:
+        """step() on raw projections: per-head RMSNorm (gains given) and RoPE inside the
+        library's kernels (wushkv_step_prep).  Gains: fp16 [128] on the device."""
+        if out is None:
+            out = torch.empty(q_raw.shape, dtype=torch.float16 if out_fp16 else torch.float32, device=q_raw.device)
+        prep = Prep(float(rope_theta), q_norm_gain.data_ptr() if q_norm_gain is not None else None,
+                    k_norm_gain.data_ptr() if k_norm_gain is not None else None, float(norm_eps))
+        _check(lib.wushkv_step_prep(ctypes.byref(self.cfg), ctypes.byref(self.bufs), k_raw.data_ptr(),
+                                    v_new.data_ptr(), k_raw.shape[1], _ptr(t_k), q_raw.data_ptr(),
+                                    t_k_inv.data_ptr(), float(softmax_scale), 1 if out.dtype == torch.float16 else 0,
+                                    out.data_ptr(), self.workspace.data_ptr(), ctypes.byref(prep),
+                                    _stream_ptr(stream)),
+               "wushkv_step_prep")
         return out
 
     def decode_attn_static(self, q: torch.Tensor, t_k_inv: torch.Tensor, softmax_scale: float,

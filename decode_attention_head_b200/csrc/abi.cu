@@ -23,6 +23,7 @@ int derive(const wushkv_config* cfg, Derived* d) {
   if (g != 1 && g != 2 && g != 4 && g != 8) return WUSHKV_EUNSUPPORTED;
   if (cfg->s_sink < 0 || cfg->s_keep < 0 || cfg->s_flush < 1 || cfg->chunk_max < 1) return WUSHKV_EINVAL;
   if (!(cfg->p_lo >= 0.f) || !(cfg->p_hi <= 100.f) || !(cfg->p_lo < cfg->p_hi)) return WUSHKV_EINVAL;
+  if (cfg->transform != WUSHKV_TRANSFORM_DENSE && cfg->transform != WUSHKV_TRANSFORM_HADAMARD) return WUSHKV_EINVAL;
   const long long units = (long long)cfg->batch * cfg->n_kv_heads;
   if (units > (1 << 24) || cfg->capacity > (1 << 28)) return WUSHKV_EINVAL;
 
@@ -194,6 +195,7 @@ static void fill_append(const wushkv_config* cfg, const Derived& d, const wushkv
   a->f_hi = d.f_hi;
   a->Hq = cfg->n_q_heads;
   a->ngroups = ceil_div(d.n_split, kMergeGroup);
+  a->transform = cfg->transform;
 }
 
 static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv_cache* cache, const void* q,
@@ -233,9 +235,10 @@ static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv
   a->wait_all = 0;
 }
 
-static int check_append(const wushkv_cache* cache, const void* k_new, const void* v_new, int32_t n_new,
-                        const void* t_k) {
-  if (!cache_ok(cache) || n_new < 0 || !aligned16(t_k)) return WUSHKV_EINVAL;
+static int check_append(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
+                        int32_t n_new, const void* t_k) {
+  if (!cache_ok(cache) || n_new < 0) return WUSHKV_EINVAL;
+  if (cfg->transform == WUSHKV_TRANSFORM_DENSE && !aligned16(t_k)) return WUSHKV_EINVAL;
   if (n_new > 0 && (!aligned16(k_new) || !aligned16(v_new))) return WUSHKV_EINVAL;
   return WUSHKV_OK;
 }
@@ -248,12 +251,22 @@ static int check_decode(const wushkv_cache* cache, const void* q, const float* t
   return WUSHKV_OK;
 }
 
+extern "C" int wushkv_hadamard(int32_t n_kv_heads, float* t_k_inv) {
+  if (!t_k_inv || n_kv_heads < 1) return WUSHKV_EINVAL;
+  const float c = (float)(1.0 / std::sqrt((double)kHeadDim));
+  for (int h = 0; h < n_kv_heads; ++h)
+    for (int r = 0; r < kHeadDim; ++r)
+      for (int i = 0; i < kHeadDim; ++i)
+        t_k_inv[((size_t)h * kHeadDim + r) * kHeadDim + i] = (__builtin_popcount(r & i) & 1) ? -c : c;
+  return WUSHKV_OK;
+}
+
 extern "C" int wushkv_append(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new,
                              const void* v_new, int32_t n_new, const void* t_k, void* stream) {
   Derived d;
   int rc = derive(cfg, &d);
   if (rc != WUSHKV_OK) return rc;
-  rc = check_append(cache, k_new, v_new, n_new, t_k);
+  rc = check_append(cfg, cache, k_new, v_new, n_new, t_k);
   if (rc != WUSHKV_OK) return rc;
   AppendArgs a;
   fill_append(cfg, d, cache, k_new, v_new, n_new, t_k, &a);
@@ -276,21 +289,36 @@ extern "C" int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* 
   return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA;
 }
 
-extern "C" int wushkv_step(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
-                           int32_t n_new, const void* t_k, const void* q, const float* t_k_inv, float softmax_scale,
-                           int32_t out_fp16, void* out, void* workspace, void* stream) {
+static int step_impl(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
+                     int32_t n_new, const void* t_k, const void* q, const float* t_k_inv, float softmax_scale,
+                     int32_t out_fp16, void* out, void* workspace, const wushkv_prep* prep, void* stream) {
   Derived d;
   int rc = derive(cfg, &d);
   if (rc != WUSHKV_OK) return rc;
-  rc = check_append(cache, k_new, v_new, n_new, t_k);
+  rc = check_append(cfg, cache, k_new, v_new, n_new, t_k);
   if (rc != WUSHKV_OK) return rc;
   rc = check_decode(cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace);
   if (rc != WUSHKV_OK) return rc;
+  PrepSpec ps;
+  std::memset(&ps, 0, sizeof(ps));
+  if (prep) {
+    if (!(prep->rope_theta > 1.0f) || !std::isfinite(prep->rope_theta)) return WUSHKV_EINVAL;
+    if ((prep->q_norm_gain || prep->k_norm_gain) && !(prep->norm_eps > 0.0f)) return WUSHKV_EINVAL;
+    if ((prep->q_norm_gain && !aligned16(prep->q_norm_gain)) || (prep->k_norm_gain && !aligned16(prep->k_norm_gain)))
+      return WUSHKV_EINVAL;
+    ps.enabled = 1;
+    ps.log2_theta = std::log2((double)prep->rope_theta);
+    ps.q_gain = static_cast<const __half*>(prep->q_norm_gain);
+    ps.k_gain = static_cast<const __half*>(prep->k_norm_gain);
+    ps.eps = prep->norm_eps;
+  }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   AppendArgs aa;
   fill_append(cfg, d, cache, k_new, v_new, n_new, t_k, &aa);
+  aa.prep = ps;
   DecodeArgs da;
   fill_decode(cfg, d, cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace, &da);
+  da.prep = ps;
   cudaError_t e;
   if (n_new <= cfg->chunk_max) {
     // one kernel appends and prepares the decode (q', counters); the main decode kernel
@@ -309,4 +337,20 @@ extern "C" int wushkv_step(const wushkv_config* cfg, const wushkv_cache* cache, 
     if (e == cudaSuccess) e = launch_decode(d, cfg->bits, da, st);
   }
   return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA;
+}
+
+extern "C" int wushkv_step(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
+                           int32_t n_new, const void* t_k, const void* q, const float* t_k_inv, float softmax_scale,
+                           int32_t out_fp16, void* out, void* workspace, void* stream) {
+  return step_impl(cfg, cache, k_new, v_new, n_new, t_k, q, t_k_inv, softmax_scale, out_fp16, out, workspace, nullptr,
+                   stream);
+}
+
+extern "C" int wushkv_step_prep(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_raw,
+                                const void* v_new, int32_t n_new, const void* t_k, const void* q_raw,
+                                const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
+                                void* workspace, const wushkv_prep* prep, void* stream) {
+  if (!prep) return WUSHKV_EINVAL;
+  return step_impl(cfg, cache, k_raw, v_new, n_new, t_k, q_raw, t_k_inv, softmax_scale, out_fp16, out, workspace, prep,
+                   stream);
 }

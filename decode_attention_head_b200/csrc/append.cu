@@ -79,7 +79,7 @@ __device__ void quantize_ring_range(const AppendArgs& a, int unit, int p_begin, 
 // 4*lane .. 4*lane+3 (all 32 float4 loads in flight at once), the warps' partial sums meet
 // in shared memory.  Also resets the unit's decode completion counters.
 template <int G>
-__device__ void prepare_query(const AppendArgs& a, int unit, int tid) {
+__device__ void prepare_query(const AppendArgs& a, int unit, int tid, int qpos) {
   __shared__ float qs[G][kHeadDim];
   __shared__ float red[4][G][kHeadDim];
   const int b = unit / a.Hkv, h = unit % a.Hkv;
@@ -91,6 +91,10 @@ __device__ void prepare_query(const AppendArgs& a, int unit, int tid) {
   for (int u = 0; u < 32; ++u) t[u] = __ldg(Ti + (size_t)u * (kHeadDim / 4));
   for (int i = tid; i < G * kHeadDim; i += 128)
     qs[i / kHeadDim][i % kHeadDim] = __half2float(a.q[((size_t)b * a.Hq + h * G) * kHeadDim + i]);
+  if (a.prep.enabled) {  // raw queries: RMSNorm + RoPE at the query's position, head by head
+    bar_sync(2, 128);
+    for (int hh = warp; hh < G; hh += 4) prep_head_warp(qs[hh], a.prep.q_gain, a.prep, qpos, lane);
+  }
   bar_sync(2, 128);
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
@@ -121,25 +125,29 @@ __device__ void prepare_query(const AppendArgs& a, int unit, int tid) {
 // separate named barriers (1: append, 2: decode preparation).
 template <int BITS, int NSEL, int G>
 __global__ void __launch_bounds__(G > 0 ? 256 : 128) append_small_kernel(const AppendArgs a) {
-  if (G > 0) {
-    griddep_launch();  // the decode kernel may launch now; it waits for this whole grid
-    if (threadIdx.x >= 128) {
-      prepare_query<(G > 0 ? G : 1)>(a, blockIdx.x, threadIdx.x - 128);
-      return;
-    }
-  }
   const int unit = blockIdx.x;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
   const int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
-  bool fits = true;
-  if (!state_ok(S, Sq, a)) {
-    if (threadIdx.x == 0) atomicOr(a.status, kStatusBadState);
-    fits = false;
-  } else if (S + a.n_new > a.cap) {
-    if (threadIdx.x == 0) atomicOr(a.status, kStatusOverflow);
-    fits = false;
+  const bool valid = state_ok(S, Sq, a);
+  const bool fits = valid && S + a.n_new <= a.cap;
+  if (G > 0) {
+    griddep_launch();  // the decode kernel may launch now; it waits for this whole grid
+    __syncthreads();   // every thread has read the state before the append half rewrites it
+    if (threadIdx.x >= 128) {
+      // the query is the newest token: position S + n_new - 1 (S - 1 if the append is refused)
+      const int qpos = max((fits ? S + a.n_new : (valid ? S : 1)) - 1, 0);
+      prepare_query<(G > 0 ? G : 1)>(a, unit, threadIdx.x - 128, qpos);
+      return;
+    }
   }
-  if (!fits) return;
+  if (!valid) {
+    if (threadIdx.x == 0) atomicOr(a.status, kStatusBadState);
+    return;
+  }
+  if (!fits) {
+    if (threadIdx.x == 0) atomicOr(a.status, kStatusOverflow);
+    return;
+  }
   // 1. the flush that closes the previous chunk (entries still in the ring)
   const FlushPlan fp = flush_plan(Sq, S, a);
   quantize_ring_range<BITS, NSEL>(a, unit, fp.lo0, fp.lo0 + fp.nf, threadIdx.x, 128);
@@ -149,11 +157,15 @@ __global__ void __launch_bounds__(G > 0 ? 256 : 128) append_small_kernel(const A
   // output row r: its 256-byte row of T_K is loaded once (16 x 16 B in flight), the
   // token's key is staged in shared memory as fp32.
   __shared__ float ks[kHeadDim];
+  __shared__ float hs[kHeadDim];  // Hadamard butterflies across warps
   const int r = threadIdx.x;
-  const uint4* Trow = reinterpret_cast<const uint4*>(a.t_k + ((size_t)h * kHeadDim + r) * kHeadDim);
+  const bool hadamard = a.transform == WUSHKV_TRANSFORM_HADAMARD;
   uint4 tr[kHeadDim / 8];
+  if (!hadamard) {
+    const uint4* Trow = reinterpret_cast<const uint4*>(a.t_k + ((size_t)h * kHeadDim + r) * kHeadDim);
 #pragma unroll
-  for (int i = 0; i < kHeadDim / 8; ++i) tr[i] = Trow[i];
+    for (int i = 0; i < kHeadDim / 8; ++i) tr[i] = Trow[i];
+  }
   for (int t = 0; t < a.n_new; ++t) {
     const int p = S + t;
     const size_t src = (((size_t)b * a.n_new + t) * a.Hkv + h) * kHeadDim;
@@ -169,19 +181,43 @@ __global__ void __launch_bounds__(G > 0 ? 256 : 128) append_small_kernel(const A
     ks[r] = __half2float(a.k_new[src + r]);
     if (r < kHeadDim / 8)
       reinterpret_cast<uint4*>(vdst)[r] = reinterpret_cast<const uint4*>(a.v_new + src)[r];
-    bar_sync(1, 128);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four interleaved partial sums, added at the end
-#pragma unroll
-    for (int i = 0; i < kHeadDim / 8; ++i) {
-      const uint32_t w[4] = {tr[i].x, tr[i].y, tr[i].z, tr[i].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 tf = __half22float2(u32_as_h2(w[e]));
-        acc[e] = fmaf(tf.x, ks[8 * i + 2 * e], acc[e]);
-        acc[e] = fmaf(tf.y, ks[8 * i + 2 * e + 1], acc[e]);
-      }
+    if (a.prep.enabled) {  // raw key: RMSNorm + RoPE at its position, by the first warp
+      bar_sync(1, 128);
+      if (r < 32) prep_head_warp(ks, a.prep.k_gain, a.prep, p, r);
     }
-    kdst[r] = __float2half_rn((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    bar_sync(1, 128);
+    if (hadamard) {
+      // fast Walsh-Hadamard transform: butterflies over bits 1..16 within the warp, 32 and
+      // 64 across warps through shared memory; then the 1/sqrt(128) normalisation
+      float y = ks[r];
+#pragma unroll
+      for (int bit = 1; bit < 32; bit <<= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, y, bit);
+        y = (r & bit) ? o - y : y + o;
+      }
+#pragma unroll
+      for (int bit = 32; bit < kHeadDim; bit <<= 1) {
+        hs[r] = y;
+        bar_sync(1, 128);
+        const float o = hs[r ^ bit];
+        y = (r & bit) ? o - y : y + o;
+        bar_sync(1, 128);
+      }
+      kdst[r] = __float2half_rn(y * 0.08838834764831845f);
+    } else {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four interleaved partial sums, added at the end
+#pragma unroll
+      for (int i = 0; i < kHeadDim / 8; ++i) {
+        const uint32_t w[4] = {tr[i].x, tr[i].y, tr[i].z, tr[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 tf = __half22float2(u32_as_h2(w[e]));
+          acc[e] = fmaf(tf.x, ks[8 * i + 2 * e], acc[e]);
+          acc[e] = fmaf(tf.y, ks[8 * i + 2 * e + 1], acc[e]);
+        }
+      }
+      kdst[r] = __float2half_rn((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    }
     bar_sync(1, 128);  // ks is rewritten by the next token
   }
   // 3. state
@@ -193,13 +229,19 @@ __global__ void __launch_bounds__(G > 0 ? 256 : 128) append_small_kernel(const A
 
 // ---------------------------------------------------------------------------------
 // Bulk append, launch 1: quantize the ring entries covered by the flush under S + n_new.
+// CTA (slice, unit): slice c takes ring positions lo0 + [16c, 16c + 16) (32 rows, K and V,
+// four lanes per row), so a long ring flush is spread over many CTAs.
+constexpr int kFlushSlice = 16;
+
 template <int BITS, int NSEL>
 __global__ void __launch_bounds__(128) flush_ring_kernel(const AppendArgs a) {
-  const int unit = blockIdx.x;
+  const int unit = blockIdx.y;
   const int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
   if (!state_ok(S, Sq, a) || S + a.n_new > a.cap) return;
   const FlushPlan fp = flush_plan(Sq, S + a.n_new, a);
-  quantize_ring_range<BITS, NSEL>(a, unit, fp.lo0, min(fp.lo0 + fp.nf, S));
+  const int p0 = fp.lo0 + kFlushSlice * blockIdx.x;
+  const int p1 = min(min(fp.lo0 + fp.nf, S), p0 + kFlushSlice);
+  quantize_ring_range<BITS, NSEL>(a, unit, p0, p1);
 }
 
 // Bulk append, launch 2.  CTA = (256-token slab, unit), 8 warps; per 64-token tile:
@@ -213,8 +255,48 @@ constexpr size_t kBulkSmem = (size_t)(kHeadDim + 2 * kBulkTile) * kPad * sizeof(
 
 constexpr int kBulkThreads = 256;
 
-template <int BITS, int NSEL>
-__global__ void __launch_bounds__(kBulkThreads) append_bulk_kernel(const AppendArgs a) {
+// RMSNorm + RoPE of one raw key row held by 16 adjacent lanes, 8 dimensions (one uint4 of
+// fp16) each: lane chunk c has dimensions col = 8c .. 8c+7, whose rotation partners are
+// in chunk c ^ 8 (dimension +-64).
+__device__ __forceinline__ uint4 prep_chunk16(uint4 raw, int col, int pos, const double* inv_freq,
+                                              const PrepSpec& p) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  float x[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(u32_as_h2(w[e]));
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+  if (p.k_gain != nullptr) {
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss = fmaf(x[j], x[j], ss);
+#pragma unroll
+    for (int off = 1; off < 16; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv = 1.0f / sqrtf(ss / 128.0f + p.eps);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = (x[j] * inv) * __half2float(p.k_gain[col + j]);
+  }
+  const bool first = col < 64;  // dimensions i < 64: out = x c - partner s; else x c + partner s
+  uint32_t o[4];
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) {
+    float r2[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float partner = __shfl_xor_sync(0xffffffffu, x[j + u], 8);
+      float c, sn;
+      rope_cs(inv_freq[(col + j + u) & 63], pos, c, sn);
+      r2[u] = first ? x[j + u] * c - partner * sn : x[j + u] * c + partner * sn;
+    }
+    o[j / 2] = h2_as_u32(__floats2half2_rn(r2[0], r2[1]));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <int BITS, int NSEL, bool PREP>
+__global__ void __launch_bounds__(kBulkThreads, 3) append_bulk_kernel(const AppendArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __half* Ts = reinterpret_cast<__half*>(smem_raw);
   __half* ks = Ts + kHeadDim * kPad;
@@ -230,12 +312,32 @@ __global__ void __launch_bounds__(kBulkThreads) append_bulk_kernel(const AppendA
   constexpr int CB = 16 * BITS;
   const QuantSpec qs = spec_of(a);
 
-  // T_K -> shared (row r = output dim, col i = input dim)
+  // T_K -> shared (row r = output dim, col i = input dim); the Hadamard transform as its
+  // exact +-1 pattern (the 1/sqrt(128) is applied to the fp32 products)
+  const bool hadamard = a.transform == WUSHKV_TRANSFORM_HADAMARD;
+  const float tscale = hadamard ? 0.08838834764831845f : 1.0f;
   const __half* T = a.t_k + (size_t)h * kHeadDim * kHeadDim;
   for (int c = tid; c < kHeadDim * 16; c += kBulkThreads) {
     const int r = c >> 4, col = (c & 15) * 8;
-    *reinterpret_cast<uint4*>(Ts + r * kPad + col) = *reinterpret_cast<const uint4*>(T + r * kHeadDim + col);
+    uint4 v;
+    if (hadamard) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t lo = (__popc(r & (col + 2 * e)) & 1) ? 0xBC00u : 0x3C00u;  // -1 / +1
+        const uint32_t hi = (__popc(r & (col + 2 * e + 1)) & 1) ? 0xBC00u : 0x3C00u;
+        w[e] = lo | (hi << 16);
+      }
+      v = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      v = *reinterpret_cast<const uint4*>(T + r * kHeadDim + col);
+    }
+    *reinterpret_cast<uint4*>(Ts + r * kPad + col) = v;
   }
+
+  // raw keys (PREP): the 64 rotation frequencies, once per CTA
+  __shared__ double inv_freq[PREP ? 64 : 1];
+  if (PREP && tid < 64) inv_freq[tid] = rope_inv_freq(a.prep, tid);
 
   const int slab0 = blockIdx.x * kBulkSlab;
   for (int tile0 = slab0; tile0 < min(slab0 + kBulkSlab, a.n_new); tile0 += kBulkTile) {
@@ -249,6 +351,7 @@ __global__ void __launch_bounds__(kBulkThreads) append_bulk_kernel(const AppendA
         kv = *reinterpret_cast<const uint4*>(a.k_new + src);
         vv = *reinterpret_cast<const uint4*>(a.v_new + src);
       }
+      if (PREP) kv = prep_chunk16(kv, col, S + t, inv_freq, a.prep);
       *reinterpret_cast<uint4*>(ks + r * kPad + col) = kv;
       *reinterpret_cast<uint4*>(vs + r * kPad + col) = vv;
     }
@@ -287,9 +390,10 @@ __global__ void __launch_bounds__(kBulkThreads) append_bulk_kernel(const AppendA
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         const int col = 64 * nw + 8 * nt + 2 * t4;
-        *reinterpret_cast<__half2*>(ks + (16 * mw + g) * kPad + col) = __floats2half2_rn(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<__half2*>(ks + (16 * mw + g) * kPad + col) =
+            __floats2half2_rn(acc[nt][0] * tscale, acc[nt][1] * tscale);
         *reinterpret_cast<__half2*>(ks + (16 * mw + g + 8) * kPad + col) =
-            __floats2half2_rn(acc[nt][2], acc[nt][3]);
+            __floats2half2_rn(acc[nt][2] * tscale, acc[nt][3] * tscale);
       }
     }
     __syncthreads();
@@ -345,13 +449,20 @@ cudaError_t launch_append_t(const Derived& d, bool small, const AppendArgs& a, c
     append_small_kernel<BITS, NSEL, 0><<<d.units, 128, 0, st>>>(a);
     return cudaGetLastError();
   }
-  flush_ring_kernel<BITS, NSEL><<<d.units, 128, 0, st>>>(a);
+  // the ring holds at most R entries, so R / kFlushSlice slices cover any flush of it
+  flush_ring_kernel<BITS, NSEL><<<dim3((d.ring + kFlushSlice - 1) / kFlushSlice, d.units), 128, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = ensure_smem_attr<append_bulk_kernel<BITS, NSEL>>((int)kBulkSmem);
-  if (e != cudaSuccess) return e;
   dim3 grid((a.n_new + kBulkSlab - 1) / kBulkSlab, d.units);
-  append_bulk_kernel<BITS, NSEL><<<grid, kBulkThreads, kBulkSmem, st>>>(a);
+  if (a.prep.enabled) {
+    e = ensure_smem_attr<append_bulk_kernel<BITS, NSEL, true>>((int)kBulkSmem);
+    if (e != cudaSuccess) return e;
+    append_bulk_kernel<BITS, NSEL, true><<<grid, kBulkThreads, kBulkSmem, st>>>(a);
+  } else {
+    e = ensure_smem_attr<append_bulk_kernel<BITS, NSEL, false>>((int)kBulkSmem);
+    if (e != cudaSuccess) return e;
+    append_bulk_kernel<BITS, NSEL, false><<<grid, kBulkThreads, kBulkSmem, st>>>(a);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   advance_state_kernel<<<(d.units + 127) / 128, 128, 0, st>>>(a);

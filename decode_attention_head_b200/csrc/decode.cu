@@ -164,6 +164,11 @@ __global__ void __launch_bounds__(128) decode_prologue_kernel(const DecodeArgs a
     const int hh = i / kHeadDim, cc = i % kHeadDim;
     qs[hh][cc] = __half2float(a.q[((size_t)b * a.Hq + h * G + hh) * kHeadDim + cc]);
   }
+  if (a.prep.enabled) {  // raw queries (fused step, bulk route): RMSNorm + RoPE at position S - 1
+    __syncthreads();
+    const int qpos = max(a.state[2 * unit] - 1, 0);
+    for (int hh = tid >> 5; hh < G; hh += 4) prep_head_warp(qs[hh], a.prep.q_gain, a.prep, qpos, tid & 31);
+  }
   __syncthreads();
   float qp[G];
 #pragma unroll

@@ -5,6 +5,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include "../../include/wushkv.h"
+#include "prep.cuh"
 
 namespace wushkv {
 
@@ -61,6 +62,8 @@ struct AppendArgs {
   float* qprime;
   uint32_t* tickets;
   int Hq, ngroups;
+  PrepSpec prep;  // raw q / k (wushkv_step_prep): RMSNorm + RoPE fused in
+  int transform;  // WUSHKV_TRANSFORM_DENSE (t_k) or WUSHKV_TRANSFORM_HADAMARD (in-kernel)
 };
 
 struct DecodeArgs {
@@ -86,6 +89,7 @@ struct DecodeArgs {
   float* partials;     // [units][n_split][G][132]
   float* gpartials;    // [units][ngroups][G][132]
   int wait_all;        // 1: the preceding kernel writes the cache (fused step): wait before any read
+  PrepSpec prep;       // raw q (wushkv_step_prep, bulk route): the prologue normalises and rotates it
 };
 
 // Raise a kernel's dynamic shared-memory limit once per device (a function attribute,

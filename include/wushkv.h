@@ -78,7 +78,14 @@ typedef struct wushkv_config {
                           appends are quantized on arrival */
   float p_lo;          /* clipping percentiles, 0 <= p_lo < p_hi <= 100; the needed order */
   float p_hi;          /* statistics must lie within 4 of either end (e.g. 1/99, 0.5/99.5) */
+  int32_t transform;   /* key transform: WUSHKV_TRANSFORM_DENSE (0) reads T_K from the t_k
+                          argument; WUSHKV_TRANSFORM_HADAMARD (1) applies the normalised
+                          Walsh-Hadamard matrix H (H[r][i] = (-1)^popcount(r & i) / sqrt(128))
+                          computed in the kernels, t_k unused (may be NULL) */
 } wushkv_config;
+
+#define WUSHKV_TRANSFORM_DENSE 0
+#define WUSHKV_TRANSFORM_HADAMARD 1
 
 /* Byte sizes of the caller-allocated buffers (wushkv_pack_layout). */
 typedef struct wushkv_layout {
@@ -132,6 +139,12 @@ int wushkv_pack_layout(const wushkv_config* cfg, wushkv_layout* out);
  * Returns WUSHKV_OK, WUSHKV_EINVAL or WUSHKV_ESINGULAR. */
 int wushkv_compensation(const uint16_t* t_k, int32_t n_kv_heads, float* t_k_inv);
 
+/* The compensation matrix of WUSHKV_TRANSFORM_HADAMARD (host only): H is orthonormal and
+ * symmetric, so T_K^{-1} = H; fills t_k_inv (fp32 [n_kv_heads][128][128]) with H rounded
+ * to fp32.  The structured transform is the pages' Hadamard baseline and their
+ * "cheaper structured transforms" direction.  Returns WUSHKV_OK or WUSHKV_EINVAL. */
+int wushkv_hadamard(int32_t n_kv_heads, float* t_k_inv);
+
 /* Append n_new >= 0 tokens to every sequence (§4.1, §4.2, §4.4 "Full-Precision Cache
  * Window", §5.3 quantizer).
  * k_new, v_new: device fp16 [B][n_new][H_kv][128]; keys after head-norm and RoPE,
@@ -179,6 +192,32 @@ int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* cache, cons
 int wushkv_step(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
                 int32_t n_new, const void* t_k, const void* q, const float* t_k_inv, float softmax_scale,
                 int32_t out_fp16, void* out, void* workspace, void* stream);
+
+/* The step before the path, for wushkv_step_prep: the queries and keys arrive as raw
+ * projections and the library applies, per head, the RMSNorm (where the model has one,
+ * as Qwen3 does) and the rotary position embedding that the path's inputs have undergone
+ * (§4.1: keys are cached after head-wise normalisation and RoPE).
+ *   RMSNorm: y = x / sqrt(mean(x^2) + norm_eps) * gain over the 128 head dimensions;
+ *   RoPE: rotate-half pairing, dimension i < 64 with i + 64, angle pos * theta^(-i/64);
+ *   each result rounded once to fp16.  Key t of an n_new-token append sits at position
+ *   S + t (S = the sequence's length before the append); the query at the newest
+ *   position, S + n_new - 1. */
+typedef struct wushkv_prep {
+  float rope_theta;        /* RoPE base, > 1 */
+  const void* q_norm_gain; /* device fp16 [128] RMSNorm gain of every query head, or NULL: no query norm */
+  const void* k_norm_gain; /* device fp16 [128] RMSNorm gain of every key head, or NULL: no key norm */
+  float norm_eps;          /* RMSNorm epsilon, > 0 when a gain is given */
+} wushkv_prep;
+
+/* wushkv_step on raw q / k: k_raw and q_raw are the projections before the per-head
+ * RMSNorm and RoPE that `prep` describes; v_new and every other argument as in
+ * wushkv_step.  The normalisation and rotation run inside the step's kernels (the
+ * append's key path and the decode's query preparation).  Returns WUSHKV_OK,
+ * WUSHKV_EINVAL (also: prep NULL, theta <= 1, a gain without eps > 0),
+ * WUSHKV_EUNSUPPORTED or WUSHKV_ECUDA. */
+int wushkv_step_prep(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_raw, const void* v_new,
+                     int32_t n_new, const void* t_k, const void* q_raw, const float* t_k_inv, float softmax_scale,
+                     int32_t out_fp16, void* out, void* workspace, const wushkv_prep* prep, void* stream);
 
 /* wushkv_decode_attn with library-owned scratch instead of a caller-allocated workspace.
  * The method has no counterpart of this call: it serves callers that cannot allocate

@@ -105,3 +105,17 @@ def test_compensation_rejects_singular(bnd):
     t = torch.zeros(1, 128, 128, dtype=torch.float16)
     with pytest.raises(bnd.WushKVError):
         bnd.compensation(t)
+
+
+def test_hadamard_helper_and_transform_field(bnd):
+    """wushkv_hadamard fills H (orthonormal, symmetric, +-1/sqrt(128) by popcount parity);
+    an unknown transform kind is rejected."""
+    import scipy.linalg
+    h = bnd.hadamard_compensation(2).numpy()
+    ref = (scipy.linalg.hadamard(128) / np.sqrt(128)).astype(np.float32)
+    np.testing.assert_array_equal(h[0], ref)
+    np.testing.assert_array_equal(h[1], ref)
+    cfg = bnd.make_config(2, 2, 8, 2, 1000, 4, 32, 16, 1, transform=bnd.TRANSFORM_HADAMARD)
+    assert bnd.pack_layout(cfg).cap_alloc == 1024
+    cfg.transform = 2
+    assert bnd.lib.wushkv_pack_layout(ctypes.byref(cfg), ctypes.byref(bnd.Layout())) == bnd.EINVAL
