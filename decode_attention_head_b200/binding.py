@@ -16,11 +16,11 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwushkv.s
 
 OK, EINVAL, EUNSUPPORTED, ECUDA, ESINGULAR, ESCRATCH = 0, -1, -2, -3, -4, -5
 STATIC_SCRATCH_BYTES = 8 << 20  # WUSHKV_STATIC_SCRATCH_BYTES
-STATUS_OVERFLOW, STATUS_EMPTY, STATUS_TIMEOUT, STATUS_BADSTATE = 1, 2, 4, 8
+STATUS_OVERFLOW, STATUS_EMPTY, STATUS_TIMEOUT, STATUS_BADSTATE, STATUS_CHUNK_QUANTIZED = 1, 2, 4, 8, 16
 _ERR = {EINVAL: "invalid argument", EUNSUPPORTED: "unsupported configuration", ECUDA: "CUDA launch failed",
         ESINGULAR: "singular key transform", ESCRATCH: "needs more than the static scratch array holds"}
 SYMBOLS = ("wushkv_pack_layout", "wushkv_compensation", "wushkv_hadamard", "wushkv_append", "wushkv_decode_attn",
-           "wushkv_step", "wushkv_step_prep", "wushkv_decode_attn_static")
+           "wushkv_chunk_attn", "wushkv_step", "wushkv_step_prep", "wushkv_decode_attn_static")
 
 
 class Prep(ctypes.Structure):
@@ -44,7 +44,8 @@ class Layout(ctypes.Structure):
                 ("sink_bytes", ctypes.c_size_t), ("ring_bytes", ctypes.c_size_t),
                 ("state_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t),
                 ("cap_alloc", ctypes.c_int32), ("ring_slots", ctypes.c_int32), ("code_bytes", ctypes.c_int32),
-                ("n_splits", ctypes.c_int32), ("split_tokens", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("n_splits", ctypes.c_int32), ("split_tokens", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("chunk_workspace_bytes", ctypes.c_size_t)]
 
 
 class CacheBufs(ctypes.Structure):
@@ -75,6 +76,9 @@ def _load() -> ctypes.CDLL:
                                      ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.POINTER(Prep), ctypes.c_void_p]
+    lib.wushkv_chunk_attn.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
+                                      ctypes.c_int32, ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_void_p]
     lib.wushkv_decode_attn_static.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
                                               ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
                                               ctypes.c_void_p]
@@ -144,7 +148,8 @@ class KVCache:
         self.k_ring = torch.zeros(L.ring_bytes // 2, dtype=torch.float16, device=device)
         self.v_ring = torch.zeros(L.ring_bytes // 2, dtype=torch.float16, device=device)
         self.state = torch.zeros(L.state_bytes // 4, dtype=torch.int32, device=device)
-        self.workspace = torch.zeros(L.workspace_bytes, **u8)
+        # one scratch buffer serves decode_attn / step and chunk_attn (never concurrently)
+        self.workspace = torch.zeros(max(L.workspace_bytes, L.chunk_workspace_bytes), **u8)
         self.bufs = CacheBufs(*(t.data_ptr() for t in (self.k_codes, self.v_codes, self.k_params, self.v_params,
                                                         self.k_sink, self.v_sink, self.k_ring, self.v_ring,
                                                         self.state)))
@@ -179,6 +184,18 @@ class KVCache:
                                       t_k_inv.data_ptr(), float(softmax_scale), 1 if out.dtype == torch.float16 else 0,
                                       out.data_ptr(), self.workspace.data_ptr(), _stream_ptr(stream)),
                "wushkv_decode_attn")
+        return out
+
+    def chunk_attn(self, q: torch.Tensor, t_k_inv: torch.Tensor, softmax_scale: float,
+                   out: Optional[torch.Tensor] = None, out_fp16: bool = False, stream=None) -> torch.Tensor:
+        """q fp16 [B, n, H_q, 128]: the n newest positions' queries (the chunk just appended,
+        n <= chunk_max), each attending causally over the cache; returns out [B, n, H_q, 128]."""
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float16 if out_fp16 else torch.float32, device=q.device)
+        _check(lib.wushkv_chunk_attn(ctypes.byref(self.cfg), ctypes.byref(self.bufs), q.data_ptr(), q.shape[1],
+                                     t_k_inv.data_ptr(), float(softmax_scale), 1 if out.dtype == torch.float16 else 0,
+                                     out.data_ptr(), self.workspace.data_ptr(), _stream_ptr(stream)),
+               "wushkv_chunk_attn")
         return out
 
     def step(self, k_new: torch.Tensor, v_new: torch.Tensor, t_k: torch.Tensor, q: torch.Tensor,

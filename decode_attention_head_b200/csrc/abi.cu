@@ -101,6 +101,32 @@ static bool cache_ok(const wushkv_cache* c) {
 
 using namespace wushkv;
 
+// Largest power of two ng with ng * g <= 8 and ng <= n: the chunk tokens one launch of
+// chunk attention takes (as ng * g query heads per KV head).
+static int chunk_block(int g, int n) {
+  int ng = 1;
+  while (2 * ng * g <= 8 && 2 * ng <= n) ng *= 2;
+  return ng;
+}
+
+// The decode derivation for a launch of chunk attention over ng tokens.
+static int derive_chunk(const wushkv_config* cfg, int ng, Derived* d) {
+  wushkv_config c2 = *cfg;
+  c2.n_q_heads = cfg->n_kv_heads * (cfg->n_q_heads / cfg->n_kv_heads) * ng;
+  return derive(&c2, d);
+}
+
+// Workspace of wushkv_chunk_attn: the largest any of its launches needs.
+static size_t chunk_workspace(const wushkv_config* cfg) {
+  const int g = cfg->n_q_heads / cfg->n_kv_heads;
+  size_t best = 0;
+  for (int n = 1; n <= cfg->chunk_max && n <= 8; n *= 2) {
+    Derived d;
+    if (derive_chunk(cfg, chunk_block(g, n), &d) == WUSHKV_OK && d.ws_total > best) best = d.ws_total;
+  }
+  return best;
+}
+
 extern "C" int wushkv_pack_layout(const wushkv_config* cfg, wushkv_layout* out) {
   if (!out) return WUSHKV_EINVAL;
   Derived d;
@@ -117,6 +143,7 @@ extern "C" int wushkv_pack_layout(const wushkv_config* cfg, wushkv_layout* out) 
   out->ring_slots = d.ring;
   out->code_bytes = d.code_bytes;
   out->n_splits = d.n_split;
+  out->chunk_workspace_bytes = chunk_workspace(cfg);
   out->split_tokens = d.split_tokens;
   return WUSHKV_OK;
 }
@@ -233,6 +260,9 @@ static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv
   a->gpartials = reinterpret_cast<float*>(ws + d.ws_gpartials);
   a->units = d.units;
   a->wait_all = 0;
+  a->gq = d.group;
+  a->chunk_n = 0;
+  a->chunk_t0 = 0;
 }
 
 static int check_append(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
@@ -353,4 +383,34 @@ extern "C" int wushkv_step_prep(const wushkv_config* cfg, const wushkv_cache* ca
   if (!prep) return WUSHKV_EINVAL;
   return step_impl(cfg, cache, k_raw, v_new, n_new, t_k, q_raw, t_k_inv, softmax_scale, out_fp16, out, workspace, prep,
                    stream);
+}
+
+extern "C" int wushkv_chunk_attn(const wushkv_config* cfg, const wushkv_cache* cache, const void* q, int32_t n_q,
+                                 const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
+                                 void* workspace, void* stream) {
+  Derived d;
+  int rc = derive(cfg, &d);
+  if (rc != WUSHKV_OK) return rc;
+  if (n_q < 1 || n_q > cfg->chunk_max) return WUSHKV_EINVAL;
+  rc = check_decode(cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace);
+  if (rc != WUSHKV_OK) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // blocks of ng tokens, each one launch pair whose ng * g query heads per KV head share
+  // one pass over the cache
+  for (int t0 = 0; t0 < n_q;) {
+    const int ng = chunk_block(d.group, n_q - t0);
+    Derived d2;
+    rc = derive_chunk(cfg, ng, &d2);
+    if (rc != WUSHKV_OK) return rc;
+    DecodeArgs a;
+    fill_decode(cfg, d2, cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace, &a);
+    a.Hq = cfg->n_q_heads;
+    a.gq = d.group;
+    a.chunk_n = n_q;
+    a.chunk_t0 = t0;
+    const cudaError_t e = launch_decode(d2, cfg->bits, a, st);
+    if (e != cudaSuccess) return WUSHKV_ECUDA;
+    t0 += ng;
+  }
+  return WUSHKV_OK;
 }

@@ -39,6 +39,7 @@
 // bit of the product's precision inside the MMA; at bits 4..9 at most 6 of 24 are lost.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <climits>
 #include <cstdint>
 #include <math_constants.h>
 #include "internal.h"
@@ -64,6 +65,15 @@ __device__ __forceinline__ float ex2(float x) {  // 2^x (hardware approximation,
   return y;
 }
 
+
+// Row (in units of 128 elements) of query head v (0..G-1) of unit (b, h) in q and out: a
+// one-token decode has its G heads side by side; chunk attention's v is token v / gq of the
+// launch's block of the chunk, head v % gq.
+__device__ __forceinline__ size_t head_row(const DecodeArgs& a, int b, int h, int v) {
+  const int t = v / a.gq, hh = v - t * a.gq;
+  const int ntok = a.chunk_n > 0 ? a.chunk_n : 1;
+  return ((size_t)b * ntok + a.chunk_t0 + t) * a.Hq + (size_t)h * a.gq + hh;
+}
 
 template <int BITS>
 struct Cfg {
@@ -162,7 +172,7 @@ __global__ void __launch_bounds__(128) decode_prologue_kernel(const DecodeArgs a
   for (int u = 0; u < 32; ++u) t[u] = __ldg(Ti + (size_t)u * kHeadDim);
   for (int i = tid; i < G * kHeadDim; i += 128) {
     const int hh = i / kHeadDim, cc = i % kHeadDim;
-    qs[hh][cc] = __half2float(a.q[((size_t)b * a.Hq + h * G + hh) * kHeadDim + cc]);
+    qs[hh][cc] = __half2float(a.q[head_row(a, b, h, hh) * kHeadDim + cc]);
   }
   if (a.prep.enabled) {  // raw queries (fused step, bulk route): RMSNorm + RoPE at position S - 1
     __syncthreads();
@@ -572,9 +582,11 @@ __device__ __forceinline__ void window_load(const DecodeArgs& a, int unit, int i
   }
 }
 
+// qlim: chunk attention's causal limit -- head v sees positions <= qlim + v / gq (a
+// one-token decode passes INT_MAX: every cached position is visible).
 template <int G>
 __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, int n_sink, int r0, int warp,
-                             int lane, WinRows<G>& w, Merge* mg, float* wpv) {
+                             int lane, WinRows<G>& w, Merge* mg, float* wpv, int qlim) {
   constexpr int KB = WinRows<G>::KB;
   float qv[G][4];
 #pragma unroll
@@ -613,10 +625,13 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) x[u][hh] += __shfl_xor_sync(0xffffffffu, x[u][hh], off);
 #pragma unroll
-    for (int u = 0; u < KB; ++u)
-      if (it0 + u * kConsumers >= wend)
+    for (int u = 0; u < KB; ++u) {
+      const int it = it0 + u * kConsumers;
+      const int pos = it < n_sink ? it : r0 + (it - n_sink);
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) x[u][hh] = -CUDART_INF_F;
+      for (int hh = 0; hh < G; ++hh)
+        if (it >= wend || pos > qlim + hh / a.gq) x[u][hh] = -CUDART_INF_F;
+    }
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
       float mn = m[hh];
@@ -701,7 +716,7 @@ __device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, 
     if (dst) {
       dst[hh * kPartStride + 4 + d] = acc;
     } else {
-      const size_t o = ((size_t)b * a.Hq + h * G + hh) * kHeadDim + d;
+      const size_t o = head_row(a, b, h, hh) * kHeadDim + d;
       if (a.out_fp16)
         reinterpret_cast<__half*>(a.out)[o] = __float2half_rn(acc);
       else
@@ -737,6 +752,9 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     S = 0;
     Sq = 0;
   }
+  // chunk attention needs the chunk in the fp16 window (so the quantized positions precede
+  // every chunk query); report a cache where that does not hold
+  if (a.chunk_n > 0 && Sq > S - a.chunk_n && tid == 0 && item == 0) atomicOr(a.status, kStatusChunkQuantized);
   // quantized positions of this item: [lo, hi) within [qlo, qhi).  The items split the
   // region as it stands now (not the capacity), in whole 128-position stages counted from
   // the stage that holds qlo, so every item but the last streams the same number of stages.
@@ -804,7 +822,8 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     WinRows<G> wr;
     window_load<G>(a, unit, wbeg + warp, wend, n_sink, r0, lane, wr);
     griddep_wait();  // q', its constants and the counter resets come from the prologue
-    window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, wr, mg, wpv);
+    const int qlim = a.chunk_n > 0 ? S - a.chunk_n + a.chunk_t0 : INT_MAX;
+    window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, wr, mg, wpv, qlim);
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) qs.o[mt][0] = qs.o[mt][1] = qs.o[mt][2] = qs.o[mt][3] = 0.f;
     // (b) quantized positions

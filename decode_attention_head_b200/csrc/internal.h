@@ -89,6 +89,10 @@ struct DecodeArgs {
   float* partials;     // [units][n_split][G][132]
   float* gpartials;    // [units][ngroups][G][132]
   int wait_all;        // 1: the preceding kernel writes the cache (fused step): wait before any read
+  // chunk attention (wushkv_chunk_attn): the kernel's G query heads per unit are gq real
+  // heads of each of G / gq consecutive chunk tokens, chunk_t0 the first of them; q and out
+  // are [B][chunk_n][H_q][128]; chunk_n = 0 for a one-token decode (gq = G)
+  int chunk_n, chunk_t0, gq;
   PrepSpec prep;       // raw q (wushkv_step_prep, bulk route): the prologue normalises and rotates it
 };
 

@@ -8,7 +8,8 @@
 namespace wushkv {
 
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
-constexpr uint32_t kStatusOverflow = 1u, kStatusEmpty = 2u, kStatusTimeout = 4u, kStatusBadState = 8u;
+constexpr uint32_t kStatusOverflow = 1u, kStatusEmpty = 2u, kStatusTimeout = 4u, kStatusBadState = 8u,
+                   kStatusChunkQuantized = 16u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -61,6 +61,9 @@ extern "C" {
 #define WUSHKV_STATUS_TIMEOUT 4u  /* a bounded in-kernel wait gave up (a library bug, not an input error) */
 #define WUSHKV_STATUS_BADSTATE 8u /* a state entry was out of range (S < 0, S > capacity, S_quant outside
                                      [0, S]): that (sequence, KV head) was skipped / read as empty */
+#define WUSHKV_STATUS_CHUNK_QUANTIZED 16u /* wushkv_chunk_attn on a cache whose newest n_q positions are
+                                             not all fp16 (e.g. after a bulk append): quantized
+                                             positions were visible to every chunk query */
 
 /* Cache configuration; one cache holds one attention layer. */
 typedef struct wushkv_config {
@@ -104,6 +107,7 @@ typedef struct wushkv_layout {
                              kernel splits each sequence's current length evenly among the
                              n_splits items, in whole multiples of 128) */
   int32_t reserved;
+  size_t chunk_workspace_bytes; /* wushkv_chunk_attn scratch (no initialisation needed) */
 } wushkv_layout;
 
 /* Device pointers of one layer's cache.
@@ -192,6 +196,21 @@ int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* cache, cons
 int wushkv_step(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
                 int32_t n_new, const void* t_k, const void* q, const float* t_k_inv, float softmax_scale,
                 int32_t out_fp16, void* out, void* workspace, void* stream);
+
+/* Chunked prefill attention (the pages' order, §4.4: a new chunk is appended in full
+ * precision and computes its own attention before it is quantized): the n_q newest
+ * positions of every sequence (the chunk just appended with n_q <= chunk_max, so all of it
+ * is in the fp16 window) attend, each causally, over the cache: query t (position
+ * S - n_q + t) sees positions 0 .. S - n_q + t.
+ * q:   device fp16 [B][n_q][H_q][128] (after head-norm and RoPE); out: [B][n_q][H_q][128],
+ *      fp32 or fp16 (out_fp16); t_k_inv, softmax_scale as in wushkv_decode_attn.
+ * workspace: layout.chunk_workspace_bytes (no initialisation needed).
+ * The chunk's queries share passes over the cache in blocks of up to 8 / g tokens.
+ * Returns WUSHKV_OK, WUSHKV_EINVAL (also n_q < 1 or n_q > chunk_max), WUSHKV_EUNSUPPORTED
+ * or WUSHKV_ECUDA. */
+int wushkv_chunk_attn(const wushkv_config* cfg, const wushkv_cache* cache, const void* q, int32_t n_q,
+                      const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out, void* workspace,
+                      void* stream);
 
 /* The step before the path, for wushkv_step_prep: the queries and keys arrive as raw
  * projections and the library applies, per head, the RMSNorm (where the model has one,

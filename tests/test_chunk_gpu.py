@@ -1,0 +1,73 @@
+"""Chunked prefill attention (wushkv_chunk_attn) against the oracle, through the C ABI:
+after each append of a chunk of n <= chunk_max tokens (still in the fp16 window), the
+chunk's n queries attend causally -- query t of the chunk sees positions up to its own --
+and must match exact softmax attention over the same (downloaded) cache truncated at that
+position.  A one-token chunk must equal wushkv_decode_attn."""
+import numpy as np
+import pytest
+import torch
+
+from decode_attention_head_b200 import binding as bnd
+from decode_attention_head_b200 import synth
+from oracle import attention as oatt
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_chunk(oc, q, T, scale):
+    """Causal attention of the n newest positions' queries q [B, n, H_q, d] over oc."""
+    B, n, Hq, d = q.shape
+    g = Hq // oc.H
+    tinv_t = oatt.compensation(T)
+    out = np.zeros((B, n, Hq, d))
+    for b in range(B):
+        S = int(oc.S[b])
+        for h in range(oc.H):
+            K, V = oc.keys_hat(b, h), oc.values_hat(b, h)
+            for t in range(n):
+                pos = S - n + t
+                for j in range(h * g, (h + 1) * g):
+                    qc = tinv_t[h] @ q[b, t, j].astype(np.float64)
+                    out[b, t, j], _, _ = oatt.softmax_attention(qc, K[:pos + 1], V[:pos + 1], scale)
+    return out
+
+
+@pytest.mark.parametrize("bits,Hkv,Hq,chunk", [(2, 2, 8, 8), (2, 2, 2, 16), (4, 1, 8, 4), (2, 2, 4, 3)])
+def test_chunk_attention_matches_oracle(bits, Hkv, Hq, chunk):
+    B = 2
+    cfg = bnd.make_config(B, Hkv, Hq, bits, 3000, 4, 32, 16, chunk)
+    wl = synth.WORKLOADS["tiny"]
+    T = np.stack([synth.key_transform(wl, 7, h).numpy() for h in range(Hkv)])
+    t_dev = H.to_dev(T)
+    tinv = bnd.compensation(torch.from_numpy(T)).cuda()
+    scale = 1 / np.sqrt(128)
+    rng = np.random.default_rng(bits * 100 + Hq + chunk)
+    gc = bnd.KVCache(cfg)
+
+    def tokens(n):
+        x = rng.standard_normal((B, n, Hkv, 128))
+        x[..., [9, 99]] *= 15
+        return H.to_dev(x.astype(np.float16))
+
+    gc.append(tokens(900), tokens(900), t_dev)  # a bulk prefill before the chunks
+    for i, n in enumerate([chunk, 1, max(chunk - 1, 1), chunk, 2 if chunk >= 2 else 1]):
+        gc.append(tokens(n), tokens(n), t_dev)
+        q = rng.standard_normal((B, n, Hq, 128)).astype(np.float16)
+        out = gc.chunk_attn(H.to_dev(q), tinv, scale)
+        torch.cuda.synchronize()
+        assert gc.status() == 0
+        ref = _oracle_chunk(H.oracle_cache_from_gpu(gc), q, T, scale)
+        H.assert_attention_close(out.cpu().numpy(), ref)
+        if n == 1:
+            dec = gc.decode_attn(H.to_dev(q[:, 0]), tinv, scale)
+            assert torch.equal(dec, out[:, 0])
+
+
+def test_chunk_attention_rejects_oversized_chunk():
+    cfg = bnd.make_config(1, 1, 4, 2, 256, 4, 32, 16, 4)
+    gc = bnd.KVCache(cfg)
+    q = torch.zeros(1, 5, 4, 128, dtype=torch.float16, device="cuda")
+    tinv = torch.eye(128, device="cuda")[None].contiguous()
+    with pytest.raises(bnd.WushKVError):
+        gc.chunk_attn(q, tinv, 0.1)
