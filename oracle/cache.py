@@ -48,12 +48,15 @@ class Cache:
 
     def __init__(self, batch, n_kv_heads, head_dim, bits, p_lo, p_hi,
                  s_sink, s_keep, s_flush, capacity, chunk_max=1,
-                 store_dtype=np.float16):
+                 store_dtype=np.float16, quantize_fn=None):
         self.B, self.H, self.d = batch, n_kv_heads, head_dim
         self.bits, self.p_lo, self.p_hi = bits, p_lo, p_hi
         self.S_sink, self.S_keep, self.S_flush = s_sink, s_keep, s_flush
         self.capacity, self.chunk_max = capacity, chunk_max
         self.store_dtype = store_dtype
+        # the per-token quantizer: x fp16 [..., d] -> (codes, s, z); the percentile-clipped
+        # affine one unless another is given (e.g. quest.quantize)
+        self.quantize_fn = quantize_fn or (lambda x: quantizer.quantize(x, self.bits, self.p_lo, self.p_hi))
         self.S = np.zeros(batch, dtype=np.int64)
         self.S_quant = np.zeros(batch, dtype=np.int64)
         shape = (batch, n_kv_heads, capacity, head_dim)
@@ -79,7 +82,7 @@ class Cache:
         for store, codes, s_arr, z_arr in ((self.k_store, self.k_codes, self.k_s, self.k_z),
                                            (self.v_store, self.v_codes, self.v_s, self.v_z)):
             x = store[b, :, sl].astype(np.float16)
-            c, s, z = quantizer.quantize(x, self.bits, self.p_lo, self.p_hi)
+            c, s, z = self.quantize_fn(x)
             codes[b, :, sl] = c
             s_arr[b, :, sl] = s
             z_arr[b, :, sl] = z
