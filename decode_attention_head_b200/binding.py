@@ -33,10 +33,11 @@ class Config(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("bits", ctypes.c_int32), ("capacity", ctypes.c_int32),
                 ("s_sink", ctypes.c_int32), ("s_keep", ctypes.c_int32), ("s_flush", ctypes.c_int32),
                 ("chunk_max", ctypes.c_int32), ("p_lo", ctypes.c_float), ("p_hi", ctypes.c_float),
-                ("transform", ctypes.c_int32)]
+                ("transform", ctypes.c_int32), ("quantizer", ctypes.c_int32), ("clip_alpha", ctypes.c_float)]
 
 
 TRANSFORM_DENSE, TRANSFORM_HADAMARD = 0, 1
+QUANT_PERCENTILE, QUANT_RMS = 0, 1
 
 
 class Layout(ctypes.Structure):
@@ -96,9 +97,10 @@ def _check(rc: int, what: str) -> None:
 
 
 def make_config(batch, n_kv_heads, n_q_heads, bits, capacity, s_sink, s_keep, s_flush=16, chunk_max=1,
-                p_lo=1.0, p_hi=99.0, head_dim=128, transform=TRANSFORM_DENSE) -> Config:
+                p_lo=1.0, p_hi=99.0, head_dim=128, transform=TRANSFORM_DENSE, quantizer=QUANT_PERCENTILE,
+                clip_alpha=0.0) -> Config:
     return Config(batch, n_kv_heads, n_q_heads, head_dim, bits, capacity, s_sink, s_keep, s_flush, chunk_max,
-                  p_lo, p_hi, transform)
+                  p_lo, p_hi, transform, quantizer, clip_alpha)
 
 
 def pack_layout(cfg: Config) -> Layout:

@@ -24,6 +24,9 @@ int derive(const wushkv_config* cfg, Derived* d) {
   if (cfg->s_sink < 0 || cfg->s_keep < 0 || cfg->s_flush < 1 || cfg->chunk_max < 1) return WUSHKV_EINVAL;
   if (!(cfg->p_lo >= 0.f) || !(cfg->p_hi <= 100.f) || !(cfg->p_lo < cfg->p_hi)) return WUSHKV_EINVAL;
   if (cfg->transform != WUSHKV_TRANSFORM_DENSE && cfg->transform != WUSHKV_TRANSFORM_HADAMARD) return WUSHKV_EINVAL;
+  if (cfg->quantizer != WUSHKV_QUANT_PERCENTILE && cfg->quantizer != WUSHKV_QUANT_RMS) return WUSHKV_EINVAL;
+  if (cfg->quantizer == WUSHKV_QUANT_RMS && !(cfg->clip_alpha > 0.f && std::isfinite(cfg->clip_alpha)))
+    return WUSHKV_EINVAL;
   const long long units = (long long)cfg->batch * cfg->n_kv_heads;
   if (units > (1 << 24) || cfg->capacity > (1 << 28)) return WUSHKV_EINVAL;
 
@@ -44,6 +47,7 @@ int derive(const wushkv_config* cfg, Derived* d) {
   const int need_hi = kHeadDim - d->i_hi;        // s[i_hi] from the top
   d->nsel = need_lo > need_hi ? need_lo : need_hi;
   if (d->nsel < 2) d->nsel = 2;
+  if (cfg->quantizer == WUSHKV_QUANT_RMS) d->nsel = 2;  // no order statistics
   if (d->nsel > 4) return WUSHKV_EUNSUPPORTED;
 
   // decode work split: n_split items per unit, chosen so that units * n_split fills whole
@@ -223,6 +227,9 @@ static void fill_append(const wushkv_config* cfg, const Derived& d, const wushkv
   a->Hq = cfg->n_q_heads;
   a->ngroups = ceil_div(d.n_split, kMergeGroup);
   a->transform = cfg->transform;
+  a->quant_rms = cfg->quantizer == WUSHKV_QUANT_RMS;
+  a->rms_kb = (float)(2.0 * (double)cfg->clip_alpha / (double)((1 << cfg->bits) - 1));
+  a->rms_alpha = cfg->clip_alpha;
 }
 
 static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv_cache* cache, const void* q,

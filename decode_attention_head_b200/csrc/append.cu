@@ -48,6 +48,9 @@ __device__ __forceinline__ QuantSpec spec_of(const AppendArgs& a) {
   q.i_hi = a.i_hi;
   q.f_lo = a.f_lo;
   q.f_hi = a.f_hi;
+  q.rms = a.quant_rms;
+  q.kb = a.rms_kb;
+  q.alpha = a.rms_alpha;
   return q;
 }
 

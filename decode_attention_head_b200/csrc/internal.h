@@ -64,6 +64,8 @@ struct AppendArgs {
   int Hq, ngroups;
   PrepSpec prep;  // raw q / k (wushkv_step_prep): RMSNorm + RoPE fused in
   int transform;  // WUSHKV_TRANSFORM_DENSE (t_k) or WUSHKV_TRANSFORM_HADAMARD (in-kernel)
+  int quant_rms;            // WUSHKV_QUANT_RMS: (s, z) from the token's RMS, not its percentiles
+  float rms_kb, rms_alpha;  // fp32(2*alpha/(2^b-1)), fp32(alpha)
 };
 
 struct DecodeArgs {

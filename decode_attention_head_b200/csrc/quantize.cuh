@@ -1,4 +1,4 @@
-// Per-token percentile-clipped asymmetric affine quantizer, one thread per token-head
+// Per-token percentile-clipped asymmetric affine quantizer, one row over 2 or 4 lanes
 // ("WUSH-KV: KV Cache Quantization with Data-Adaptive Transforms", §5.3: percentile
 // clipping with asymmetric affine scaling and an adaptive zero point; §1: per-token
 // clipped quantizers).
@@ -14,6 +14,9 @@
 // The division is done as a multiplication by the correctly rounded reciprocal; where
 // that product lies within its error bound of a rounding midpoint, the exact IEEE
 // division decides, so the code always equals round(fl32(fl32(x - z) / s)).
+// The RMS-scaled symmetric alternative (QuEST-style, same page §4.3 and Appendix B.3)
+// replaces only (s, z): sigma = sqrt(sum x^2 / 128) in fp32 in a fixed order,
+// s = fp16(fp32(2 alpha / (2^bits - 1)) * sigma), z = fp16(-alpha * sigma).
 #pragma once
 #include <cuda_fp16.h>
 #include <cstdint>
@@ -24,6 +27,8 @@ namespace wushkv {
 struct QuantSpec {
   int i_lo, i_hi;   // ranks floor(p/100 * 127)
   float f_lo, f_hi; // fractional parts, fp32
+  int rms;          // 1: RMS-scaled symmetric grid instead of percentiles
+  float kb, alpha;  // fp32(2*alpha/(2^b-1)), fp32(alpha)
 };
 
 // Insert x into the ascending list a[0..K-1] of the K smallest seen so far (both halves
@@ -97,89 +102,7 @@ __device__ __forceinline__ uint32_t quantize_one(float v, float zf, float sf, fl
   return static_cast<uint32_t>(c);
 }
 
-// Quantize the 128 fp16 values at x (global or shared, 16-byte aligned) and write the
-// packed codes (16*BITS bytes, 16-byte aligned) and the half2 (s, z).
-template <int BITS, int NSEL>
-__device__ __noinline__ void quantize_row(const __half* __restrict__ x, uint8_t* __restrict__ codes_out,
-                                          uint32_t* __restrict__ params_out, const QuantSpec qs) {
-  __half2 v[64];
-  const uint4* src = reinterpret_cast<const uint4*>(x);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    uint4 u = src[i];
-    v[4 * i + 0] = u32_as_h2(u.x);
-    v[4 * i + 1] = u32_as_h2(u.y);
-    v[4 * i + 2] = u32_as_h2(u.z);
-    v[4 * i + 3] = u32_as_h2(u.w);
-  }
-  // --- order statistics at both ends
-  const __half2 pinf = __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));
-  const __half2 ninf = __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));
-  __half2 a[NSEL], b[NSEL];
-#pragma unroll
-  for (int j = 0; j < NSEL; ++j) {
-    a[j] = pinf;
-    b[j] = ninf;
-  }
-#pragma unroll
-  for (int i = 0; i < 64; ++i) {
-    insert_small<NSEL>(a, v[i]);
-    insert_large<NSEL>(b, v[i]);
-  }
-  float lo_s[NSEL], lo_t[NSEL], hi_s[NSEL], hi_t[NSEL];
-#pragma unroll
-  for (int j = 0; j < NSEL; ++j) {
-    lo_s[j] = __low2float(a[j]);
-    lo_t[j] = __high2float(a[j]);
-    hi_s[j] = __low2float(b[j]);
-    hi_t[j] = __high2float(b[j]);
-  }
-  merge_small<NSEL>(lo_s, lo_t);  // lo_s[j] = s[j]
-  merge_large<NSEL>(hi_s, hi_t);  // hi_s[j] = s[127 - j]
-  // s[i] for i in {i_lo, i_lo+1} from the bottom list, {i_hi, min(i_hi+1,127)} from the top
-  float slo0 = 0.f, slo1 = 0.f, shi0 = 0.f, shi1 = 0.f;
-  const int jh0 = 127 - qs.i_hi;
-  const int jh1 = 127 - min(qs.i_hi + 1, 127);
-#pragma unroll
-  for (int j = 0; j < NSEL; ++j) {
-    if (j == qs.i_lo) slo0 = lo_s[j];
-    if (j == qs.i_lo + 1) slo1 = lo_s[j];
-    if (j == jh0) shi0 = hi_s[j];
-    if (j == jh1) shi1 = hi_s[j];
-  }
-  const float lo = interp(slo0, slo1, qs.f_lo);
-  const float hi = interp(shi0, shi1, qs.f_hi);
-  const float scale32 = __fdiv_rn(__fsub_rn(hi, lo), float((1 << BITS) - 1));
-  const __half s_h = __float2half_rn(scale32);
-  const __half z_h = __float2half_rn(lo);
-  const float sf = __half2float(s_h);
-  const float zf = __half2float(z_h);
-
-  constexpr int NW = 4 * BITS;  // 32-bit words of packed codes
-  uint32_t w[NW];
-#pragma unroll
-  for (int i = 0; i < NW; ++i) w[i] = 0u;
-  if (sf != 0.0f) {
-    const float rcp = __frcp_rn(sf);
-#pragma unroll
-    for (int k = 0; k < 64; ++k) {
-      const float2 f = __half22float2(v[k]);
-      const uint32_t c0 = quantize_one<BITS>(f.x, zf, sf, rcp);
-      const uint32_t c1 = quantize_one<BITS>(f.y, zf, sf, rcp);
-      if (BITS == 2) {
-        w[k / 8] |= (c0 | (c1 << 2)) << (4 * (k % 8));
-      } else {
-        w[k / 4] |= (c0 | (c1 << 4)) << (8 * (k % 4));
-      }
-    }
-  }
-  uint4* dst = reinterpret_cast<uint4*>(codes_out);
-#pragma unroll
-  for (int i = 0; i < NW / 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-  *params_out = h2_as_u32(__halves2half2(s_h, z_h));
-}
-
-// The same quantizer with one row split over P adjacent lanes (P = 2 or 4; lanes
+// The quantizer with one row split over P adjacent lanes (P = 2 or 4; lanes
 // P*k .. P*k+P-1 of a warp, all active together): lane `part` takes values
 // [part*128/P, (part+1)*128/P), keeps its own NSEL smallest / largest, the lists are merged
 // over log2(P) xor-shuffle rounds (every lane ends with the same order statistics, so
@@ -202,6 +125,30 @@ __device__ __forceinline__ void quantize_row_part(const __half* __restrict__ x, 
     v[4 * i + 2] = u32_as_h2(u.z);
     v[4 * i + 3] = u32_as_h2(u.w);
   }
+  const int lane = threadIdx.x & 31;
+  const unsigned group = ((1u << P) - 1u) << (lane & ~(P - 1));
+  __half s_h, z_h;
+  if (qs.rms) {
+    // sigma^2: runs of 32 consecutive squares summed left to right, then (g0+g1)+(g2+g3)
+    float gsum[V / 32];
+#pragma unroll
+    for (int r = 0; r < V / 32; ++r) {
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 16 * r; k < 16 * r + 16; ++k) {
+        const float2 f = __half22float2(v[k]);
+        acc = __fadd_rn(acc, __fmul_rn(f.x, f.x));
+        acc = __fadd_rn(acc, __fmul_rn(f.y, f.y));
+      }
+      gsum[r] = acc;
+    }
+    float ss = V == 64 ? __fadd_rn(gsum[0], gsum[V / 32 - 1]) : gsum[0];  // P = 2: this lane's pair
+    if (P == 4) ss = __fadd_rn(ss, __shfl_xor_sync(group, ss, 1));          // g0+g1 | g2+g3
+    ss = __fadd_rn(ss, __shfl_xor_sync(group, ss, P == 4 ? 2 : 1));         // (g0+g1)+(g2+g3)
+    const float sigma = __fsqrt_rn(__fdiv_rn(ss, 128.0f));
+    s_h = __float2half_rn(__fmul_rn(qs.kb, sigma));
+    z_h = __float2half_rn(__fmul_rn(-qs.alpha, sigma));
+  } else {
   const __half2 pinf = __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));
   const __half2 ninf = __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));
   __half2 a[NSEL], b[NSEL];
@@ -225,8 +172,6 @@ __device__ __forceinline__ void quantize_row_part(const __half* __restrict__ x, 
   }
   merge_small<NSEL>(lo_s, lo_t);
   merge_large<NSEL>(hi_s, hi_t);
-  const int lane = threadIdx.x & 31;
-  const unsigned group = ((1u << P) - 1u) << (lane & ~(P - 1));
 #pragma unroll
   for (int off = 1; off < P; off <<= 1) {
 #pragma unroll
@@ -250,8 +195,9 @@ __device__ __forceinline__ void quantize_row_part(const __half* __restrict__ x, 
   const float lo = interp(slo0, slo1, qs.f_lo);
   const float hi = interp(shi0, shi1, qs.f_hi);
   const float scale32 = __fdiv_rn(__fsub_rn(hi, lo), float((1 << BITS) - 1));
-  const __half s_h = __float2half_rn(scale32);
-  const __half z_h = __float2half_rn(lo);
+  s_h = __float2half_rn(scale32);
+  z_h = __float2half_rn(lo);
+  }
   const float sf = __half2float(s_h);
   const float zf = __half2float(z_h);
 

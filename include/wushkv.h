@@ -85,10 +85,21 @@ typedef struct wushkv_config {
                           argument; WUSHKV_TRANSFORM_HADAMARD (1) applies the normalised
                           Walsh-Hadamard matrix H (H[r][i] = (-1)^popcount(r & i) / sqrt(128))
                           computed in the kernels, t_k unused (may be NULL) */
+  int32_t quantizer;   /* WUSHKV_QUANT_PERCENTILE (0): percentile-clipped affine (p_lo, p_hi);
+                          WUSHKV_QUANT_RMS (1): QuEST-style symmetric grid scaled by each
+                          token's RMS, clipped at +-clip_alpha * RMS (p_lo, p_hi unused) */
+  float clip_alpha;    /* WUSHKV_QUANT_RMS: clipping endpoint in RMS units, > 0 (the
+                          Gaussian-optimal value for the bit width, e.g. 1.4936 at 2 bits) */
 } wushkv_config;
 
 #define WUSHKV_TRANSFORM_DENSE 0
 #define WUSHKV_TRANSFORM_HADAMARD 1
+#define WUSHKV_QUANT_PERCENTILE 0
+/* WUSHKV_QUANT_RMS: per token sigma = sqrt(sum(x^2) / 128) in fp32, the squares summed in
+ * four runs of 32 consecutive elements, then (g0 + g1) + (g2 + g3); s = fp16(fp32(2*alpha /
+ * (2^b - 1)) * sigma), z = fp16(-fp32(alpha) * sigma); codes and storage as the affine
+ * quantizer's (the decode is unchanged). */
+#define WUSHKV_QUANT_RMS 1
 
 /* Byte sizes of the caller-allocated buffers (wushkv_pack_layout). */
 typedef struct wushkv_layout {

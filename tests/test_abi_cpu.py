@@ -119,3 +119,17 @@ def test_hadamard_helper_and_transform_field(bnd):
     assert bnd.pack_layout(cfg).cap_alloc == 1024
     cfg.transform = 2
     assert bnd.lib.wushkv_pack_layout(ctypes.byref(cfg), ctypes.byref(bnd.Layout())) == bnd.EINVAL
+
+
+def test_rms_quantizer_config_checks(bnd):
+    ok = bnd.make_config(1, 1, 4, 2, 256, 4, 32, 16, 1, quantizer=bnd.QUANT_RMS, clip_alpha=1.4936)
+    assert bnd.lib.wushkv_pack_layout(ctypes.byref(ok), ctypes.byref(bnd.Layout())) == bnd.OK
+    # percentiles are not used by the RMS quantizer, so ranks outside the supported four are fine
+    ok.p_lo, ok.p_hi = 10.0, 90.0
+    assert bnd.lib.wushkv_pack_layout(ctypes.byref(ok), ctypes.byref(bnd.Layout())) == bnd.OK
+    for alpha in (0.0, -1.0, float("inf")):
+        bad = bnd.make_config(1, 1, 4, 2, 256, 4, 32, 16, 1, quantizer=bnd.QUANT_RMS, clip_alpha=alpha)
+        assert bnd.lib.wushkv_pack_layout(ctypes.byref(bad), ctypes.byref(bnd.Layout())) == bnd.EINVAL
+    bad = bnd.make_config(1, 1, 4, 2, 256, 4, 32, 16, 1)
+    bad.quantizer = 7
+    assert bnd.lib.wushkv_pack_layout(ctypes.byref(bad), ctypes.byref(bnd.Layout())) == bnd.EINVAL
