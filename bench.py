@@ -122,30 +122,36 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def code_sha256(path):
-    """sha256 of a C++/CUDA source with // comments and blank lines removed: it changes when
-    the code changes, not when only its comments do."""
+def code_sha256(paths):
+    """sha256 of C++/CUDA sources (one path or several, concatenated in order) with //
+    comments and blank lines removed: it changes when the code changes, not when only its
+    comments do."""
     lines = []
-    for line in open(path, encoding="utf-8"):
-        code = line.split("//", 1)[0].rstrip()
-        if code.strip():
-            lines.append(code)
+    for path in [paths] if isinstance(paths, str) else paths:
+        for line in open(path, encoding="utf-8"):
+            code = line.split("//", 1)[0].rstrip()
+            if code.strip():
+                lines.append(code)
     return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
+# the decode kernels' source: decode.cu and the headers it includes from csrc/
+DECODE_SOURCES = ("decode.cu", "internal.h", "ptx.cuh", "prep.cuh")
 
 
 def profile_traffic(kernel_file):
     """DRAM bytes per launch of the decode kernel from the committed ncu summary, if that
     summary was taken on the current kernel code (its code sha256 is recorded there)."""
-    src = os.path.join(ROOT, "decode_attention_head_b200", "csrc", "decode.cu")
+    srcs = [os.path.join(ROOT, "decode_attention_head_b200", "csrc", f) for f in DECODE_SOURCES]
     path = os.path.join(ROOT, "profiles", kernel_file)
     try:
-        sha = code_sha256(src)
+        sha = code_sha256(srcs)
         info = {}
         for line in open(path):
             if ":" in line and line.strip().startswith("- "):
                 k, v = line.strip()[2:].split(":", 1)
                 info[k.strip()] = v.strip().strip("`")
-        if info.get("decode.cu code sha256") != sha:
+        if info.get("decode code sha256") != sha:
             return None
         return float(info["dram bytes per launch (full workload)"])
     except Exception:
