@@ -7,6 +7,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include "internal.h"
+#include "qfrag.cuh"
 
 namespace wushkv {
 
@@ -84,6 +85,8 @@ int derive(const wushkv_config* cfg, Derived* d) {
   off = round_up(off + U * 4 * (1 + (size_t)ceil_div(d->n_split, kMergeGroup)), 256);
   d->ws_qprime = off;
   off = round_up(off + U * g * kHeadDim * 4, 256);
+  d->ws_qfrag = off;
+  off = round_up(off + U * kQFragBytes, 256);
   d->ws_partials = off;
   off = round_up(off + U * (size_t)d->n_split * g * 132 * 4, 256);
   const size_t ngroups = (size_t)ceil_div(d->n_split, kMergeGroup);
@@ -263,6 +266,7 @@ static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a->tickets = reinterpret_cast<uint32_t*>(ws + d.ws_tickets);
   a->qprime = reinterpret_cast<float*>(ws + d.ws_qprime);
+  a->qfrag = ws + d.ws_qfrag;
   a->partials = reinterpret_cast<float*>(ws + d.ws_partials);
   a->gpartials = reinterpret_cast<float*>(ws + d.ws_gpartials);
   a->units = d.units;
@@ -363,6 +367,8 @@ static int step_impl(const wushkv_config* cfg, const wushkv_cache* cache, const 
     aa.q = da.q;
     aa.t_k_inv = da.t_k_inv;
     aa.qprime = da.qprime;
+    aa.qfrag = da.qfrag;
+    aa.scale_log2 = da.scale_log2;
     aa.tickets = da.tickets;
     e = launch_append_fused(d, cfg->bits, aa, st);
     if (e == cudaSuccess) {

@@ -21,6 +21,7 @@
 #include "internal.h"
 #include "ptx.cuh"
 #include "quantize.cuh"
+#include "qfrag.cuh"
 
 namespace wushkv {
 namespace {
@@ -80,8 +81,9 @@ __device__ void quantize_ring_range(const AppendArgs& a, int unit, int p_begin, 
 // q'_j = T_K^{-T} q_j (fp32) of the unit's G query heads into the decode workspace, by the
 // CTA's 128 threads: warp w sums rows [32w, 32w+32) of T_K^{-1} for the four dimensions
 // 4*lane .. 4*lane+3 (all 32 float4 loads in flight at once), the warps' partial sums meet
-// in shared memory.  Also resets the unit's decode completion counters.
-template <int G>
+// in shared memory.  Also resets the unit's decode completion counters and builds the
+// unit's query fragments for the decode kernel (qfrag.cuh).
+template <int BITS, int G>
 __device__ void prepare_query(const AppendArgs& a, int unit, int tid, int qpos) {
   __shared__ float qs[G][kHeadDim];
   __shared__ float red[4][G][kHeadDim];
@@ -115,10 +117,16 @@ __device__ void prepare_query(const AppendArgs& a, int unit, int tid, int qpos) 
   bar_sync(2, 128);
   for (int i = tid; i < G * kHeadDim; i += 128) {
     const int hh = i / kHeadDim, j = i % kHeadDim;
-    a.qprime[(size_t)unit * G * kHeadDim + i] = (red[0][hh][j] + red[1][hh][j]) + (red[2][hh][j] + red[3][hh][j]);
+    const float v = (red[0][hh][j] + red[1][hh][j]) + (red[2][hh][j] + red[3][hh][j]);
+    qs[hh][j] = v;  // q is no longer read
+    a.qprime[(size_t)unit * G * kHeadDim + i] = v;
   }
   for (int i = tid; i < a.ngroups; i += 128) a.tickets[a.B * a.Hkv + (size_t)unit * a.ngroups + i] = 0u;
   if (tid == 0) a.tickets[unit] = 0u;
+  bar_sync(2, 128);
+  __shared__ float cred[64];
+  build_query_frags<BITS, G>(qs, tid, 128, cred, a.scale_log2, a.qfrag + (size_t)unit * kQFragBytes,
+                             [] { bar_sync(2, 128); });
 }
 
 // Small append: one CTA per (sequence, KV head); threads 0..127 append.  G > 0: the fused
@@ -139,7 +147,7 @@ __global__ void __launch_bounds__(G > 0 ? 256 : 128) append_small_kernel(const A
     if (threadIdx.x >= 128) {
       // the query is the newest token: position S + n_new - 1 (S - 1 if the append is refused)
       const int qpos = max((fits ? S + a.n_new : (valid ? S : 1)) - 1, 0);
-      prepare_query<(G > 0 ? G : 1)>(a, unit, threadIdx.x - 128, qpos);
+      prepare_query<BITS, (G > 0 ? G : 1)>(a, unit, threadIdx.x - 128, qpos);
       return;
     }
   }

@@ -44,11 +44,11 @@
 #include <math_constants.h>
 #include "internal.h"
 #include "ptx.cuh"
+#include "qfrag.cuh"
 
 namespace wushkv {
 namespace {
 
-constexpr float kQMax = 1073741824.0f;  // |fixed-point query| <= 2^30; four signed 8-bit limbs hold +-2.1e9
 constexpr int kThreads = 160;            // 4 consumer warps + 1 producer warp
 constexpr int kConsumers = 4;
 constexpr int kSlice = 32;               // positions per consumer warp per stage
@@ -81,36 +81,6 @@ struct Cfg {
   static constexpr int NSTAGE = BITS == 2 ? 4 : 3;
   static constexpr int STAGE = kTileTokens * (2 * CB + 8);
 };
-
-template <int G>
-struct GCfg {
-  static constexpr int NHS = G <= 4 ? 1 : 2;  // head sets handled per lane
-  static constexpr int NT = 2 * NHS;          // QK n-tiles: limbs {0,1} then {2,3} per head set
-};
-
-// Dimension that (kstep j, reg r, lane t4, byte i) of a key-side operand carries, and the
-// power-of-two scale its codes have after masking.
-template <int BITS>
-__host__ __device__ __forceinline__ void key_slot(int dim, int& kstep, int& t4, int& r, int& byte, int& log2scale) {
-  if (BITS == 2) {
-    const int w = dim >> 4;  // word of 16 codes
-    byte = (dim & 15) >> 2;
-    const int plane = dim & 3;
-    t4 = w >> 1;
-    r = w & 1;
-    kstep = plane;
-    log2scale = 2 * plane;
-  } else {
-    const int w = dim >> 3;  // word of 8 codes
-    byte = (dim & 7) >> 1;
-    const int plane = dim & 1;
-    t4 = w >> 2;
-    const int rem = w & 3;
-    r = rem & 1;
-    kstep = 2 * (rem >> 1) + plane;
-    log2scale = 4 * plane;
-  }
-}
 
 // Value-side: dimension carried by row (g or g+8) of m-tile mt for lane group g, and the
 // log2 of the scale its masked codes carry.
@@ -154,30 +124,34 @@ __device__ __forceinline__ uint32_t vcode4(uint32_t x, int mi) {
 }
 
 // ---------------------------------------------------------------------------------
-// Prologue: CTA (unit, quarter c), 128 threads; thread (part, jj) sums 32 of the 128 terms
-// of q'[j] = sum_i Tinv[i][j] q[i] for j = 32c + jj.
-template <int G>
-__global__ void __launch_bounds__(128) decode_prologue_kernel(const DecodeArgs a) {
-  __shared__ float qs[G][kHeadDim];
-  __shared__ float part[4][G][32];
+// Prologue: one CTA per unit, 512 threads; thread (part, j) sums 32 of the 128 terms of
+// q'[j] = sum_i Tinv[i][j] q[i], the four parts are added in shared memory, and the CTA
+// then builds the unit's query fragments (qfrag.cuh) for every work item of the unit.
+constexpr int kPrologueThreads = 512;
+
+template <int BITS, int G>
+__global__ void __launch_bounds__(kPrologueThreads) decode_prologue_kernel(const DecodeArgs a) {
+  __shared__ float qs[G][kHeadDim];  // q, then q'
+  __shared__ float part[4][G][kHeadDim];
+  __shared__ float red[64];
   griddep_launch();
-  const int unit = blockIdx.x, c = blockIdx.y;
+  const int unit = blockIdx.x;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
-  const int tid = threadIdx.x, jj = tid & 31, pt = tid >> 5;
-  const int j = 32 * c + jj;
+  const int tid = threadIdx.x, j = tid & (kHeadDim - 1), pt = tid >> 7;
   const float* Ti = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim + (size_t)(32 * pt) * kHeadDim + j;
   // all 32 of this thread's T_K^{-1} loads are in flight before q is staged: one round trip
   float t[32];
 #pragma unroll
   for (int u = 0; u < 32; ++u) t[u] = __ldg(Ti + (size_t)u * kHeadDim);
-  for (int i = tid; i < G * kHeadDim; i += 128) {
+  for (int i = tid; i < G * kHeadDim; i += kPrologueThreads) {
     const int hh = i / kHeadDim, cc = i % kHeadDim;
     qs[hh][cc] = __half2float(a.q[head_row(a, b, h, hh) * kHeadDim + cc]);
   }
   if (a.prep.enabled) {  // raw queries (fused step, bulk route): RMSNorm + RoPE at position S - 1
     __syncthreads();
     const int qpos = max(a.state[2 * unit] - 1, 0);
-    for (int hh = tid >> 5; hh < G; hh += 4) prep_head_warp(qs[hh], a.prep.q_gain, a.prep, qpos, tid & 31);
+    for (int hh = tid >> 5; hh < G; hh += kPrologueThreads / 32)
+      prep_head_warp(qs[hh], a.prep.q_gain, a.prep, qpos, tid & 31);
   }
   __syncthreads();
   float qp[G];
@@ -188,101 +162,47 @@ __global__ void __launch_bounds__(128) decode_prologue_kernel(const DecodeArgs a
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) qp[hh] = fmaf(t[u], qs[hh][32 * pt + u], qp[hh]);
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh) part[pt][hh][jj] = qp[hh];
+  for (int hh = 0; hh < G; ++hh) part[pt][hh][j] = qp[hh];
   __syncthreads();
-  for (int i = tid; i < G * 32; i += 128) {
-    const int hh = i / 32, q = i % 32;
-    a.qprime[((size_t)unit * G + hh) * kHeadDim + 32 * c + q] =
-        (part[0][hh][q] + part[1][hh][q]) + (part[2][hh][q] + part[3][hh][q]);
+  for (int i = tid; i < G * kHeadDim; i += kPrologueThreads) {
+    const int hh = i / kHeadDim, q = i % kHeadDim;
+    const float v = (part[0][hh][q] + part[1][hh][q]) + (part[2][hh][q] + part[3][hh][q]);
+    qs[hh][q] = v;
+    a.qprime[((size_t)unit * G + hh) * kHeadDim + q] = v;
   }
-  if (c == 0) {  // completion counters of the unit: its group counters, then the unit counter
-    const int ngroups = (a.n_split + kMergeGroup - 1) / kMergeGroup;
-    for (int i = tid; i < ngroups; i += 128) a.tickets[a.units + (size_t)unit * ngroups + i] = 0u;
-    if (tid == 0) a.tickets[unit] = 0u;
-  }
+  // completion counters of the unit: its group counters, then the unit counter
+  const int ngroups = (a.n_split + kMergeGroup - 1) / kMergeGroup;
+  for (int i = tid; i < ngroups; i += kPrologueThreads) a.tickets[a.units + (size_t)unit * ngroups + i] = 0u;
+  if (tid == 0) a.tickets[unit] = 0u;
+  __syncthreads();
+  build_query_frags<BITS, G>(qs, tid, kPrologueThreads, red, a.scale_log2, a.qfrag + (size_t)unit * kQFragBytes,
+                             [] { __syncthreads(); });
 }
 
-// The query-side B fragments of one lane, built in registers from q' (fp32, in global
-// memory): lane (g, t4) holds, for k-step j, n-tile nt and register r, four bytes = limb
-// l = 2*(nt / NHS) + (g & 1) of the fixed-point Q of head 4*(nt % NHS) + (g >> 1) at the
-// four dimensions key_slot maps (j, t4, r, byte) to.  Q_d = rint(q'_d / (sigma * scale_d)),
-// sigma = max_d |q'_d| / scale_d / 2^30 per head (scale_d = the power of two that masking
-// leaves on dimension d's codes).  Also returns, for the lane's logit head t4 + 4*hs, the
-// constants log2e*scale*sum(q') (zero-point term) and log2e*scale*sigma.
-template <int BITS, int G>
-__device__ __forceinline__ void build_query(const DecodeArgs& a, int unit, int g, int t4,
-                                            uint32_t (&bq)[4][GCfg<G>::NT][2], float (&Ah)[GCfg<G>::NHS],
-                                            float (&Bh)[GCfg<G>::NHS]) {
-  constexpr int NHS = GCfg<G>::NHS;
+// The unit's query fragments and per-head constants (built by the prologue or the fused
+// append, staged in shared memory), loaded by one lane: bq[j][nt][r], and for the lane's
+// logit head t4 + 4*hs the constants log2e*scale*sum(q') (zero-point term) and
+// log2e*scale*sigma.
+template <int G>
+__device__ __forceinline__ void load_query(const uint8_t* qfs, int lane, int t4, uint32_t (&bq)[4][GCfg<G>::NT][2],
+                                           float (&Ah)[GCfg<G>::NHS], float (&Bh)[GCfg<G>::NHS]) {
+  constexpr int NT = GCfg<G>::NT, NHS = GCfg<G>::NHS, FW = GCfg<G>::FW;
+  const uint4* src = reinterpret_cast<const uint4*>(qfs) + lane;
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
+  for (int m = 0; m < FW / 4; ++m) {
+    const uint4 u = src[32 * m];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int nt = 0; nt < GCfg<G>::NT; ++nt) bq[j][nt][0] = bq[j][nt][1] = 0u;
+    for (int e = 0; e < 4; ++e) {
+      const int idx = 4 * m + e;
+      bq[(idx >> 1) / NT][(idx >> 1) % NT][idx & 1] = w[e];
+    }
+  }
+  const float* hc = reinterpret_cast<const float*>(qfs + FW * 32 * 4);
 #pragma unroll
   for (int hs = 0; hs < NHS; ++hs) {
-    const int hh = 4 * hs + (g >> 1);
-    const float4* src = reinterpret_cast<const float4*>(a.qprime + ((size_t)unit * G + hh) * kHeadDim + 32 * t4);
-    // dimension 32*t4 + k: its masking scale is 2^l2s(k); pass 1: max and sum
-    float amax = 0.f, sum = 0.f;
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const float4 f = hh < G ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float fv[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int k = 4 * v + e;
-        const int l2s = BITS == 2 ? 2 * (k & 3) : 4 * (k & 1);
-        amax = fmaxf(amax, fabsf(fv[e]) * (1.0f / float(1 << l2s)));
-        sum += fv[e];
-      }
-    }
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-    const float sigma = amax > 0.f ? amax / kQMax : 1.0f;
-    const float rs = 1.0f / sigma;
-    const int lp = g & 1;
-    // pass 2 (values re-read from L1/L2): fixed-point digits into the fragment bytes
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const float4 f = hh < G ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float fv[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int k = 4 * v + e;
-        int j, r, i, l2s;
-        if (BITS == 2) {
-          r = k >> 4;
-          i = (k & 15) >> 2;
-          j = k & 3;
-          l2s = 2 * j;
-        } else {
-          const int wl = k >> 3;
-          r = wl & 1;
-          i = (k & 7) >> 1;
-          j = 2 * (wl >> 1) + (k & 1);
-          l2s = 4 * (k & 1);
-        }
-        const int Q = __float2int_rn(fv[e] * (rs / float(1 << l2s)));
-        // balanced base-256 digits, each in [-128, 127]
-        const int L0 = ((Q + 128) & 255) - 128;
-        const int Q1 = (Q - L0) >> 8;
-        const int L1 = ((Q1 + 128) & 255) - 128;
-        const int Q2 = (Q1 - L1) >> 8;
-        const int L2 = ((Q2 + 128) & 255) - 128;
-        const int L3 = (Q2 - L2) >> 8;
-        const uint32_t lo = (uint32_t)((lp ? L1 : L0) & 255), hi = (uint32_t)((lp ? L3 : L2) & 255);
-        bq[j][hs][r] |= lo << (8 * i);
-        bq[j][NHS + hs][r] |= hi << (8 * i);
-      }
-    }
-    // the lane's logit head is t4 + 4*hs: its totals live in lanes with g = 2*t4
-    const float sum_t = __shfl_sync(0xffffffffu, sum, 8 * t4);
-    const float sig_t = __shfl_sync(0xffffffffu, sigma, 8 * t4);
-    const bool ok = t4 + 4 * hs < G;
-    Ah[hs] = ok ? a.scale_log2 * sum_t : 0.f;
-    Bh[hs] = ok ? a.scale_log2 * sig_t : 0.f;
+    Ah[hs] = hc[t4 + 4 * hs];
+    Bh[hs] = hc[8 + t4 + 4 * hs];
   }
 }
 
@@ -297,7 +217,8 @@ struct Shared {
   static constexpr int kPv = kConsumers * G * kHeadDim * 4;  // [4][G][128] fp32, reuses the stages
   static constexpr int kArena = kStages > kPv ? kStages : kPv;
   static size_t bytes(int nitems) {
-    return (size_t)kArena + 2 * Cfg<BITS>::NSTAGE * 8 + sizeof(Merge) + (size_t)kPv + (size_t)nitems * G * 4;
+    return (size_t)kArena + 2 * Cfg<BITS>::NSTAGE * 8 + sizeof(Merge) + (size_t)kPv + kQFragBytes +
+           (size_t)nitems * G * 4;
   }
 };
 
@@ -671,25 +592,29 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
   }
 }
 
-// Merge `count` consecutive partials (m, l, pad, pad, o[128] per head, base 2, o not yet
-// normalised) of one unit.  dst != nullptr: write the merged partial there; else write the
-// normalised output rows of the unit's G query heads.  wts: shared [count][G].
+// Merge `count` (<= 32) consecutive partials (m, l, pad, pad, o[128] per head, base 2, o not
+// yet normalised) of one unit.  dst != nullptr: write the merged partial there; else write
+// the normalised output rows of the unit's G query heads.  wts: shared [count][G].  Lane
+// `it` of the warp of head hh reads partial it's (m, l) in one round trip.
+static_assert(kMergeGroup <= 32 && (kMaxSplits + kMergeGroup - 1) / kMergeGroup <= 32,
+              "a merge level reads at most one partial per lane");
 template <int G>
 __device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, int count, float* dst,
                                float* wts) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int hh = warp; hh < G; hh += kThreads / 32) {
-    float M = -CUDART_INF_F;
-    for (int it = lane; it < count; it += 32) M = fmaxf(M, __ldcg(src + ((size_t)it * G + hh) * kPartStride));
+    const bool has = lane < count;
+    float mi = -CUDART_INF_F, li = 0.f;
+    if (has) {
+      mi = __ldcg(src + ((size_t)lane * G + hh) * kPartStride);
+      li = __ldcg(src + ((size_t)lane * G + hh) * kPartStride + 1);
+    }
+    float M = mi;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
-    for (int it = lane; it < count; it += 32) {
-      const float mi = __ldcg(src + ((size_t)it * G + hh) * kPartStride);
-      const float e = (M == -CUDART_INF_F) ? 0.f : exp2f(mi - M);
-      wts[it * G + hh] = e;
-      L = fmaf(e, __ldcg(src + ((size_t)it * G + hh) * kPartStride + 1), L);
-    }
+    const float e = (!has || M == -CUDART_INF_F) ? 0.f : exp2f(mi - M);
+    if (has) wts[lane * G + hh] = e;
+    float L = fmaf(e, li, 0.f);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
     __syncwarp();
@@ -738,7 +663,8 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   uint64_t* empty = full + C::NSTAGE;
   Merge* mg = reinterpret_cast<Merge*>(empty + C::NSTAGE);
   float* wpv = reinterpret_cast<float*>(mg + 1);   // window path [4][G][128]
-  float* wts = wpv + kConsumers * G * kHeadDim;    // [nitems][G] (last item only)
+  uint8_t* qfs = reinterpret_cast<uint8_t*>(wpv + kConsumers * G * kHeadDim);  // the unit's query fragments
+  float* wts = reinterpret_cast<float*>(qfs + kQFragBytes);  // [nitems][G] (last item only)
   __shared__ uint32_t s_last;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -821,15 +747,23 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     // for the prologue (they do not depend on it), the rest while the first tiles land
     WinRows<G> wr;
     window_load<G>(a, unit, wbeg + warp, wend, n_sink, r0, lane, wr);
-    griddep_wait();  // q', its constants and the counter resets come from the prologue
+    griddep_wait();  // q', the query fragments and the counter resets come from the prologue
+    {  // the unit's query fragments into shared memory while the window share runs
+      constexpr int n16 = GCfg<G>::FW * 8 + 4;
+      const uint8_t* src = a.qfrag + (size_t)unit * kQFragBytes;
+      for (int i = tid; i < n16; i += kConsumers * 32) cp_async16(qfs + 16 * i, src + 16 * i);
+      cp_async_commit();
+    }
     const int qlim = a.chunk_n > 0 ? S - a.chunk_n + a.chunk_t0 : INT_MAX;
     window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, wr, mg, wpv, qlim);
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) qs.o[mt][0] = qs.o[mt][1] = qs.o[mt][2] = qs.o[mt][3] = 0.f;
     // (b) quantized positions
+    cp_async_wait_all();
+    bar_sync(1, kConsumers * 32);  // every consumer thread's copies have landed
     uint32_t bq[4][NT][2];
     float Ah[NHS], Bh[NHS];
-    build_query<BITS, G>(a, unit, g, t4, bq, Ah, Bh);
+    load_query<G>(qfs, lane, t4, bq, Ah, Bh);
     const int base = kSlice * warp;
     for (int t = 0; t < ntiles; ++t) {
       const int s = t % C::NSTAGE;
@@ -968,7 +902,7 @@ cudaError_t launch_main_t(const Derived& d, const DecodeArgs& a, cudaStream_t st
 
 template <int BITS, int G>
 cudaError_t launch_decode_t(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
-  decode_prologue_kernel<G><<<dim3(d.units, 4), 128, 0, st>>>(a);
+  decode_prologue_kernel<BITS, G><<<d.units, kPrologueThreads, 0, st>>>(a);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // the main kernel may start before the prologue ends; its consumers wait

@@ -30,7 +30,7 @@ struct Derived {
   float f_lo, f_hi;
   int n_split, split_tokens;
   // workspace offsets (bytes)
-  size_t ws_tickets, ws_qprime, ws_partials, ws_gpartials, ws_total;
+  size_t ws_tickets, ws_qprime, ws_qfrag, ws_partials, ws_gpartials, ws_total;
   // cache buffer sizes (bytes)
   size_t codes_bytes, params_bytes, sink_bytes, ring_bytes, state_bytes;
 };
@@ -60,6 +60,8 @@ struct AppendArgs {
   const __half* q;
   const float* t_k_inv;
   float* qprime;
+  uint8_t* qfrag;      // the unit's query fragments for the decode kernel (qfrag.cuh)
+  float scale_log2;    // softmax_scale * log2(e)
   uint32_t* tickets;
   int Hq, ngroups;
   PrepSpec prep;  // raw q / k (wushkv_step_prep): RMSNorm + RoPE fused in
@@ -87,7 +89,8 @@ struct DecodeArgs {
   int out_fp16;
   int units;
   uint32_t* tickets;   // [units] unit counters, then [units][ngroups] group counters
-  float* qprime;
+  float* qprime;       // [units][G][128] fp32
+  uint8_t* qfrag;      // [units][kQFragBytes]: query fragments and constants (qfrag.cuh)
   float* partials;     // [units][n_split][G][132]
   float* gpartials;    // [units][ngroups][G][132]
   int wait_all;        // 1: the preceding kernel writes the cache (fused step): wait before any read
