@@ -356,11 +356,25 @@ def run_gpu(args, rank, world, local_rank):
         g_step.append(gs)
         g_app.append(ga)
         g_dec.append(gd)
+    # the timed path as a serving engine launches it: one graph holding the fused steps of
+    # all L layers in layer order (one graph launch per decode step of the model)
+    g_model = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_model, stream=stream):
+        for c in range(L):
+            caches[c].step(k_pool[c % P], v_pool[c % P], tks[c], q_pool[c % P], tinvs[c], scale, out=outs[c],
+                           stream=stream)
     # capture does not execute; the state mirrors stay in step with the device state
 
     def step_graphs(n, first):
-        for j in range(n):
-            g_step[(first + j) % L].replay()
+        j = 0
+        while j < n:
+            c = (first + j) % L
+            if c == 0 and n - j >= L:
+                g_model.replay()
+                j += L
+            else:
+                g_step[c].replay()
+                j += 1
 
     def split_graphs(n, first, evs):
         for j in range(n):
@@ -490,7 +504,8 @@ def run_gpu(args, rank, world, local_rank):
             "layers_rotated": L,
             "l2": f"inputs larger than L2: {L} rotating layer caches, "
                   f"{L * (bnd.pack_layout(cfg).codes_bytes * 2 + bnd.pack_layout(cfg).params_bytes * 2) / 1e9:.1f} GB",
-            "launch": "per-layer CUDA graphs of wushkv_step (append fused with decode)",
+            "launch": "one CUDA graph per model decode step: wushkv_step (append fused with decode) of "
+                      "each rotated layer in turn; per-layer graphs where K does not fill a whole step",
             "per_kernel_timing": "append and decode as separate calls, events per launch, "
                                  "min(K, 4000) more steps of the same workload",
             "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",

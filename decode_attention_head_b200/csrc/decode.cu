@@ -592,12 +592,13 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
   }
 }
 
-// Merge `count` (<= 32) consecutive partials (m, l, pad, pad, o[128] per head, base 2, o not
+// Merge `count` (<= kMergeMax) consecutive partials (m, l, pad, pad, o[128] per head, base 2, o not
 // yet normalised) of one unit.  dst != nullptr: write the merged partial there; else write
 // the normalised output rows of the unit's G query heads.  wts: shared [count][G].  Lane
 // `it` of the warp of head hh reads partial it's (m, l) in one round trip.
-static_assert(kMergeGroup <= 32 && (kMaxSplits + kMergeGroup - 1) / kMergeGroup <= 32,
-              "a merge level reads at most one partial per lane");
+constexpr int kMergeMax = 16;  // partials one merge level reads at most
+static_assert(kMergeGroup <= kMergeMax && (kMaxSplits + kMergeGroup - 1) / kMergeGroup <= kMergeMax,
+              "a merge level reads at most kMergeMax partials (one per lane of a warp)");
 template <int G>
 __device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, int count, float* dst,
                                float* wts) {
@@ -631,21 +632,39 @@ __device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, 
   }
   __syncthreads();
   const int b = unit / a.Hkv, h = unit % a.Hkv;
-  for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
-    const int hh = idx / kHeadDim, d = idx % kHeadDim;
-    float acc = 0.f;
-    // every partial is finite (an empty one holds o = 0), so no term needs skipping
-#pragma unroll 4
-    for (int it = 0; it < count; ++it)
-      acc = fmaf(wts[it * G + hh], __ldcg(src + ((size_t)it * G + hh) * kPartStride + 4 + d), acc);
+  // thread (hh, quad) takes dimensions 4*quad .. 4*quad+3: every partial's row is loaded at
+  // once (one round trip), then they are summed in partial order.  Every partial is finite
+  // (an empty one holds o = 0), so no term needs skipping.
+  constexpr int kQuads = kHeadDim / 4;
+  for (int idx = tid; idx < G * kQuads; idx += kThreads) {
+    const int hh = idx / kQuads, d = 4 * (idx % kQuads);
+    float4 ov[kMergeMax];
+#pragma unroll
+    for (int it = 0; it < kMergeMax; ++it)
+      ov[it] = it < count ? __ldcg(reinterpret_cast<const float4*>(src + ((size_t)it * G + hh) * kPartStride + 4 + d))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int it = 0; it < kMergeMax; ++it) {
+      if (it < count) {
+        const float w = wts[it * G + hh];
+        acc.x = fmaf(w, ov[it].x, acc.x);
+        acc.y = fmaf(w, ov[it].y, acc.y);
+        acc.z = fmaf(w, ov[it].z, acc.z);
+        acc.w = fmaf(w, ov[it].w, acc.w);
+      }
+    }
     if (dst) {
-      dst[hh * kPartStride + 4 + d] = acc;
+      *reinterpret_cast<float4*>(dst + hh * kPartStride + 4 + d) = acc;
     } else {
       const size_t o = head_row(a, b, h, hh) * kHeadDim + d;
-      if (a.out_fp16)
-        reinterpret_cast<__half*>(a.out)[o] = __float2half_rn(acc);
-      else
-        reinterpret_cast<float*>(a.out)[o] = acc;
+      if (a.out_fp16) {
+        __half2* oh = reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + o);
+        oh[0] = __floats2half2_rn(acc.x, acc.y);
+        oh[1] = __floats2half2_rn(acc.z, acc.w);
+      } else {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + o) = acc;
+      }
     }
   }
 }
