@@ -242,8 +242,11 @@ static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv
   a->B = cfg->batch;
   a->Hkv = cfg->n_kv_heads;
   a->Hq = cfg->n_q_heads;
+  a->cap = cfg->capacity;
   a->cap_alloc = d.cap_alloc;
   a->s_sink = cfg->s_sink;
+  a->s_keep = cfg->s_keep;
+  a->s_flush = cfg->s_flush;
   a->R = d.ring;
   a->sink_dim = d.sink_dim;
   a->n_split = d.n_split;
@@ -270,7 +273,8 @@ static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv
   a->partials = reinterpret_cast<float*>(ws + d.ws_partials);
   a->gpartials = reinterpret_cast<float*>(ws + d.ws_gpartials);
   a->units = d.units;
-  a->wait_all = 0;
+  a->fused = 0;
+  a->n_new = 0;
   a->gq = d.group;
   a->chunk_n = 0;
   a->chunk_t0 = 0;
@@ -364,6 +368,7 @@ static int step_impl(const wushkv_config* cfg, const wushkv_cache* cache, const 
   if (n_new <= cfg->chunk_max) {
     // one kernel appends and prepares the decode (q', counters); the main decode kernel
     // is its programmatic dependent and waits for it before reading the cache
+    aa.defer_state = 1;
     aa.q = da.q;
     aa.t_k_inv = da.t_k_inv;
     aa.qprime = da.qprime;
@@ -372,7 +377,8 @@ static int step_impl(const wushkv_config* cfg, const wushkv_cache* cache, const 
     aa.tickets = da.tickets;
     e = launch_append_fused(d, cfg->bits, aa, st);
     if (e == cudaSuccess) {
-      da.wait_all = 1;
+      da.fused = 1;
+      da.n_new = n_new;
       e = launch_decode_main(d, cfg->bits, da, st);
     }
   } else {

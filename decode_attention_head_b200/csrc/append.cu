@@ -32,9 +32,7 @@ struct FlushPlan {
 
 __device__ __forceinline__ FlushPlan flush_plan(int Sq, int L, const AppendArgs& a) {
   FlushPlan f;
-  f.lo0 = max(Sq, a.s_sink);
-  const int e = L - a.s_keep - f.lo0;
-  f.nf = (e >= a.s_flush) ? (e / a.s_flush) * a.s_flush : 0;
+  flush_bounds(Sq, L, a.s_sink, a.s_keep, a.s_flush, f.lo0, f.nf);
   return f;
 }
 
@@ -231,8 +229,8 @@ __global__ void __launch_bounds__(G > 0 ? 256 : 128) append_small_kernel(const A
     }
     bar_sync(1, 128);  // ks is rewritten by the next token
   }
-  // 3. state
-  if (threadIdx.x == 0) {
+  // 3. state (a fused step's decode kernel writes it instead, once it has read the old one)
+  if (threadIdx.x == 0 && !a.defer_state) {
     a.state[2 * unit] = S + a.n_new;
     if (fp.nf) a.state[2 * unit + 1] = fp.lo0 + fp.nf;
   }

@@ -4,20 +4,22 @@
 // §4.4 fp16 sink / recent windows around the quantized middle region).
 //
 // Two launches per call:
-//  1. decode_prologue (four CTAs per (sequence, KV head), a quarter of the dimensions
-//     each): q'_j = T_K^{-T} q_j for its g query heads in fp32, and the reset of the
-//     unit's completion counters.  It releases the main kernel at once (programmatic
-//     dependent launch), so the main kernel's KV stream starts while it runs.  (In a
-//     fused step, wushkv_step, the append kernel does this work instead and the main
-//     kernel waits for it before reading anything.)
+//  1. decode_prologue (one 512-thread CTA per (sequence, KV head)): q'_j = T_K^{-T} q_j
+//     for its g query heads in fp32, the query's fixed-point tensor-core fragments built
+//     from it (qfrag.cuh), and the reset of the unit's completion counters.  It releases
+//     the main kernel at once (programmatic dependent launch), so the main kernel's KV
+//     stream starts while it runs.  (In a fused step, wushkv_step, the append kernel does
+//     this work instead; the main kernel then derives the post-append state itself,
+//     streams the tiles the append cannot touch at once and waits for the append before
+//     reading anything else -- see DecodeArgs::fused.)
 //  2. decode_main: grid (n_split, units).  Work item s of a unit takes the s-th share of
 //     the unit's current quantized region [S_sink, S_quant) (whole 128-position stages)
 //     and of its fp16 window positions (sink [0, S_sink) and recent [S_quant, S)).
 //     The quantized positions stream through shared memory in 128-position stages
 //     (K codes, V codes, K and V (s, z)) via bulk copies on an mbarrier ring: one
 //     producer warp, four consumer warps, 32 positions per consumer warp per stage.
-//     Each consumer warp re-expresses q' as a 31-bit fixed-point integer split into four
-//     signed 8-bit limbs, directly in the mma.sync B-fragment registers it needs:
+//     The consumer warps take q' as a 31-bit fixed-point integer split into four signed
+//     8-bit limbs, already laid out as the mma.sync B fragments they need:
 //       QK  : u8 codes x s8 query limbs on tensor cores (mma m16n8k32, exact int32),
 //             logit = log2e*scale*(z*sum(q') + s*sigma*D)  (dequantization folded);
 //       softmax: online, base 2, with a running max that may go stale by 2^8;
@@ -78,7 +80,7 @@ __device__ __forceinline__ size_t head_row(const DecodeArgs& a, int b, int h, in
 template <int BITS>
 struct Cfg {
   static constexpr int CB = 16 * BITS;
-  static constexpr int NSTAGE = BITS == 2 ? 4 : 3;
+  static constexpr int NSTAGE = BITS == 2 ? 4 : 2;  // 4-bit: two 17 KB stages keep four CTAs per SM
   static constexpr int STAGE = kTileTokens * (2 * CB + 8);
 };
 
@@ -209,6 +211,8 @@ __device__ __forceinline__ void load_query(const uint8_t* qfs, int lane, int t4,
 // ---------------------------------------------------------------------------------
 struct Merge {  // per pseudo-warp (0..3 quantized path, 4..7 window path) and head
   float m[8][8], l[8][8], bias[8][8];
+  float e[8][8];      // the pseudo-warps' weights 2^(m - M) in the item's merge
+  float M[8], L[8];   // the item's merged max and denominator per head
 };
 
 template <int BITS, int G>
@@ -558,7 +562,10 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
       float mn = m[hh];
 #pragma unroll
       for (int u = 0; u < KB; ++u) mn = fmaxf(mn, x[u][hh]);
-      const float al = ex2(m[hh] - mn);  // 2^-inf = 0 on the first batch
+      // no visible position yet (a causally masked head): every factor below is 2^-inf = 0
+      // rather than 2^(-inf - -inf) = NaN
+      const float ms = mn == -CUDART_INF_F ? 0.f : mn;
+      const float al = ex2(m[hh] - ms);  // 2^-inf = 0 on the first batch
       l[hh] *= al;
       o[hh][0] *= al;
       o[hh][1] *= al;
@@ -566,7 +573,7 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
       o[hh][3] *= al;
 #pragma unroll
       for (int u = 0; u < KB; ++u) {
-        const float p = ex2(x[u][hh] - mn);
+        const float p = ex2(x[u][hh] - ms);
         const float2 v01 = __half22float2(u32_as_h2(w.v[u].x)), v23 = __half22float2(u32_as_h2(w.v[u].y));
         l[hh] += p;
         o[hh][0] = fmaf(p, v01.x, o[hh][0]);
@@ -690,8 +697,21 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   const int g = lane >> 2, t4 = lane & 3;
   const int unit = blockIdx.y, item = blockIdx.x;
   const int nitems = a.n_split;
-  if (a.wait_all) griddep_wait();  // fused step: the append before this kernel writes the cache
   int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
+  // fused step: the state read above is the one before the append (that kernel leaves the
+  // state words to this one); the append's outcome follows from it as the append derives it
+  const int sq_stable = Sq;  // quantized positions below it are not touched by the append
+  int S_next = -1, Sq_next = 0;
+  if (a.fused) {
+    if (S >= 0 && S <= a.cap && Sq >= 0 && Sq <= S && S + a.n_new <= a.cap) {
+      int lo0, nf;
+      flush_bounds(Sq, S, a.s_sink, a.s_keep, a.s_flush, lo0, nf);  // the flush under the old S
+      S_next = S + a.n_new;
+      Sq_next = nf ? lo0 + nf : Sq;
+      S = S_next;
+      Sq = Sq_next;
+    }  // else the append is refused (it reports why): decode the cache as it stands
+  }
   if (S < 0 || S > a.cap_alloc || Sq < 0 || Sq > S) {  // never read outside the buffers
     if (tid == 0 && item == 0) atomicOr(a.status, kStatusBadState);
     S = 0;
@@ -744,8 +764,13 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     // ---------------- producer: streams the item's tiles; needs nothing from the prologue
     if (lane == 0 && ntiles > 0) {
       int issued = 0;
+      bool waited = !a.fused;  // fused step: tiles below the old S_quant stream at once
       for (int t = 0; t < ntiles; ++t) {
         const int s = t % C::NSTAGE;
+        if (!waited && tile0 + (t + 1) * kTileTokens > sq_stable) {
+          griddep_wait();
+          waited = true;
+        }
         if (t >= C::NSTAGE && !mbar_wait(&empty[s], ((t / C::NSTAGE) - 1) & 1, a.status)) break;
         uint8_t* st = stages + s * C::STAGE;
         const size_t rec = (size_t)unit * a.cap_alloc + tile0 + (size_t)t * kTileTokens;
@@ -765,6 +790,7 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     // (a) this warp's share of the fp16 window: the first rows are loaded before the wait
     // for the prologue (they do not depend on it), the rest while the first tiles land
     WinRows<G> wr;
+    if (a.fused) griddep_wait();  // the window holds the appended tokens
     window_load<G>(a, unit, wbeg + warp, wend, n_sink, r0, lane, wr);
     griddep_wait();  // q', the query fragments and the counter resets come from the prologue
     {  // the unit's query fragments into shared memory while the window share runs
@@ -838,28 +864,38 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   }
   __syncthreads();
 
-  // ======================= merge the 8 pseudo-warps, write this item's partial
-  float* part = a.partials + ((size_t)unit * nitems + item) * G * kPartStride;
-  for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
-    const int hh = idx / kHeadDim, d = idx % kHeadDim;
+  // ======================= merge the 8 pseudo-warps, write this item's partial: the
+  // weights once per (pseudo-warp, head), then the rows
+  if (tid < G) {
+    const int hh = tid;
     float M = -CUDART_INF_F;
 #pragma unroll
     for (int w = 0; w < 2 * kConsumers; ++w) M = fmaxf(M, mg->m[w][hh]);
-    float O = 0.f, L = 0.f;
-    if (M != -CUDART_INF_F) {
+    float L = 0.f;
 #pragma unroll
-      for (int w = 0; w < 2 * kConsumers; ++w) {
-        const float e = exp2f(mg->m[w][hh] - M);
-        const float ov = w < kConsumers ? pv[((size_t)w * G + hh) * kHeadDim + d]
-                                        : wpv[((size_t)(w - kConsumers) * G + hh) * kHeadDim + d];
-        O = fmaf(e, ov + mg->bias[w][hh], O);
-        L = fmaf(e, mg->l[w][hh], L);
-      }
+    for (int w = 0; w < 2 * kConsumers; ++w) {
+      const float e = M != -CUDART_INF_F ? exp2f(mg->m[w][hh] - M) : 0.f;
+      mg->e[w][hh] = e;
+      L = fmaf(e, mg->l[w][hh], L);
+    }
+    mg->M[hh] = M;
+    mg->L[hh] = L;
+  }
+  __syncthreads();
+  float* part = a.partials + ((size_t)unit * nitems + item) * G * kPartStride;
+  for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
+    const int hh = idx / kHeadDim, d = idx % kHeadDim;
+    float O = 0.f;
+#pragma unroll
+    for (int w = 0; w < 2 * kConsumers; ++w) {
+      const float ov = w < kConsumers ? pv[((size_t)w * G + hh) * kHeadDim + d]
+                                      : wpv[((size_t)(w - kConsumers) * G + hh) * kHeadDim + d];
+      O = fmaf(mg->e[w][hh], ov + mg->bias[w][hh], O);
     }
     part[hh * kPartStride + 4 + d] = O;
     if (d == 0) {
-      part[hh * kPartStride + 0] = M;
-      part[hh * kPartStride + 1] = L;
+      part[hh * kPartStride + 0] = mg->M[hh];
+      part[hh * kPartStride + 1] = mg->L[hh];
     }
   }
   // ======================= two-level merge: the last item of each group of kMergeGroup
@@ -880,6 +916,10 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   const float* up = a.partials + ((size_t)unit * nitems + g0) * G * kPartStride;
   if (ngroups == 1) {
     merge_partials<G>(a, unit, up, gn, nullptr, wts);
+    if (S_next >= 0 && tid == 0) {  // every item of the unit has read the old state
+      a.state[2 * unit] = S_next;
+      a.state[2 * unit + 1] = Sq_next;
+    }
     return;
   }
   float* gp = a.gpartials + ((size_t)unit * ngroups + grp) * G * kPartStride;
@@ -891,6 +931,10 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   if (!s_last) return;
   __threadfence();
   merge_partials<G>(a, unit, a.gpartials + (size_t)unit * ngroups * G * kPartStride, ngroups, nullptr, wts);
+  if (S_next >= 0 && tid == 0) {  // every item of the unit has read the old state
+    a.state[2 * unit] = S_next;
+    a.state[2 * unit + 1] = Sq_next;
+  }
 }
 
 // The main kernel as the programmatic dependent of the kernel before it in the stream: it

@@ -38,6 +38,16 @@ struct Derived {
 // Validates cfg and fills d; returns WUSHKV_OK / WUSHKV_EINVAL / WUSHKV_EUNSUPPORTED.
 int derive(const wushkv_config* cfg, Derived* d);
 
+// The flush under length L of a (sequence, KV head) whose quantized region ends at Sq:
+// lo0 = max(Sq, S_sink); e = L - S_keep - lo0; e >= S_flush -> nf = floor(e / S_flush) *
+// S_flush positions [lo0, lo0 + nf) are quantized and S_quant moves to lo0 + nf (else nf = 0).
+__host__ __device__ __forceinline__ void flush_bounds(int Sq, int L, int s_sink, int s_keep, int s_flush, int& lo0,
+                                                     int& nf) {
+  lo0 = Sq > s_sink ? Sq : s_sink;
+  const int e = L - s_keep - lo0;
+  nf = (e >= s_flush) ? (e / s_flush) * s_flush : 0;
+}
+
 struct AppendArgs {
   int B, Hkv, cap, cap_alloc, s_sink, s_keep, s_flush, R, sink_dim, n_new;
   uint8_t* k_codes;
@@ -65,13 +75,14 @@ struct AppendArgs {
   uint32_t* tickets;
   int Hq, ngroups;
   PrepSpec prep;  // raw q / k (wushkv_step_prep): RMSNorm + RoPE fused in
+  int defer_state;  // 1 (fused step): leave the state words to the decode kernel that follows
   int transform;  // WUSHKV_TRANSFORM_DENSE (t_k) or WUSHKV_TRANSFORM_HADAMARD (in-kernel)
   int quant_rms;            // WUSHKV_QUANT_RMS: (s, z) from the token's RMS, not its percentiles
   float rms_kb, rms_alpha;  // fp32(2*alpha/(2^b-1)), fp32(alpha)
 };
 
 struct DecodeArgs {
-  int B, Hkv, Hq, cap_alloc, s_sink, R, sink_dim, n_split, split_tokens;
+  int B, Hkv, Hq, cap, cap_alloc, s_sink, s_keep, s_flush, R, sink_dim, n_split, split_tokens;
   const uint8_t* k_codes;
   const uint8_t* v_codes;
   const uint32_t* k_params;
@@ -80,7 +91,7 @@ struct DecodeArgs {
   const __half* v_sink;
   const __half* k_ring;
   const __half* v_ring;
-  const int32_t* state;
+  int32_t* state;     // read; written only in a fused step (below)
   uint32_t* status;
   const __half* q;
   const float* t_k_inv;
@@ -93,7 +104,12 @@ struct DecodeArgs {
   uint8_t* qfrag;      // [units][kQFragBytes]: query fragments and constants (qfrag.cuh)
   float* partials;     // [units][n_split][G][132]
   float* gpartials;    // [units][ngroups][G][132]
-  int wait_all;        // 1: the preceding kernel writes the cache (fused step): wait before any read
+  // fused step (wushkv_step's one-kernel append of n_new tokens runs just before): that
+  // kernel leaves the state words alone, so this one reads the pre-append state, derives the
+  // post-append (S, S_quant) from it, streams the tiles below the old S_quant before the
+  // append has finished (nothing there changes), reads everything else after it, and writes
+  // the new state once every item of the unit has read the old one (the final merge).
+  int fused, n_new;
   // chunk attention (wushkv_chunk_attn): the kernel's G query heads per unit are gq real
   // heads of each of G / gq consecutive chunk tokens, chunk_t0 the first of them; q and out
   // are [B][chunk_n][H_q][128]; chunk_n = 0 for a one-token decode (gq = G)
