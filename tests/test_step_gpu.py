@@ -91,3 +91,36 @@ def test_step_refused_append_still_decodes():
     assert g.status() & bnd.STATUS_OVERFLOW
     assert int(g.lengths()[0][0, 0]) == 300
     assert (out - ref).abs().max().item() <= 1e-5
+
+
+def test_step_with_corrupt_state_is_isolated():
+    """A fused step over a cache whose (sequence 1, KV head 0) state word is corrupt: that
+    unit is reported (STATUS_BADSTATE), not appended to and decoded as empty; every other
+    unit is appended to, advances its state and decodes like append + decode on a twin."""
+    cfg = bnd.make_config(2, 2, 8, 2, 500, 4, 32, 16, 1)
+    T = np.broadcast_to(np.eye(128, dtype=np.float16), (2, 128, 128)).copy()
+    t_dev = H.to_dev(T)
+    tinv = bnd.compensation(torch.from_numpy(T)).cuda()
+    rng = np.random.default_rng(11)
+    ga, gb = bnd.KVCache(cfg), bnd.KVCache(cfg)
+    k = H.to_dev(_tokens(rng, 2, 300, 2))
+    for g in (ga, gb):
+        g.append(k, k, t_dev)
+    units = 4
+    for g in (ga, gb):
+        g.state[: 2 * units].view(units, 2)[2, 0] = 10 ** 6
+    for i in range(20):  # crosses a flush boundary of the healthy units
+        one = H.to_dev(_tokens(rng, 2, 1, 2))
+        q = H.to_dev(rng.standard_normal((2, 8, 128)).astype(np.float16))
+        out_a = ga.step(one, one, t_dev, q, tinv, 0.1)
+        gb.append(one, one, t_dev)
+        out_b = gb.decode_attn(q, tinv, 0.1)
+        torch.cuda.synchronize()
+        assert torch.isfinite(out_a).all()
+        assert torch.all(out_a[1, 0:4] == 0)
+        assert (out_a - out_b).abs().max().item() <= 1e-5, i
+    assert ga.status() & bnd.STATUS_BADSTATE
+    sa = ga.state[: 2 * units].view(units, 2).cpu()
+    sb = gb.state[: 2 * units].view(units, 2).cpu()
+    assert torch.equal(sa, sb)
+    assert int(sa[2, 0]) == 10 ** 6 and int(sa[0, 0]) == 320 and int(sa[3, 0]) == 320
