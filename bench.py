@@ -136,7 +136,7 @@ def code_sha256(paths):
 
 
 # the decode kernels' source: decode.cu and the headers it includes from csrc/
-DECODE_SOURCES = ("decode.cu", "internal.h", "ptx.cuh", "prep.cuh")
+DECODE_SOURCES = ("decode.cu", "internal.h", "ptx.cuh", "prep.cuh", "qfrag.cuh")
 
 
 def profile_traffic(kernel_file):

@@ -83,7 +83,7 @@ __device__ void quantize_ring_range(const AppendArgs& a, int unit, int p_begin, 
 // unit's query fragments for the decode kernel (qfrag.cuh).
 template <int BITS, int G>
 __device__ void prepare_query(const AppendArgs& a, int unit, int tid, int qpos) {
-  __shared__ float qs[G][kHeadDim];
+  __shared__ __align__(16) float qs[G][kHeadDim];
   __shared__ float red[4][G][kHeadDim];
   const int b = unit / a.Hkv, h = unit % a.Hkv;
   const int warp = tid >> 5, lane = tid & 31;

@@ -133,7 +133,7 @@ constexpr int kPrologueThreads = 512;
 
 template <int BITS, int G>
 __global__ void __launch_bounds__(kPrologueThreads) decode_prologue_kernel(const DecodeArgs a) {
-  __shared__ float qs[G][kHeadDim];  // q, then q'
+  __shared__ __align__(16) float qs[G][kHeadDim];  // q, then q'
   __shared__ float part[4][G][kHeadDim];
   __shared__ float red[64];
   griddep_launch();

@@ -47,27 +47,37 @@ __device__ __forceinline__ void frag_dim(int j, int r, int t4, int byte, int& di
 }
 
 // Build the unit's fragments from q' (fp32 [G][128] in shared memory) with `nthr` threads
-// (tid = 0 .. nthr-1, all of them calling).  red: shared scratch of 2 * 8 * 4 floats.
-// sync() is the barrier of those threads (a named barrier in a kernel whose other threads
-// do other work).  The per-head sum is taken in the order (s0 + s1) + (s2 + s3), s_c the
-// left-to-right sum over dimensions 32c .. 32c+31.
+// (tid = 0 .. nthr-1, a multiple of 32, all of them calling; qf 16-byte aligned).  red: shared scratch of
+// 2 * 8 floats.  sync() is the barrier of those threads (a named barrier in a kernel whose
+// other threads do other work).  Per head, one warp reduces max |q'_d / scale_d| and the
+// sum of q' (lane l holds dimensions 4l .. 4l+3; xor-shuffle tree, a fixed order).
 template <int BITS, int G, typename Sync>
 __device__ __forceinline__ void build_query_frags(const float (*qf)[kHeadDim], int tid, int nthr, float* red,
                                                   float scale_log2, uint8_t* out, Sync sync) {
   constexpr int NHS = GCfg<G>::NHS, NT = GCfg<G>::NT, FW = GCfg<G>::FW;
-  float* amax_q = red;           // [G][4]
-  float* sum_q = red + 8 * 4;    // [G][4]
-  for (int i = tid; i < G * 4; i += nthr) {
-    const int hh = i >> 2, c = i & 3;
-    float amax = 0.f, sum = 0.f;
-    for (int k = 0; k < 32; ++k) {
-      const float v = qf[hh][32 * c + k];
+  float* amax_h = red;      // [G]
+  float* sum_h = red + 8;   // [G]
+  const int wl = tid & 31;
+  for (int hh = tid >> 5; hh < G; hh += nthr >> 5) {
+    const float4 v = *reinterpret_cast<const float4*>(&qf[hh][4 * wl]);
+    const float fv[4] = {v.x, v.y, v.z, v.w};
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int k = 4 * wl + e;  // the key-code scale depends on the dimension's low bits
       const int l2s = BITS == 2 ? 2 * (k & 3) : 4 * (k & 1);
-      amax = fmaxf(amax, fabsf(v) * (1.0f / float(1 << l2s)));
-      sum += v;
+      amax = fmaxf(amax, fabsf(fv[e]) * (1.0f / float(1 << l2s)));
     }
-    amax_q[i] = amax;
-    sum_q[i] = sum;
+    float sum = (fv[0] + fv[1]) + (fv[2] + fv[3]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    }
+    if (wl == 0) {
+      amax_h[hh] = amax;
+      sum_h[hh] = sum;
+    }
   }
   sync();
   uint32_t* words = reinterpret_cast<uint32_t*>(out);
@@ -79,7 +89,7 @@ __device__ __forceinline__ void build_query_frags(const float (*qf)[kHeadDim], i
     const int limb = 2 * (nt / NHS) + (g & 1);
     uint32_t word = 0u;
     if (hh < G) {
-      const float amax = fmaxf(fmaxf(amax_q[4 * hh], amax_q[4 * hh + 1]), fmaxf(amax_q[4 * hh + 2], amax_q[4 * hh + 3]));
+      const float amax = amax_h[hh];
       const float sigma = amax > 0.f ? amax / kQMax : 1.0f;
       const float rs = 1.0f / sigma;
 #pragma unroll
@@ -106,10 +116,9 @@ __device__ __forceinline__ void build_query_frags(const float (*qf)[kHeadDim], i
     float v = 0.f;
     if (hh < G) {
       if (i < 8) {
-        v = scale_log2 * ((sum_q[4 * hh] + sum_q[4 * hh + 1]) + (sum_q[4 * hh + 2] + sum_q[4 * hh + 3]));
+        v = scale_log2 * sum_h[hh];
       } else {
-        const float amax =
-            fmaxf(fmaxf(amax_q[4 * hh], amax_q[4 * hh + 1]), fmaxf(amax_q[4 * hh + 2], amax_q[4 * hh + 3]));
+        const float amax = amax_h[hh];
         v = scale_log2 * (amax > 0.f ? amax / kQMax : 1.0f);
       }
     }
