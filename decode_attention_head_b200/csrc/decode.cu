@@ -610,6 +610,20 @@ template <int G>
 __device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, int count, float* dst,
                                float* wts) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // thread (hh, quad) takes dimensions 4*quad .. 4*quad+3 of head hh: every partial's row is
+  // loaded at once, the first (head, quad)'s rows before the weights are known, so that
+  // their round trip overlaps the (m, l) one; then they are summed in partial order.  Every
+  // partial is finite (an empty one holds o = 0), so no term needs skipping.
+  constexpr int kQuads = kHeadDim / 4;
+  float4 ov[kMergeMax];
+  auto load_rows = [&](int idx) {
+    const int hh = idx / kQuads, d = 4 * (idx % kQuads);
+#pragma unroll
+    for (int it = 0; it < kMergeMax; ++it)
+      ov[it] = it < count ? __ldcg(reinterpret_cast<const float4*>(src + ((size_t)it * G + hh) * kPartStride + 4 + d))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  if (tid < G * kQuads) load_rows(tid);
   for (int hh = warp; hh < G; hh += kThreads / 32) {
     const bool has = lane < count;
     float mi = -CUDART_INF_F, li = 0.f;
@@ -639,17 +653,9 @@ __device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, 
   }
   __syncthreads();
   const int b = unit / a.Hkv, h = unit % a.Hkv;
-  // thread (hh, quad) takes dimensions 4*quad .. 4*quad+3: every partial's row is loaded at
-  // once (one round trip), then they are summed in partial order.  Every partial is finite
-  // (an empty one holds o = 0), so no term needs skipping.
-  constexpr int kQuads = kHeadDim / 4;
   for (int idx = tid; idx < G * kQuads; idx += kThreads) {
     const int hh = idx / kQuads, d = 4 * (idx % kQuads);
-    float4 ov[kMergeMax];
-#pragma unroll
-    for (int it = 0; it < kMergeMax; ++it)
-      ov[it] = it < count ? __ldcg(reinterpret_cast<const float4*>(src + ((size_t)it * G + hh) * kPartStride + 4 + d))
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (idx != tid) load_rows(idx);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int it = 0; it < kMergeMax; ++it) {
