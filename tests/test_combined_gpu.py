@@ -54,7 +54,23 @@ def test_all_options_together(bits, Hkv, Hq):
             # fp16 output: one more rounding of the result
             H.assert_attention_close(out.float().cpu().numpy(), ref, atol=2e-3 + 1e-3 * np.abs(ref).max())
     assert np.array_equal(gc.lengths()[0][:, 0].cpu().numpy(), np.full(B, S))
-    st = H.compare_caches(oc, H.download(gc), cfg, gc.layout.ring_slots, exact=False)
+    g = H.download(gc)
+    st = H.compare_caches(oc, g, cfg, gc.layout.ring_slots, exact=False)
     print(f"[combined] cache vs oracle: {st}")
     assert st["code_maxdiff"] <= 1 and st["code_diff"] <= 1e-4 * st["code_elems"], st
-    assert st["fp16_maxulp"] <= 8 and st["param_diff"] <= 0.02 * st["param_tokens"], st
+    assert st["param_diff"] <= 0.02 * st["param_tokens"], st
+    # fp16 window keys: the GPU sums the butterflies in fp32, the oracle in float64, so a key
+    # may round to a neighbouring fp16 value; a key near zero (cancellation in the sum) is
+    # off by more of its own ulps, so the error is measured in ulps of its row's magnitude
+    worst = 0.0
+    for b in range(B):
+        Sq = int(g["Sq"][b, 0])
+        ns = min(cfg.s_sink, S)
+        rpos = np.arange(max(Sq, cfg.s_sink), S)
+        gk = np.concatenate([g["k_sink"][b][:, :ns], g["k_ring"][b][:, rpos % gc.layout.ring_slots]], axis=1)
+        ok = np.concatenate([oc.k_store[b][:, :ns], oc.k_store[b][:, rpos]], axis=1).astype(np.float64)
+        rowmax = np.abs(ok).max(axis=-1, keepdims=True)
+        ulp_row = np.exp2(np.floor(np.log2(np.maximum(rowmax, 2.0 ** -14))) - 10)
+        worst = max(worst, float((np.abs(gk.astype(np.float64) - ok) / ulp_row).max()))
+    print(f"[combined] fp16 window keys: max error {worst:.3f} ulps of the row magnitude")
+    assert worst <= 1.0
