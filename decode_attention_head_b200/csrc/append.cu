@@ -82,7 +82,7 @@ __device__ void quantize_ring_range(const AppendArgs& a, int unit, int p_begin, 
 // in shared memory.  Also resets the unit's decode completion counters and builds the
 // unit's query fragments for the decode kernel (qfrag.cuh).
 template <int BITS, int G>
-__device__ void prepare_query(const AppendArgs& a, int unit, int tid, int qpos) {
+__device__ void prepare_query(const AppendArgs& a, int unit, int tid) {
   __shared__ __align__(16) float qs[G][kHeadDim];
   __shared__ float red[4][G][kHeadDim];
   const int b = unit / a.Hkv, h = unit % a.Hkv;
@@ -95,6 +95,12 @@ __device__ void prepare_query(const AppendArgs& a, int unit, int tid, int qpos) 
   for (int i = tid; i < G * kHeadDim; i += 128)
     qs[i / kHeadDim][i % kHeadDim] = __half2float(a.q[((size_t)b * a.Hq + h * G) * kHeadDim + i]);
   if (a.prep.enabled) {  // raw queries: RMSNorm + RoPE at the query's position, head by head
+    // the query is the newest token: position S + n_new - 1 (S - 1 if the append is refused);
+    // the state is read here, after the loads above are in flight
+    const int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
+    const bool valid = state_ok(S, Sq, a);
+    const bool fits = valid && S + a.n_new <= a.cap;
+    const int qpos = max((fits ? S + a.n_new : (valid ? S : 1)) - 1, 0);
     bar_sync(2, 128);
     for (int hh = warp; hh < G; hh += 4) prep_head_warp(qs[hh], a.prep.q_gain, a.prep, qpos, lane);
   }
@@ -136,19 +142,21 @@ template <int BITS, int NSEL, int G>
 __global__ void __launch_bounds__(G > 0 ? 256 : 128) append_small_kernel(const AppendArgs a) {
   const int unit = blockIdx.x;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
-  const int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
-  const bool valid = state_ok(S, Sq, a);
-  const bool fits = valid && S + a.n_new <= a.cap;
   if (G > 0) {
     griddep_launch();  // the decode kernel may launch now; it waits for this whole grid
-    __syncthreads();   // every thread has read the state before the append half rewrites it
+    // the unit's key transform into L2 while the state is read (the rows are loaded below)
+    if (threadIdx.x == 0 && a.transform == WUSHKV_TRANSFORM_DENSE)
+      bulk_prefetch_l2(a.t_k + (size_t)h * kHeadDim * kHeadDim, kHeadDim * kHeadDim * 2);
+    // the fused step leaves the state words to the decode kernel (defer_state), so the two
+    // halves need not order their reads of them
     if (threadIdx.x >= 128) {
-      // the query is the newest token: position S + n_new - 1 (S - 1 if the append is refused)
-      const int qpos = max((fits ? S + a.n_new : (valid ? S : 1)) - 1, 0);
-      prepare_query<BITS, (G > 0 ? G : 1)>(a, unit, threadIdx.x - 128, qpos);
+      prepare_query<BITS, (G > 0 ? G : 1)>(a, unit, threadIdx.x - 128);
       return;
     }
   }
+  const int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
+  const bool valid = state_ok(S, Sq, a);
+  const bool fits = valid && S + a.n_new <= a.cap;
   if (!valid) {
     if (threadIdx.x == 0) atomicOr(a.status, kStatusBadState);
     return;

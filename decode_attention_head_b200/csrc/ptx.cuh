@@ -79,6 +79,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Prefetch [src, src + bytes) into L2 (bulk; src 16-byte aligned, bytes a multiple of 16).
+// Only warms the cache: a later load still sees any newer write.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // 16-byte asynchronous global -> shared copy through L2 (cp.async); a group of them is
 // closed by cp_async_commit and waited for by cp_async_wait_all.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
