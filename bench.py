@@ -551,6 +551,7 @@ def run_gpu(args, rank, world, local_rank):
         del caches, outs
         torch.cuda.empty_cache()
         result["prefill_append"] = measure_prefill(bnd, synth, dev)
+        result["chunk_prefill"] = measure_chunk(bnd, synth, dev)
     return result, wl
 
 
@@ -623,6 +624,59 @@ def measure_prefill(bnd, synth, dev, reps=5):
             "reps": reps}
 
 
+def measure_chunk(bnd, synth, dev, n=8, reps=20):
+    """Chunked prefill on the Llama-3-8B-shaped layer: an n-token chunk appended to a cache of
+    32,768 - n positions (the decode-time append path), then its n queries attending
+    causally (wushkv_chunk_attn: ng = 8 / g tokens per pass over the cache).  Repeated from
+    the same state, each timed with CUDA events."""
+    import torch
+    wl = synth.WORKLOADS["llama3-8b-layer"]
+    base = wl.context - n
+    cfg = bnd.config_for_workload(wl, extra_capacity=64, chunk_max=n)
+    c = bnd.KVCache(cfg, device=dev)
+    T = synth.key_transforms(wl, 0)
+    tk, tinv = T.to(dev), bnd.compensation(T).to(dev)
+    for s0 in range(0, base, 4096):
+        m = min(4096, base - s0)
+        c.append(synth.bulk_tokens(wl, 0, s0, m, device=dev, which="k"),
+                 synth.bulk_tokens(wl, 0, s0, m, device=dev, which="v"), tk)
+    kk = synth.bulk_tokens(wl, 0, base, n, device=dev, which="k")
+    vv = synth.bulk_tokens(wl, 0, base, n, device=dev, which="v")
+    q = torch.stack([synth.bulk_queries(wl, 0, base + t, device=dev) for t in range(n)], dim=1).contiguous()
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+    state0, kring0, vring0 = c.state.clone(), c.k_ring.clone(), c.v_ring.clone()
+    scale = synth.default_softmax_scale(wl.head_dim)
+    app_ms, att_ms = [], []
+    for r in range(reps + 1):
+        c.state.copy_(state0)
+        c.k_ring.copy_(kring0)
+        c.v_ring.copy_(vring0)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        torch.cuda.synchronize()
+        e0.record()
+        c.append(kk, vv, tk)
+        e1.record()
+        c.chunk_attn(q, tinv, scale, out=out)
+        e2.record()
+        torch.cuda.synchronize()
+        if r:
+            app_ms.append(e0.elapsed_time(e1))
+            att_ms.append(e1.elapsed_time(e2))
+    assert c.status() == 0
+    att_s = sum(att_ms) / len(att_ms) / 1e3
+    app_s = sum(app_ms) / len(app_ms) / 1e3
+    S1, Sq1 = (int(t[0, 0].item()) for t in c.lengths())
+    ng = max(1, 8 // wl.group)
+    passes = (n + ng - 1) // ng
+    cache_bytes = StateMirror(wl, S1, Sq1).decode_bytes()
+    return {"workload": wl.name, "chunk_tokens": n, "cached_before": base,
+            "append_us": round(app_s * 1e6, 2), "chunk_attn_us": round(att_s * 1e6, 2),
+            "passes_over_cache": passes, "chunk_attn_gbs": round(passes * cache_bytes / att_s / 1e9, 2),
+            "query_tokens_per_s": round(wl.batch * n / (app_s + att_s), 1),
+            "launch": "eager: 1 append launch + 2 launches per pass (prologue, main)", "reps": reps}
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -662,6 +716,7 @@ def main():
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
         print(json.dumps(measure_prefill(bnd, synth, dev)))
+        print(json.dumps(measure_chunk(bnd, synth, dev)))
         return 0
     if world > 1:
         import datetime
