@@ -12,7 +12,7 @@ from oracle import attention as oatt
 from oracle import cache as ocache
 from oracle import quantizer as oq
 
-# attention-output tolerance (the benchmark spec: 2e-3 max abs, 1e-3 relative): both must hold,
+# attention-output tolerance of the path's specification (2e-3 max abs, 1e-3 relative): both must hold,
 # the relative one on the 2-norm of each output row
 ATOL = 2e-3
 RTOL = 1e-3
