@@ -133,26 +133,27 @@ __device__ void prepare_query(const AppendArgs& a, int unit, int tid) {
                              [] { bar_sync(2, 128); });
 }
 
-// Small append: one CTA per (sequence, KV head); threads 0..127 append.  G > 0: the fused
-// step (wushkv_step) also prepares the decode that follows (q' and its counters) on
-// threads 128..255, in parallel with the append and for every unit, including one whose
-// append is refused (its cache is decoded as it stands).  The two halves synchronise on
-// separate named barriers (1: append, 2: decode preparation).
+// Small append: one 128-thread CTA per (sequence, KV head).  G > 0: the fused step
+// (wushkv_step) also prepares the decode that follows (q', its query fragments and its
+// counters) in a second CTA per unit (blockIdx.y = 1), in parallel with the append and
+// for every unit, including one whose append is refused (its cache is decoded as it
+// stands).  Each role synchronises on its own named barrier (1: append, 2: decode
+// preparation).
 template <int BITS, int NSEL, int G>
-__global__ void __launch_bounds__(G > 0 ? 256 : 128) append_small_kernel(const AppendArgs a) {
+__global__ void __launch_bounds__(128) append_small_kernel(const AppendArgs a) {
   const int unit = blockIdx.x;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
   if (G > 0) {
     griddep_launch();  // the decode kernel may launch now; it waits for this whole grid
+    // the fused step leaves the state words to the decode kernel (defer_state), so the two
+    // roles need not order their reads of them
+    if (blockIdx.y == 1) {
+      prepare_query<BITS, (G > 0 ? G : 1)>(a, unit, threadIdx.x);
+      return;
+    }
     // the unit's key transform into L2 while the state is read (the rows are loaded below)
     if (threadIdx.x == 0 && a.transform == WUSHKV_TRANSFORM_DENSE)
       bulk_prefetch_l2(a.t_k + (size_t)h * kHeadDim * kHeadDim, kHeadDim * kHeadDim * 2);
-    // the fused step leaves the state words to the decode kernel (defer_state), so the two
-    // halves need not order their reads of them
-    if (threadIdx.x >= 128) {
-      prepare_query<BITS, (G > 0 ? G : 1)>(a, unit, threadIdx.x - 128);
-      return;
-    }
   }
   const int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
   const bool valid = state_ok(S, Sq, a);
@@ -489,10 +490,10 @@ cudaError_t launch_append_t(const Derived& d, bool small, const AppendArgs& a, c
 template <int BITS, int NSEL>
 cudaError_t launch_fused_t(const Derived& d, const AppendArgs& a, cudaStream_t st) {
   switch (d.group) {
-    case 1: append_small_kernel<BITS, NSEL, 1><<<d.units, 256, 0, st>>>(a); break;
-    case 2: append_small_kernel<BITS, NSEL, 2><<<d.units, 256, 0, st>>>(a); break;
-    case 4: append_small_kernel<BITS, NSEL, 4><<<d.units, 256, 0, st>>>(a); break;
-    default: append_small_kernel<BITS, NSEL, 8><<<d.units, 256, 0, st>>>(a); break;
+    case 1: append_small_kernel<BITS, NSEL, 1><<<dim3(d.units, 2), 128, 0, st>>>(a); break;
+    case 2: append_small_kernel<BITS, NSEL, 2><<<dim3(d.units, 2), 128, 0, st>>>(a); break;
+    case 4: append_small_kernel<BITS, NSEL, 4><<<dim3(d.units, 2), 128, 0, st>>>(a); break;
+    default: append_small_kernel<BITS, NSEL, 8><<<dim3(d.units, 2), 128, 0, st>>>(a); break;
   }
   return cudaGetLastError();
 }
