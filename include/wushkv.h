@@ -199,9 +199,13 @@ int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* cache, cons
 /* One decode step: wushkv_append(k_new, v_new, n_new) followed by wushkv_decode_attn(q) on
  * the same stream, with the same arguments, buffers and results as those two calls
  * (§4.4: the new tokens are appended in full precision and serve the step's attention).
- * With n_new <= chunk_max the append also prepares the decode (the compensated queries and
- * the workspace's counters) and the decode kernel is launched as its programmatic
- * dependent, so the step costs two kernel launches instead of three.  The decode of a
+ * With n_new <= chunk_max the append also prepares the decode (the compensated queries,
+ * their tensor-core fragments and the workspace's counters) and the decode kernel is
+ * launched as its programmatic dependent, so the step costs two kernel launches instead of
+ * three; the decode kernel then reads the quantized positions the append cannot touch while
+ * the append runs, and it is the decode kernel that advances the state words, at its end
+ * (the cache is in the same state as after the two separate calls once the step has
+ * completed in stream order).  The decode of a
  * sequence whose append is refused (STATUS_OVERFLOW) attends over its cache unchanged.
  * Returns WUSHKV_OK, WUSHKV_EINVAL, WUSHKV_EUNSUPPORTED or WUSHKV_ECUDA. */
 int wushkv_step(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
