@@ -124,3 +124,26 @@ def test_step_with_corrupt_state_is_isolated():
     sb = gb.state[: 2 * units].view(units, 2).cpu()
     assert torch.equal(sa, sb)
     assert int(sa[2, 0]) == 10 ** 6 and int(sa[0, 0]) == 320 and int(sa[3, 0]) == 320
+
+
+def test_step_with_no_new_tokens_is_a_decode():
+    """n_new = 0: the step appends nothing (a flush that is due still happens, as in
+    wushkv_append) and its output equals wushkv_decode_attn over the same cache."""
+    cfg = bnd.make_config(2, 2, 8, 2, 800, 4, 32, 16, 1)
+    T = np.broadcast_to(np.eye(128, dtype=np.float16), (2, 128, 128)).copy()
+    t_dev = H.to_dev(T)
+    tinv = bnd.compensation(torch.from_numpy(T)).cuda()
+    rng = np.random.default_rng(5)
+    ga, gb = bnd.KVCache(cfg), bnd.KVCache(cfg)
+    k = H.to_dev(_tokens(rng, 2, 300, 2))
+    for g in (ga, gb):
+        g.append(k, k, t_dev)
+    empty = torch.empty(2, 0, 2, 128, dtype=torch.float16, device="cuda")
+    q = H.to_dev(rng.standard_normal((2, 8, 128)).astype(np.float16))
+    out_a = ga.step(empty, empty, t_dev, q, tinv, 0.1)
+    gb.append(empty, empty, t_dev)
+    out_b = gb.decode_attn(q, tinv, 0.1)
+    torch.cuda.synchronize()
+    assert ga.status() == 0 and gb.status() == 0
+    assert (out_a - out_b).abs().max().item() <= 1e-5
+    _assert_same_cache(ga, gb)
