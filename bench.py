@@ -516,10 +516,7 @@ def run_gpu(args, rank, world, local_rank):
         "dtype": "u8xs8->s32 QK^T, f16xf16->f32 PV, f32 softmax (2-bit codes)",
         "data": "synthetic",
         "config": {
-            "workload": wl.name, "batch": wl.batch, "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads,
-            "head_dim": wl.head_dim, "context": wl.context, "bits": wl.bits, "clip_percentiles": [wl.p_lo, wl.p_hi],
-            "s_sink": wl.s_sink, "s_keep": wl.s_keep, "s_flush": wl.s_flush,
-            "step": "append 1 token/sequence + decode 1 query/sequence, one layer",
+            **workload_config(wl),
             "layers_rotated": L,
             "l2": f"inputs larger than L2: {L} rotating layer caches, "
                   f"{L * (bnd.pack_layout(cfg).codes_bytes * 2 + bnd.pack_layout(cfg).params_bytes * 2) / 1e9:.1f} GB",
@@ -624,6 +621,14 @@ def measure_prefill(bnd, synth, dev, reps=5):
             "reps": reps}
 
 
+def workload_config(wl):
+    """The workload keys both arms report in `config`."""
+    return {"workload": wl.name, "batch": wl.batch, "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads,
+            "head_dim": wl.head_dim, "context": wl.context, "bits": wl.bits, "clip_percentiles": [wl.p_lo, wl.p_hi],
+            "s_sink": wl.s_sink, "s_keep": wl.s_keep, "s_flush": wl.s_flush,
+            "step": "append 1 token/sequence + decode 1 query/sequence, one layer"}
+
+
 def measure_chunk(bnd, synth, dev, n=8, reps=20):
     """Chunked prefill on the Llama-3-8B-shaped layer: an n-token chunk appended to a cache of
     32,768 - n positions (the decode-time append path), then its n queries attending
@@ -699,7 +704,7 @@ def main():
                "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / max(steps, 1), 3), "higher_is_better": True,
                "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fp32 quantizer decisions)",
                "data": "synthetic", "impl": "reference",
-               "config": {"workload": wl.name, "batch": wl.batch, "context": wl.context, "bits": wl.bits},
+               "config": {**workload_config(wl), "sample": "bounded: see cpu_baseline.sample"},
                "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": sample},
                "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
