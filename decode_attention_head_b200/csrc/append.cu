@@ -69,9 +69,11 @@ __device__ void quantize_ring_range(const AppendArgs& a, int unit, int p_begin, 
     const __half* ring = kind ? a.v_ring : a.k_ring;
     const __half* row = ring + ((size_t)unit * a.R + (p % a.R)) * kHeadDim;
     const size_t rec = (size_t)unit * a.cap_alloc + p;
-    uint8_t* codes = (kind ? a.v_codes : a.k_codes) + rec * CB;
     uint32_t* params = (kind ? a.v_params : a.k_params) + rec;
-    quantize_row_part<BITS, NSEL, P>(row, tid % P, codes, params, qs);
+    if (kind)  // value codes: the position's 16-position group (cap_alloc is a multiple of 16)
+      quantize_row_part<BITS, NSEL, P>(row, tid % P, a.v_codes + (rec & ~(size_t)15) * CB, params, qs, p & 15);
+    else
+      quantize_row_part<BITS, NSEL, P>(row, tid % P, a.k_codes + rec * CB, params, qs);
   }
 }
 
@@ -431,8 +433,11 @@ __global__ void __launch_bounds__(kBulkThreads, 3) append_bulk_kernel(const Appe
             reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
         } else if (p < sq_new) {
           const size_t rec = (size_t)unit * a.cap_alloc + p;
-          quantize_row_part<BITS, NSEL, 2>(src, part, (kind ? a.v_codes : a.k_codes) + rec * CB,
-                                           (kind ? a.v_params : a.k_params) + rec, qs);
+          if (kind)  // value codes: the position's 16-position group
+            quantize_row_part<BITS, NSEL, 2>(src, part, a.v_codes + (rec & ~(size_t)15) * CB, a.v_params + rec, qs,
+                                             p & 15);
+          else
+            quantize_row_part<BITS, NSEL, 2>(src, part, a.k_codes + rec * CB, a.k_params + rec, qs);
         } else {
           __half* dst = (kind ? a.v_ring : a.k_ring) + ((size_t)unit * a.R + p % a.R) * kHeadDim;
           for (int i = 8 * part; i < 8 * part + 8; ++i)

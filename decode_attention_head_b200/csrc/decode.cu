@@ -439,13 +439,13 @@ __device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, 
         pbl[0] = pbl[1] = 0u;
       }
     }
-    const int ta = base + 16 * i + t4;
+    // the V codes of k-block i are one 16-position group in the value layout (vgroup_half):
+    // lane (g, t4) reads the words pairing positions (t4, t4 + 8) and (t4 + 4, t4 + 12) for
+    // its chunks -- four consecutive words, one 16-byte load, the warp's loads contiguous
+    const uint8_t* vgrp = vc + (size_t)(base + 16 * i) * CB;
     if (BITS == 2) {
-      const uint32_t* vw = reinterpret_cast<const uint32_t*>(vc);
-      const uint32_t w0 = vw[ta * 8 + g], w1 = vw[(ta + 8) * 8 + g];
-      const uint32_t w2 = vw[(ta + 4) * 8 + g], w3 = vw[(ta + 12) * 8 + g];
-      const uint32_t xl1 = __byte_perm(w0, w1, 0x5410), xh1 = __byte_perm(w0, w1, 0x7632);
-      const uint32_t xl2 = __byte_perm(w2, w3, 0x5410), xh2 = __byte_perm(w2, w3, 0x7632);
+      const uint4 vv = *reinterpret_cast<const uint4*>(vgrp + 64 * g + 16 * t4);
+      const uint32_t xl1 = vv.x, xl2 = vv.y, xh1 = vv.z, xh2 = vv.w;
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
         const uint32_t A[4] = {vcode2(xl1, mt), vcode2(xh1, mt), vcode2(xl2, mt), vcode2(xh2, mt)};
@@ -453,15 +453,10 @@ __device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, 
         if (NHS == 2) mma_f16(s.o[mt], A, pbl);
       }
     } else {
-      const uint2* vw = reinterpret_cast<const uint2*>(vc);
-      const uint2 u0 = vw[ta * 8 + g], u1 = vw[(ta + 8) * 8 + g];
-      const uint2 u2 = vw[(ta + 4) * 8 + g], u3 = vw[(ta + 12) * 8 + g];
 #pragma unroll
       for (int ws = 0; ws < 2; ++ws) {
-        const uint32_t a0 = ws ? u0.y : u0.x, a1 = ws ? u1.y : u1.x;
-        const uint32_t a2 = ws ? u2.y : u2.x, a3 = ws ? u3.y : u3.x;
-        const uint32_t xl1 = __byte_perm(a0, a1, 0x5410), xh1 = __byte_perm(a0, a1, 0x7632);
-        const uint32_t xl2 = __byte_perm(a2, a3, 0x5410), xh2 = __byte_perm(a2, a3, 0x7632);
+        const uint4 vv = *reinterpret_cast<const uint4*>(vgrp + 512 * ws + 64 * g + 16 * t4);
+        const uint32_t xl1 = vv.x, xl2 = vv.y, xh1 = vv.z, xh2 = vv.w;
 #pragma unroll
         for (int mi = 0; mi < 4; ++mi) {
           const uint32_t A[4] = {vcode4(xl1, mi), vcode4(xh1, mi), vcode4(xl2, mi), vcode4(xh2, mi)};

@@ -102,16 +102,35 @@ __device__ __forceinline__ uint32_t quantize_one(float v, float zf, float sf, fl
   return static_cast<uint32_t>(c);
 }
 
+// Value codes are stored in groups of 16 positions laid out for the decode's PV operand:
+// each 32-bit word pairs the 16-bit chunk c (codes of 16 / BITS consecutive dimensions) of
+// group positions t and t + 8 (t = 0 .. 7; position t in the low half), and the four words
+// one lane of the decode needs sit together, lane after lane, so that a warp reads a group
+// with one conflict-free 16-byte load per lane (two at 4 bits).  Word of (t, c):
+//   2 bits:  16 * (c >> 1) + 4 * (t & 3) + 2 * (c & 1) + (t >> 2)
+//   4 bits: 128 * ((c >> 1) & 1) + 16 * (c >> 2) + 4 * (t & 3) + 2 * (c & 1) + (t >> 2)
+// This returns the index of the 16-bit half holding chunk c of group position r (0 .. 15).
+template <int BITS>
+__host__ __device__ __forceinline__ int vgroup_half(int r, int c) {
+  const int t = r & 7;
+  const int lane_part = 4 * (t & 3) + 2 * (c & 1) + (t >> 2);
+  const int word = BITS == 2 ? 16 * (c >> 1) + lane_part : 128 * ((c >> 1) & 1) + 16 * (c >> 2) + lane_part;
+  return 2 * word + (r >> 3);
+}
+
 // The quantizer with one row split over P adjacent lanes (P = 2 or 4; lanes
 // P*k .. P*k+P-1 of a warp, all active together): lane `part` takes values
 // [part*128/P, (part+1)*128/P), keeps its own NSEL smallest / largest, the lists are merged
 // over log2(P) xor-shuffle rounds (every lane ends with the same order statistics, so
 // every lane computes the same s and z), and each lane quantizes and writes its own
 // slice of the packed codes (16*BITS/P bytes); part 0 writes (s, z).
+// vrow < 0: codes_out is the row's record (key layout); vrow >= 0: codes_out is the base of
+// the row's 16-position group and vrow its position there (value layout, vgroup_half).
 template <int BITS, int NSEL, int P>
 __device__ __forceinline__ void quantize_row_part(const __half* __restrict__ x, int part,
                                                   uint8_t* __restrict__ codes_out,
-                                                  uint32_t* __restrict__ params_out, const QuantSpec qs) {
+                                                  uint32_t* __restrict__ params_out, const QuantSpec qs,
+                                                  int vrow = -1) {
   static_assert(P == 2 || P == 4, "two or four lanes per row");
   constexpr int V = 128 / P;  // values of this lane
   constexpr int H = V / 2;    // half2 of this lane
@@ -218,6 +237,17 @@ __device__ __forceinline__ void quantize_row_part(const __half* __restrict__ x, 
         w[k / 4] |= (c0 | (c1 << 4)) << (8 * (k % 4));
       }
     }
+  }
+  if (vrow >= 0) {
+    uint16_t* grp = reinterpret_cast<uint16_t*>(codes_out);
+#pragma unroll
+    for (int k = 0; k < NW; ++k) {
+      const int c = 2 * (part * NW + k);
+      grp[vgroup_half<BITS>(vrow, c)] = (uint16_t)(w[k] & 0xFFFFu);
+      grp[vgroup_half<BITS>(vrow, c + 1)] = (uint16_t)(w[k] >> 16);
+    }
+    if (part == 0) *params_out = h2_as_u32(__halves2half2(s_h, z_h));
+    return;
   }
   uint8_t* dst = codes_out + part * (NW * 4);
   if (NW % 4 == 0) {

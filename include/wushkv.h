@@ -122,9 +122,15 @@ typedef struct wushkv_layout {
 } wushkv_layout;
 
 /* Device pointers of one layer's cache.
- *  codes: code j (0..127) of position p is in byte (j*bits)/8 at bit offset (j*bits)%8 of
- *         the code_bytes-long record of p (little-endian within the byte); records are
- *         indexed by absolute position p; only S_sink <= p < S_quant are meaningful.
+ *  codes: the packed record of position p (code_bytes bytes) holds code j (0..127) in byte
+ *         (j*bits)/8 at bit offset (j*bits)%8 (little-endian within the byte); only
+ *         S_sink <= p < S_quant are meaningful.
+ *         k_codes: record p at byte offset p * code_bytes of the unit's array.
+ *         v_codes: in groups of 16 positions (group p / 16 at byte offset (p & ~15) *
+ *         code_bytes), laid out for the decode's PV operand: the 16-bit chunk c of record
+ *         p (bytes 2c, 2c+1; c < 8*bits) is 16-bit half 2*w + (r >> 3) of the group,
+ *         r = p % 16, t = r & 7, w = 16*(c>>1) + 4*(t&3) + 2*(c&1) + (t>>2) at 2 bits,
+ *         w = 128*((c>>1)&1) + 16*(c>>2) + 4*(t&3) + 2*(c&1) + (t>>2) at 4 bits.
  *  params: (s, z) of position p; the token's values dequantize to z + s * code.
  *  sink:  k' / v of positions p < s_sink at index p.
  *  ring:  k' / v of fp16 positions p >= max(S_quant, s_sink) at slot p % ring_slots.

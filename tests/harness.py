@@ -18,6 +18,47 @@ ATOL = 2e-3
 RTOL = 1e-3
 
 
+def _vgroup_index(bits):
+    """[16, 8*bits]: the 16-bit half of a 16-position value group that holds chunk c (bytes
+    2c, 2c+1 of the row's packed record) of group position r (the value layout of wushkv.h)."""
+    nc = 8 * bits
+    idx = np.empty((16, nc), np.int64)
+    for r in range(16):
+        t = r & 7
+        for c in range(nc):
+            lp = 4 * (t & 3) + 2 * (c & 1) + (t >> 2)
+            w = 16 * (c >> 1) + lp if bits == 2 else 128 * ((c >> 1) & 1) + 16 * (c >> 2) + lp
+            idx[r, c] = 2 * w + (r >> 3)
+    return idx
+
+
+def v_rows_from_groups(buf: np.ndarray, bits: int) -> np.ndarray:
+    """Value codes as stored (uint8 [..., positions, 16*bits], positions a multiple of 16) ->
+    one packed record per position, the key layout."""
+    buf = np.ascontiguousarray(buf)
+    shp = buf.shape
+    halves = buf.reshape(shp[:-2] + (shp[-2] // 16, 16 * shp[-1])).view(np.uint16)
+    rows = halves[..., _vgroup_index(bits)]
+    return np.ascontiguousarray(rows).reshape(shp[:-2] + (shp[-2], shp[-1] // 2)).view(np.uint8)
+
+
+def v_groups_from_rows(rows: np.ndarray, bits: int) -> np.ndarray:
+    """Inverse of v_rows_from_groups."""
+    rows = np.ascontiguousarray(rows)
+    shp = rows.shape
+    r16 = rows.view(np.uint16).reshape(shp[:-2] + (shp[-2] // 16, 16, shp[-1] // 2))
+    out = np.zeros(shp[:-2] + (shp[-2] // 16, 8 * shp[-1]), np.uint16)
+    out[..., _vgroup_index(bits)] = r16
+    return out.view(np.uint8).reshape(shp)
+
+
+def stored_codes(gc, kind, b=None, h=None) -> np.ndarray:
+    """One packed record per position of the GPU cache's codes (uint8 [..., cap_alloc, CB])."""
+    t = gc.codes_view(kind) if b is None else gc.codes_view(kind)[b, h]
+    a = t.cpu().numpy()
+    return v_rows_from_groups(a, gc.cfg.bits) if kind == "v" else a
+
+
 def oracle_cache_for(cfg, store_dtype=np.float16) -> ocache.Cache:
     return ocache.Cache(cfg.batch, cfg.n_kv_heads, 128, cfg.bits, cfg.p_lo, cfg.p_hi, cfg.s_sink, cfg.s_keep,
                         cfg.s_flush, capacity=cfg.capacity, chunk_max=cfg.chunk_max, store_dtype=store_dtype)
@@ -33,6 +74,8 @@ def upload(oc: ocache.Cache, gc) -> None:
         codes = getattr(oc, f"{kind}_codes")[:, :, :cap]
         packed = np.zeros((B, H, L.cap_alloc, L.code_bytes), dtype=np.uint8)
         packed[:, :, :cap] = oq.pack(codes, cfg.bits)
+        if kind == "v":
+            packed = v_groups_from_rows(packed, cfg.bits)
         gc.codes_view(kind).copy_(torch.from_numpy(packed))
         s = getattr(oc, f"{kind}_s")
         z = getattr(oc, f"{kind}_z")
@@ -64,7 +107,7 @@ def download(gc):
     S, Sq = (t.cpu().numpy() for t in gc.lengths())
     out = {"S": S, "Sq": Sq, "status": gc.status()}
     for kind in ("k", "v"):
-        out[f"{kind}_codes"] = oq.unpack(gc.codes_view(kind).cpu().numpy(), gc.cfg.bits)
+        out[f"{kind}_codes"] = oq.unpack(stored_codes(gc, kind), gc.cfg.bits)
         par = gc.params_view(kind).cpu().numpy()
         out[f"{kind}_s"] = par[..., 0]
         out[f"{kind}_z"] = par[..., 1]

@@ -39,7 +39,7 @@ def _unit_cache_from_gpu(gc, b, h, T):
                       capacity=L.cap_alloc, chunk_max=cfg.chunk_max)
     oc.S[0], oc.S_quant[0] = S, Sq
     for kind in ("k", "v"):
-        codes = oq.unpack(gc.codes_view(kind)[b, h].cpu().numpy(), cfg.bits)
+        codes = oq.unpack(H.stored_codes(gc, kind, b, h), cfg.bits)
         par = gc.params_view(kind)[b, h].cpu().numpy()
         getattr(oc, f"{kind}_codes")[0, 0] = codes
         getattr(oc, f"{kind}_s")[0, 0] = par[:, 0]
