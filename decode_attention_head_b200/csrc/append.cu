@@ -70,10 +70,10 @@ __device__ void quantize_ring_range(const AppendArgs& a, int unit, int p_begin, 
     const __half* row = ring + ((size_t)unit * a.R + (p % a.R)) * kHeadDim;
     const size_t rec = (size_t)unit * a.cap_alloc + p;
     uint32_t* params = (kind ? a.v_params : a.k_params) + rec;
-    if (kind)  // value codes: the position's 16-position group (cap_alloc is a multiple of 16)
-      quantize_row_part<BITS, NSEL, P>(row, tid % P, a.v_codes + (rec & ~(size_t)15) * CB, params, qs, p & 15);
-    else
-      quantize_row_part<BITS, NSEL, P>(row, tid % P, a.k_codes + rec * CB, params, qs);
+    // value codes go to the position's 16-position group (cap_alloc is a multiple of 16); one
+    // call site, so that the quantizer is inlined once
+    uint8_t* codes = kind ? a.v_codes + (rec & ~(size_t)15) * CB : a.k_codes + rec * CB;
+    quantize_row_part<BITS, NSEL, P>(row, tid % P, codes, params, qs, kind ? (p & 15) : -1);
   }
 }
 
@@ -271,7 +271,12 @@ __global__ void __launch_bounds__(128) flush_ring_kernel(const AppendArgs a) {
 constexpr int kBulkTile = 64;
 constexpr int kBulkSlab = 256;
 constexpr int kPad = 136;  // halves per padded shared row (272 bytes: conflict-free ldmatrix)
-constexpr size_t kBulkSmem = (size_t)(kHeadDim + 2 * kBulkTile) * kPad * sizeof(__half);
+// value codes of a tile are staged by 16-position group (a 64-token tile spans at most 5);
+// sized per code width so that three CTAs still fit an SM
+template <int BITS>
+constexpr size_t bulk_smem() {
+  return (size_t)(kHeadDim + 2 * kBulkTile) * kPad * sizeof(__half) + 5 * 16 * 16 * BITS;
+}
 
 constexpr int kBulkThreads = 256;
 
@@ -321,6 +326,7 @@ __global__ void __launch_bounds__(kBulkThreads, 3) append_bulk_kernel(const Appe
   __half* Ts = reinterpret_cast<__half*>(smem_raw);
   __half* ks = Ts + kHeadDim * kPad;
   __half* vs = ks + kBulkTile * kPad;
+  uint8_t* vstg = reinterpret_cast<uint8_t*>(vs + kBulkTile * kPad);  // value groups of the tile
 
   const int unit = blockIdx.y;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
@@ -433,15 +439,47 @@ __global__ void __launch_bounds__(kBulkThreads, 3) append_bulk_kernel(const Appe
             reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
         } else if (p < sq_new) {
           const size_t rec = (size_t)unit * a.cap_alloc + p;
-          if (kind)  // value codes: the position's 16-position group
-            quantize_row_part<BITS, NSEL, 2>(src, part, a.v_codes + (rec & ~(size_t)15) * CB, a.v_params + rec, qs,
-                                             p & 15);
-          else
-            quantize_row_part<BITS, NSEL, 2>(src, part, a.k_codes + rec * CB, a.k_params + rec, qs);
+          // value codes into the tile's staged copy of the position's group; one call site, so
+          // that the quantizer is inlined once
+          uint8_t* codes = kind ? vstg + (size_t)((p >> 4) - ((S + tile0) >> 4)) * 16 * CB : a.k_codes + rec * CB;
+          quantize_row_part<BITS, NSEL, 2>(src, part, codes, (kind ? a.v_params : a.k_params) + rec, qs,
+                                           kind ? (p & 15) : -1);
         } else {
           __half* dst = (kind ? a.v_ring : a.k_ring) + ((size_t)unit * a.R + p % a.R) * kHeadDim;
           for (int i = 8 * part; i < 8 * part + 8; ++i)
             reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
+        }
+      }
+    }
+    __syncthreads();
+
+    // the staged value groups out, 16 bytes at a time (the four positions t4, t4 + 8,
+    // t4 + 4, t4 + 12 of one decode lane's unit); halves of positions this tile does not
+    // quantize (a group shared with another append or with the windows) are left alone
+    {
+      const int p_first = S + tile0, p_end = S + min(tile0 + kBulkTile, a.n_new);
+      const int q_lo = max(p_first, a.s_sink), q_hi = min(p_end, sq_new);
+      if (q_lo < q_hi) {
+        const int g0 = p_first >> 4, ga = q_lo >> 4, gb = (q_hi - 1) >> 4;
+        for (int u = tid; u < (gb - ga + 1) * CB; u += kBulkThreads) {  // CB 16-byte units per group
+          const int gi = ga + u / CB, ul = u % CB;
+          const int pb = 16 * gi, t4 = ul & 3;
+          // halves 0..7 of the unit belong to positions pb + t4 + {0, 8, 4, 12, 0, 8, 4, 12}
+          const unsigned own = (pb + t4 >= q_lo && pb + t4 < q_hi ? 0x11u : 0u) |
+                               (pb + t4 + 8 >= q_lo && pb + t4 + 8 < q_hi ? 0x22u : 0u) |
+                               (pb + t4 + 4 >= q_lo && pb + t4 + 4 < q_hi ? 0x44u : 0u) |
+                               (pb + t4 + 12 >= q_lo && pb + t4 + 12 < q_hi ? 0x88u : 0u);
+          const uint4* srcu = reinterpret_cast<const uint4*>(vstg + (size_t)(gi - g0) * 16 * CB) + ul;
+          uint8_t* dstg = a.v_codes + ((size_t)unit * a.cap_alloc + pb) * CB;
+          if (own == 0xFFu) {
+            reinterpret_cast<uint4*>(dstg)[ul] = *srcu;
+          } else {
+            const uint16_t* sh = reinterpret_cast<const uint16_t*>(srcu);
+            uint16_t* dh = reinterpret_cast<uint16_t*>(dstg) + 8 * ul;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              if (own & (1u << k)) dh[k] = sh[k];
+          }
         }
       }
     }
@@ -478,13 +516,13 @@ cudaError_t launch_append_t(const Derived& d, bool small, const AppendArgs& a, c
   if (e != cudaSuccess) return e;
   dim3 grid((a.n_new + kBulkSlab - 1) / kBulkSlab, d.units);
   if (a.prep.enabled) {
-    e = ensure_smem_attr<append_bulk_kernel<BITS, NSEL, true>>((int)kBulkSmem);
+    e = ensure_smem_attr<append_bulk_kernel<BITS, NSEL, true>>((int)bulk_smem<BITS>());
     if (e != cudaSuccess) return e;
-    append_bulk_kernel<BITS, NSEL, true><<<grid, kBulkThreads, kBulkSmem, st>>>(a);
+    append_bulk_kernel<BITS, NSEL, true><<<grid, kBulkThreads, bulk_smem<BITS>(), st>>>(a);
   } else {
-    e = ensure_smem_attr<append_bulk_kernel<BITS, NSEL, false>>((int)kBulkSmem);
+    e = ensure_smem_attr<append_bulk_kernel<BITS, NSEL, false>>((int)bulk_smem<BITS>());
     if (e != cudaSuccess) return e;
-    append_bulk_kernel<BITS, NSEL, false><<<grid, kBulkThreads, kBulkSmem, st>>>(a);
+    append_bulk_kernel<BITS, NSEL, false><<<grid, kBulkThreads, bulk_smem<BITS>(), st>>>(a);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
