@@ -444,7 +444,9 @@ def run_gpu(args, rank, world, local_rank):
     # ---- end to end through the public API: pinned host inputs in, result out, every step.
     # Per layer step: one host->device copy of that step's k, v and q (packed in one pinned
     # buffer), wushkv_step on views of the device copy, one device->host copy of the output.
-    # One CUDA graph per model step holds the 32 layers' copies and steps in layer order.
+    # One CUDA graph per model step holds the 32 layers' copies and steps in layer order; the
+    # copies run on their own streams (two device input buffers), so that a layer's inputs go
+    # in while the layer before it computes and its output comes back while the next one does.
     e2e = None
     if e2e_steps:
         nk, nq = k_pool[0].numel(), q_pool[0].numel()
@@ -452,20 +454,39 @@ def run_gpu(args, rank, world, local_rank):
                    .pin_memory() for c in range(L)]
         host_out = [torch.empty(wl.batch, wl.n_q_heads, wl.head_dim, dtype=torch.float32).pin_memory()
                     for _ in range(L)]
-        dev_in = torch.empty(2 * nk + nq, dtype=torch.float16, device=dev)
-        dk = dev_in[:nk].view_as(k_pool[0])
-        dv = dev_in[nk:2 * nk].view_as(v_pool[0])
-        dq = dev_in[2 * nk:].view_as(q_pool[0])
+        dev_in = [torch.empty(2 * nk + nq, dtype=torch.float16, device=dev) for _ in range(2)]
+        views = [(d[:nk].view_as(k_pool[0]), d[nk:2 * nk].view_as(v_pool[0]), d[2 * nk:].view_as(q_pool[0]))
+                 for d in dev_in]
+        h2d_stream, d2h_stream = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
-        def e2e_layer(c):
-            dev_in.copy_(host_in[c], non_blocking=True)
+        def e2e_layer(c):  # one layer step, all on the compute stream
+            dk, dv, dq = views[0]
+            dev_in[0].copy_(host_in[c], non_blocking=True)
             caches[c].step(dk, dv, tks[c], dq, tinvs[c], scale, out=outs[c], stream=stream)
             host_out[c].copy_(outs[c], non_blocking=True)
 
+        ev_in = [torch.cuda.Event() for _ in range(L)]
+        ev_done = [torch.cuda.Event() for _ in range(L)]
         g_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_e2e, stream=stream):
+            h2d_stream.wait_stream(stream)
+            d2h_stream.wait_stream(stream)
             for c in range(L):
-                e2e_layer(c)
+                buf = c % 2
+                with torch.cuda.stream(h2d_stream):
+                    if c >= 2:  # the buffer's previous user has run
+                        h2d_stream.wait_event(ev_done[c - 2])
+                    dev_in[buf].copy_(host_in[c], non_blocking=True)
+                    ev_in[c].record(h2d_stream)
+                stream.wait_event(ev_in[c])
+                dk, dv, dq = views[buf]
+                caches[c].step(dk, dv, tks[c], dq, tinvs[c], scale, out=outs[c], stream=stream)
+                ev_done[c].record(stream)
+                with torch.cuda.stream(d2h_stream):
+                    d2h_stream.wait_event(ev_done[c])
+                    host_out[c].copy_(outs[c], non_blocking=True)
+            stream.wait_stream(h2d_stream)
+            stream.wait_stream(d2h_stream)
         first_e = first2 + K2
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
@@ -490,10 +511,11 @@ def run_gpu(args, rank, world, local_rank):
             e2e_bytes += mirrors[c].append_bytes(1) + mirrors[c].decode_bytes()
         (t_e2e,) = max_over_ranks([e0.elapsed_time(e1) / 1e3], dev, world)
         e2e = {"value": round(job_throughput(world, e2e_bytes, t_e2e), 2), "unit": "GB/s",
-               "h2d_bytes_per_step": int(dev_in.numel() * 2),
+               "h2d_bytes_per_step": int(dev_in[0].numel() * 2),
                "d2h_bytes_per_step": int(host_out[0].numel() * 4),
-               "launch": "one CUDA graph per model step: per layer one H2D copy (packed k/v/q), wushkv_step, "
-                         "one D2H copy of the output"}
+               "launch": "one CUDA graph per model step: per layer one H2D copy (packed k/v/q, two device "
+                         "buffers, on its own stream, overlapping the layer before), wushkv_step, one D2H copy "
+                         "of the output (on its own stream, overlapping the layer after)"}
         del g_e2e
 
     peak, peak_kind = measured_peaks()
