@@ -19,11 +19,13 @@ Modules:
   rope       -- per-head RMSNorm and rotate-half RoPE of the path's raw inputs
   transform  -- the normalised Walsh-Hadamard key transform
   quest      -- the RMS-scaled symmetric (QuEST-style) alternative quantizer
+  calibration -- per-KV-head Gram matrices of cached vectors (calibration statistics)
 
 Parity status: every function is pinned by a ``-m "not gpu"`` test in
 ``tests/test_oracle_pins.py``, ``tests/test_oracle_rope.py``,
-``tests/test_oracle_transform.py`` and ``tests/test_oracle_quest.py``; none is "parity
+``tests/test_oracle_transform.py``, ``tests/test_oracle_quest.py`` and
+``tests/test_oracle_calibration.py``; none is "parity
 unpinned" (the QuEST-style quantizer's reading of the lost Eq. 5 is pinned by the Gaussian
 optimum and its grid, not by the pages' equation).
 """
-from . import quantizer, cache, attention, footprint, rope, transform, quest  # noqa: F401
+from . import quantizer, cache, attention, footprint, rope, transform, quest, calibration  # noqa: F401
