@@ -48,6 +48,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--gram-only", action="store_true",
+                   help="only the calibration Gram-matrix measurement (one JSON line)")
     p.add_argument("--prefill-only", action="store_true",
                    help="only the prefill workload's bulk append + decode measurement (one JSON line)")
     return p.parse_args()
@@ -571,6 +573,7 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         result["prefill_append"] = measure_prefill(bnd, synth, dev)
         result["chunk_prefill"] = measure_chunk(bnd, synth, dev)
+        result["calibration_gram"] = measure_gram(bnd, synth, dev)
     return result, wl
 
 
@@ -704,6 +707,41 @@ def measure_chunk(bnd, synth, dev, n=8, reps=20):
             "launch": "eager: 1 append launch + 2 launches per pass (prologue, main)", "reps": reps}
 
 
+def measure_gram(bnd, synth, dev, n_seq=4, seq_len=32768, reps=10):
+    """Calibration statistics: the per-KV-head key Gram matrices of n_seq calibration
+    sequences of seq_len tokens (the pages calibrate on 32,768-token sequences), Qwen3-8B
+    shaped: 8 KV heads, keys after RMSNorm and RoPE.  One wushkv_gram_accumulate launch per
+    repetition over all n_seq * seq_len tokens (268 MB of fp16 keys, more than L2), each
+    timed with CUDA events.  Algorithmic bytes: the keys once, plus the fp64 Gram matrices
+    read and written once."""
+    import torch
+    wl = synth.scaled(synth.WORKLOADS["qwen3-8b-layer"], batch=n_seq)
+    x = synth.bulk_tokens(wl, 0, 0, seq_len, device=dev, which="k")
+    H = wl.n_kv_heads
+    gram = torch.zeros(H, 128, 128, dtype=torch.float64, device=dev)
+    for _ in range(3):
+        bnd.gram_accumulate(x, gram)
+    ms = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        bnd.gram_accumulate(x, gram)
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    t = sum(ms) / len(ms) / 1e3
+    tokens = n_seq * seq_len
+    nbytes = tokens * H * 128 * 2 + H * 128 * 128 * 8 * 2
+    peak, peak_kind = measured_peaks()
+    mma_flops = 2 * tokens * H * 10 * 32 * 32  # the 10 blocks of 32 x 32 on and above the diagonal
+    return {"workload": "qwen3-8b calibration keys", "sequences": n_seq, "tokens_per_sequence": seq_len,
+            "kv_heads": H, "us": round(t * 1e6, 2), "gbs": round(nbytes / t / 1e9, 2),
+            "frac_hbm": round(nbytes / t / 1e9 / peak, 4), "peak_kind": peak_kind,
+            "mma_tflops": round(mma_flops / t / 1e12, 2), "tokens_per_s": round(tokens / t, 1),
+            "launch": "eager: 1 launch per call", "reps": reps}
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -735,6 +773,15 @@ def main():
 
     import torch
     import torch.distributed as dist
+    if args.gram_only:
+        from decode_attention_head_b200 import binding as bnd
+        from decode_attention_head_b200 import build as _build
+        from decode_attention_head_b200 import synth
+        _build.build()
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        print(json.dumps(measure_gram(bnd, synth, dev)))
+        return 0
     if args.prefill_only:
         from decode_attention_head_b200 import binding as bnd
         from decode_attention_head_b200 import build as _build
@@ -744,6 +791,7 @@ def main():
         torch.cuda.set_device(dev)
         print(json.dumps(measure_prefill(bnd, synth, dev)))
         print(json.dumps(measure_chunk(bnd, synth, dev)))
+        print(json.dumps(measure_gram(bnd, synth, dev)))
         return 0
     if world > 1:
         import datetime

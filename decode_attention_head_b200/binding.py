@@ -20,7 +20,8 @@ STATUS_OVERFLOW, STATUS_EMPTY, STATUS_TIMEOUT, STATUS_BADSTATE, STATUS_CHUNK_QUA
 _ERR = {EINVAL: "invalid argument", EUNSUPPORTED: "unsupported configuration", ECUDA: "CUDA launch failed",
         ESINGULAR: "singular key transform", ESCRATCH: "needs more than the static scratch array holds"}
 SYMBOLS = ("wushkv_pack_layout", "wushkv_compensation", "wushkv_hadamard", "wushkv_append", "wushkv_decode_attn",
-           "wushkv_chunk_attn", "wushkv_step", "wushkv_step_prep", "wushkv_decode_attn_static")
+           "wushkv_chunk_attn", "wushkv_step", "wushkv_step_prep", "wushkv_decode_attn_static",
+           "wushkv_gram_accumulate")
 
 
 class Prep(ctypes.Structure):
@@ -83,6 +84,8 @@ def _load() -> ctypes.CDLL:
     lib.wushkv_decode_attn_static.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
                                               ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
                                               ctypes.c_void_p]
+    lib.wushkv_gram_accumulate.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p,
+                                           ctypes.c_void_p]
     for name in SYMBOLS:
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -122,6 +125,21 @@ def hadamard_compensation(n_kv_heads: int) -> torch.Tensor:
     out = torch.empty(n_kv_heads, 128, 128, dtype=torch.float32)
     _check(lib.wushkv_hadamard(n_kv_heads, out.data_ptr()), "wushkv_hadamard")
     return out
+
+
+def gram_accumulate(x: torch.Tensor, gram: torch.Tensor, stream=None) -> torch.Tensor:
+    """gram[h] += sum_t x[t, h] x[t, h]^T on the device (wushkv_gram_accumulate).
+    x: fp16 [..., n_heads, 128], contiguous (leading dimensions are tokens);
+    gram: fp64 [n_heads, 128, 128], contiguous.  Returns gram."""
+    if x.dtype != torch.float16 or gram.dtype != torch.float64 or not x.is_contiguous() \
+            or not gram.is_contiguous() or x.dim() < 2 or x.shape[-1] != 128 \
+            or tuple(gram.shape) != (x.shape[-2], 128, 128):
+        raise WushKVError("gram_accumulate: x must be contiguous fp16 [..., H, 128], gram fp64 [H, 128, 128]")
+    n_heads = x.shape[-2]
+    n_tokens = x.numel() // (n_heads * 128) if n_heads else 0
+    _check(lib.wushkv_gram_accumulate(x.data_ptr(), n_tokens, n_heads, gram.data_ptr(), _stream_ptr(stream)),
+           "wushkv_gram_accumulate")
+    return gram
 
 
 def _ptr(t: Optional[torch.Tensor]):

@@ -7,7 +7,7 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libwushkv.so")
-SOURCES = ["abi.cu", "append.cu", "decode.cu", "decode_static.cu"]
+SOURCES = ["abi.cu", "append.cu", "decode.cu", "decode_static.cu", "gram.cu"]
 NVCC_FLAGS = ["-std=c++17", "-O3", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
               "-Xcompiler", "-fPIC", "-shared"]
 

@@ -306,6 +306,18 @@ extern "C" int wushkv_hadamard(int32_t n_kv_heads, float* t_k_inv) {
   return WUSHKV_OK;
 }
 
+extern "C" int wushkv_gram_accumulate(const void* x, int64_t n_tokens, int32_t n_heads, double* gram,
+                                      void* stream) {
+  if (!aligned16(gram) || n_tokens < 0 || n_heads < 1 || n_heads > 65535) return WUSHKV_EINVAL;
+  // keeps the kernel's element offsets (t * n_heads + h) * 128 and its grid size in range
+  if (n_tokens > (INT64_C(1) << 40) / n_heads) return WUSHKV_EINVAL;
+  if (n_tokens == 0) return WUSHKV_OK;
+  if (!aligned16(x)) return WUSHKV_EINVAL;
+  const cudaError_t e = launch_gram(static_cast<const uint16_t*>(x), n_tokens, n_heads, gram,
+                                    static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA;
+}
+
 extern "C" int wushkv_append(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new,
                              const void* v_new, int32_t n_new, const void* t_k, void* stream) {
   Derived d;

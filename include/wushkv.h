@@ -166,6 +166,25 @@ int wushkv_compensation(const uint16_t* t_k, int32_t n_kv_heads, float* t_k_inv)
  * "cheaper structured transforms" direction.  Returns WUSHKV_OK or WUSHKV_EINVAL. */
 int wushkv_hadamard(int32_t n_kv_heads, float* t_k_inv);
 
+/* Calibration statistics (offline, before T_K is built): accumulate the per-head Gram
+ * matrices of a batch of cached vectors ("WUSH-KV: KV Cache Quantization with
+ * Data-Adaptive Transforms": §3, the transform is built from the Gram matrix M of the
+ * quantized tensor; Appendix B.1, M = X X^T with one quantization group, here one token,
+ * per column; §5.2 Setup, a calibration pass accumulates key Gram matrices after RMS
+ * normalisation and RoPE, and value Gram matrices, per KV head).
+ * x:     device fp16 [n_tokens][n_heads][128], 16-byte aligned: keys after head-norm and
+ *        RoPE (before T_K), or values.  [B][n][H_kv][128] is the same array with
+ *        n_tokens = B * n.
+ * gram:  device fp64 [n_heads][128][128] row-major, 16-byte aligned, accumulated in place:
+ *        gram[h] += sum_t x[t][h] x[t][h]^T.  Zero it before the first batch.
+ * Precision: a block of at most 4096 tokens of one head is summed on the tensor cores
+ * (exact fp16 products, fp32 sums), then added into gram with fp64 atomics.  The order of
+ * those fp64 additions is not fixed, so the last bits can differ between calls.
+ * n_tokens == 0 queues nothing (x may then be null).  The two buffers must not overlap.
+ * Returns WUSHKV_OK, WUSHKV_EINVAL (null or misaligned pointer, n_tokens < 0, n_heads
+ * outside [1, 65535], n_tokens * n_heads > 2^40) or WUSHKV_ECUDA. */
+int wushkv_gram_accumulate(const void* x, int64_t n_tokens, int32_t n_heads, double* gram, void* stream);
+
 /* Append n_new >= 0 tokens to every sequence (§4.1, §4.2, §4.4 "Full-Precision Cache
  * Window", §5.3 quantizer).
  * k_new, v_new: device fp16 [B][n_new][H_kv][128]; keys after head-norm and RoPE,

@@ -133,3 +133,25 @@ def test_rms_quantizer_config_checks(bnd):
     bad = bnd.make_config(1, 1, 4, 2, 256, 4, 32, 16, 1)
     bad.quantizer = 7
     assert bnd.lib.wushkv_pack_layout(ctypes.byref(bad), ctypes.byref(bnd.Layout())) == bnd.EINVAL
+
+
+def test_gram_accumulate_argument_checks(bnd):
+    """wushkv_gram_accumulate validates on the host before any CUDA call; zero tokens
+    queue nothing (the aligned fake pointers are never dereferenced)."""
+    f = bnd.lib.wushkv_gram_accumulate
+    fake = 1 << 20
+    assert f(None, 10, 2, fake, None) == bnd.EINVAL
+    assert f(fake, 10, 2, None, None) == bnd.EINVAL
+    assert f(fake + 8, 10, 2, fake, None) == bnd.EINVAL
+    assert f(fake, 10, 2, fake + 8, None) == bnd.EINVAL
+    assert f(fake, -1, 2, fake, None) == bnd.EINVAL
+    assert f(fake, 10, 0, fake, None) == bnd.EINVAL
+    assert f(fake, 10, 65536, fake, None) == bnd.EINVAL
+    assert f(fake, (1 << 40) // 8 + 1, 8, fake, None) == bnd.EINVAL
+    assert f(fake, 0, 8, fake, None) == bnd.OK
+    assert f(None, 0, 8, fake, None) == bnd.OK
+    assert f(None, 0, 8, None, None) == bnd.EINVAL
+    with pytest.raises(bnd.WushKVError):
+        bnd.gram_accumulate(torch.zeros(4, 2, 128, dtype=torch.float32), torch.zeros(2, 128, 128, dtype=torch.float64))
+    with pytest.raises(bnd.WushKVError):
+        bnd.gram_accumulate(torch.zeros(4, 2, 128, dtype=torch.float16), torch.zeros(3, 128, 128, dtype=torch.float64))
