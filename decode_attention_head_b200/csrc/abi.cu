@@ -7,6 +7,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include "internal.h"
+#include "gram.h"
 #include "qfrag.cuh"
 
 namespace wushkv {

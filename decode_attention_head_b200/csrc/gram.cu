@@ -23,6 +23,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include "gram.h"
 #include "internal.h"
 #include "ptx.cuh"
 

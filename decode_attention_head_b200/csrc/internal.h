@@ -17,7 +17,6 @@ constexpr int kB200SMs = 148;         // split policy sizes the decode grid for 
 constexpr int decode_ctas_per_sm(int group) { return group == 8 ? 3 : 4; }
 constexpr int kMaxSplits = 255;       // quantized work items per (sequence, KV head)
 constexpr int kMergeGroup = 16;       // work items merged together at the first merge level
-constexpr int kGramTokens = 4096;     // tokens of one head per Gram-matrix CTA (one fp32 partial sum)
 
 struct Derived {
   int units;        // B * H_kv
@@ -140,7 +139,5 @@ cudaError_t launch_decode(const Derived& d, int bits, const DecodeArgs& a, cudaS
 // kernel's programmatic dependent (it waits for it before reading anything).
 cudaError_t launch_append_fused(const Derived& d, int bits, const AppendArgs& a, cudaStream_t st);
 cudaError_t launch_decode_main(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st);
-// wushkv_gram_accumulate: arguments already validated (n_tokens >= 1, 1 <= n_heads <= 65535).
-cudaError_t launch_gram(const uint16_t* x, int64_t n_tokens, int n_heads, double* gram, cudaStream_t st);
 
 }  // namespace wushkv
