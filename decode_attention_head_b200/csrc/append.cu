@@ -10,6 +10,8 @@
 // Small appends (n_new <= chunk_max), one CTA per (sequence, KV head), one launch:
 //   flush under S (the step that closes the previous chunk, whose attention has been
 //   computed by now), then transform + store the new tokens fp16, then advance S.
+//   In a fused decode step (wushkv_step) a second CTA per unit prepares the decode query
+//   in the same launch, and the state words are left to the decode kernel.
 // Bulk appends (n_new > chunk_max), three launches in stream order:
 //   flush_ring   quantize the ring entries the flush under S + n_new covers;
 //   append_bulk  T_K GEMM on tensor cores (mma.sync m16n8k16, fp32 accumulate) per
