@@ -135,11 +135,22 @@ def gram_accumulate(x: torch.Tensor, gram: torch.Tensor, stream=None) -> torch.T
             or not gram.is_contiguous() or x.dim() < 2 or x.shape[-1] != 128 \
             or tuple(gram.shape) != (x.shape[-2], 128, 128):
         raise WushKVError("gram_accumulate: x must be contiguous fp16 [..., H, 128], gram fp64 [H, 128, 128]")
+    _require_cuda(x, gram)
+    if x.device != gram.device:
+        raise WushKVError("gram_accumulate: x and gram must be on the same device")
     n_heads = x.shape[-2]
     n_tokens = x.numel() // (n_heads * 128) if n_heads else 0
     _check(lib.wushkv_gram_accumulate(x.data_ptr(), n_tokens, n_heads, gram.data_ptr(), _stream_ptr(stream)),
            "wushkv_gram_accumulate")
     return gram
+
+
+def _require_cuda(*tensors) -> None:
+    """The library reads and writes these through device pointers: a host tensor would hand
+    a kernel an address it cannot use, so it is refused here (None entries are skipped)."""
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise WushKVError("expected CUDA tensors: the library's kernels read them on the device")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -191,6 +202,7 @@ class KVCache:
 
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, t_k: torch.Tensor, stream=None) -> None:
         """k_new, v_new: fp16 [B, n_new, H_kv, 128] on the device; t_k fp16 [H_kv, 128, 128]."""
+        _require_cuda(k_new, v_new, t_k)
         n_new = k_new.shape[1]
         _check(lib.wushkv_append(ctypes.byref(self.cfg), ctypes.byref(self.bufs), k_new.data_ptr(),
                                  v_new.data_ptr(), n_new, _ptr(t_k), _stream_ptr(stream)), "wushkv_append")
@@ -198,6 +210,7 @@ class KVCache:
     def decode_attn(self, q: torch.Tensor, t_k_inv: torch.Tensor, softmax_scale: float,
                     out: Optional[torch.Tensor] = None, out_fp16: bool = False, stream=None) -> torch.Tensor:
         """q fp16 [B, H_q, 128]; t_k_inv fp32 [H_kv, 128, 128] (T_K^{-1}); returns out [B, H_q, 128]."""
+        _require_cuda(q, t_k_inv, out)
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float16 if out_fp16 else torch.float32, device=q.device)
         _check(lib.wushkv_decode_attn(ctypes.byref(self.cfg), ctypes.byref(self.bufs), q.data_ptr(),
@@ -210,6 +223,7 @@ class KVCache:
                    out: Optional[torch.Tensor] = None, out_fp16: bool = False, stream=None) -> torch.Tensor:
         """q fp16 [B, n, H_q, 128]: the n newest positions' queries (the chunk just appended,
         n <= chunk_max), each attending causally over the cache; returns out [B, n, H_q, 128]."""
+        _require_cuda(q, t_k_inv, out)
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float16 if out_fp16 else torch.float32, device=q.device)
         _check(lib.wushkv_chunk_attn(ctypes.byref(self.cfg), ctypes.byref(self.bufs), q.data_ptr(), q.shape[1],
@@ -222,6 +236,7 @@ class KVCache:
              t_k_inv: torch.Tensor, softmax_scale: float, out: Optional[torch.Tensor] = None,
              out_fp16: bool = False, stream=None) -> torch.Tensor:
         """append(k_new, v_new) then decode_attn(q) in one call (wushkv_step)."""
+        _require_cuda(k_new, v_new, t_k, q, t_k_inv, out)
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float16 if out_fp16 else torch.float32, device=q.device)
         _check(lib.wushkv_step(ctypes.byref(self.cfg), ctypes.byref(self.bufs), k_new.data_ptr(), v_new.data_ptr(),
@@ -238,6 +253,7 @@ class KVCache:
                   stream=None) -> torch.Tensor:
         """step() on raw projections: per-head RMSNorm (gains given) and RoPE inside the
         library's kernels (wushkv_step_prep).  Gains: fp16 [128] on the device."""
+        _require_cuda(k_raw, v_new, t_k, q_raw, t_k_inv, q_norm_gain, k_norm_gain, out)
         if out is None:
             out = torch.empty(q_raw.shape, dtype=torch.float16 if out_fp16 else torch.float32, device=q_raw.device)
         prep = Prep(float(rope_theta), q_norm_gain.data_ptr() if q_norm_gain is not None else None,
@@ -254,6 +270,7 @@ class KVCache:
                            out: torch.Tensor, stream=None) -> torch.Tensor:
         """decode_attn through wushkv_decode_attn_static: scratch in the library's own device
         array, `out` supplied by the caller (fp32 or fp16), nothing allocated."""
+        _require_cuda(q, t_k_inv, out)
         _check(lib.wushkv_decode_attn_static(ctypes.byref(self.cfg), ctypes.byref(self.bufs), q.data_ptr(),
                                              t_k_inv.data_ptr(), float(softmax_scale),
                                              1 if out.dtype == torch.float16 else 0, out.data_ptr(),

@@ -155,3 +155,14 @@ def test_gram_accumulate_argument_checks(bnd):
         bnd.gram_accumulate(torch.zeros(4, 2, 128, dtype=torch.float32), torch.zeros(2, 128, 128, dtype=torch.float64))
     with pytest.raises(bnd.WushKVError):
         bnd.gram_accumulate(torch.zeros(4, 2, 128, dtype=torch.float16), torch.zeros(3, 128, 128, dtype=torch.float64))
+    # well-formed but on the host: refused before the library is called
+    with pytest.raises(bnd.WushKVError, match="CUDA"):
+        bnd.gram_accumulate(torch.zeros(4, 2, 128, dtype=torch.float16), torch.zeros(2, 128, 128, dtype=torch.float64))
+
+
+def test_binding_refuses_host_tensors(bnd):
+    """The check every binding entry runs before handing tensors to the library: host
+    tensors are refused (a host pointer on the device would fault), None is allowed."""
+    bnd._require_cuda(None)
+    with pytest.raises(bnd.WushKVError, match="CUDA"):
+        bnd._require_cuda(None, torch.zeros(1))
