@@ -101,3 +101,22 @@ def test_bulk_append_bytes_follow_the_oracle_flush(S0, n):
     expect = n * 512 + from_ring * 512 + nq * 72 + kept * 512 + 128 * 128 * 2
     assert bench.bulk_append_bytes(wl, S, Sq, n) == expect
     assert int(oc.S[0]) == S + n
+
+
+@pytest.mark.parametrize("name,expect", [
+    ("llama3-8b-layer", 155.4e6), ("qwen3-8b-layer", 76.5e6), ("mha-32l", 74.8e9),
+    ("prefill-append-decode", 304.6e6)])
+def test_decode_bytes_follow_the_per_unit_costs(name, expect):
+    """The roofline's numerator at steady state (S_quant = S - S_keep): per quantized
+    token-head (128 * bits / 8 + 4) B for K and again for V, 512 B per fp16 window
+    token-head (K and V), 256 B in + 512 B out per query head, 64 KiB of fp32 T_K^{-1} per KV
+    head, summed over the workload's layers.  `expect` is that sum to four significant digits."""
+    wl = synth.WORKLOADS[name]
+    S = wl.context
+    got = bench.StateMirror(wl, S, S - wl.s_keep).decode_bytes() * wl.n_layers
+    units = wl.batch * wl.n_kv_heads
+    nq = S - wl.s_keep - wl.s_sink
+    closed = wl.n_layers * (units * (nq * 2 * (128 * wl.bits // 8 + 4) + (wl.s_sink + wl.s_keep) * 512)
+                            + wl.batch * wl.n_q_heads * (256 + 512) + wl.n_kv_heads * 128 * 128 * 4)
+    assert got == closed
+    assert abs(got - expect) <= 5e-4 * expect
