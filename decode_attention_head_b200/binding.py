@@ -39,6 +39,7 @@ class Config(ctypes.Structure):
 
 TRANSFORM_DENSE, TRANSFORM_HADAMARD = 0, 1
 QUANT_PERCENTILE, QUANT_RMS = 0, 1
+CODE_ORDER_CANONICAL, CODE_ORDER_VGROUP16 = 0, 1
 
 
 class Layout(ctypes.Structure):
@@ -46,7 +47,7 @@ class Layout(ctypes.Structure):
                 ("sink_bytes", ctypes.c_size_t), ("ring_bytes", ctypes.c_size_t),
                 ("state_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t),
                 ("cap_alloc", ctypes.c_int32), ("ring_slots", ctypes.c_int32), ("code_bytes", ctypes.c_int32),
-                ("n_splits", ctypes.c_int32), ("split_tokens", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("n_splits", ctypes.c_int32), ("split_tokens", ctypes.c_int32), ("code_order", ctypes.c_int32),
                 ("chunk_workspace_bytes", ctypes.c_size_t)]
 
 

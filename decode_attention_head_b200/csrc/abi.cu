@@ -153,6 +153,7 @@ extern "C" int wushkv_pack_layout(const wushkv_config* cfg, wushkv_layout* out) 
   out->n_splits = d.n_split;
   out->chunk_workspace_bytes = chunk_workspace(cfg);
   out->split_tokens = d.split_tokens;
+  out->code_order = WUSHKV_CODE_ORDER_VGROUP16;
   return WUSHKV_OK;
 }
 

@@ -101,6 +101,14 @@ typedef struct wushkv_config {
  * quantizer's (the decode is unchanged). */
 #define WUSHKV_QUANT_RMS 1
 
+/* Code orders of wushkv_layout.code_order.
+ *  WUSHKV_CODE_ORDER_CANONICAL (0): every position's record holds code j (0..127) in byte
+ *    (j*bits)/8 at bit offset (j*bits)%8, record p at byte offset p * code_bytes (K and V).
+ *  WUSHKV_CODE_ORDER_VGROUP16 (1): k_codes canonical; v_codes in the 16-position group
+ *    layout that wushkv_cache describes (the layout this library writes and reads). */
+#define WUSHKV_CODE_ORDER_CANONICAL 0
+#define WUSHKV_CODE_ORDER_VGROUP16 1
+
 /* Byte sizes of the caller-allocated buffers (wushkv_pack_layout). */
 typedef struct wushkv_layout {
   size_t codes_bytes;     /* each of k_codes, v_codes: uint8 [B][H_kv][cap_alloc][code_bytes] */
@@ -117,7 +125,7 @@ typedef struct wushkv_layout {
   int32_t split_tokens;   /* most positions one decode work item streams (at full capacity; the
                              kernel splits each sequence's current length evenly among the
                              n_splits items, in whole multiples of 128) */
-  int32_t reserved;
+  int32_t code_order;     /* how the packed codes are ordered (WUSHKV_CODE_ORDER_*) */
   size_t chunk_workspace_bytes; /* wushkv_chunk_attn scratch (no initialisation needed) */
 } wushkv_layout;
 

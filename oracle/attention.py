@@ -10,7 +10,9 @@ query-side compensation is applied after normalisation and RoPE; with
 k' = T_K k the compensated query is q' = T_K^{-T} q, so q' . k' = q . k),
 §4.5 (the value transform is folded into the weights, so the output stays in
 the value-transform basis) and §4.4 (attention reads the fp16 sink and recent
-windows and the dequantized middle region).
+windows and the dequantized middle region; a new chunk is first appended in
+full precision and is used to compute its own attention output, before the
+flush quantizes it).
 
 Query head j reads KV head floor(j / g), g = H_q / H_kv.  All arithmetic is
 float64; the inverse of T_K is LAPACK's (numpy.linalg.inv).
@@ -55,4 +57,29 @@ def decode(cache, q: np.ndarray, T_K: np.ndarray, softmax_scale: float) -> np.nd
             for j in range(h * g, (h + 1) * g):
                 qc = Tinv_T[h] @ q[b, j].astype(np.float64)
                 out[b, j], _, _ = softmax_attention(qc, K, V, softmax_scale)
+    return out
+
+
+def chunk_decode(cache, q: np.ndarray, T_K: np.ndarray, softmax_scale: float) -> np.ndarray:
+    """Attention of a just-appended chunk's own queries (§4.4): q fp16 [B, n, H_q, d] holds
+    the queries of the n newest positions S - n .. S - 1 of every sequence; query t of the
+    chunk sits at position S - n + t and, as in any causal decoder, attends to the cached
+    positions 0 .. S - n + t only.  Returns float64 [B, n, H_q, d].
+
+    The cache must hold the chunk already (it was appended before its attention runs).
+    """
+    B, n, Hq, d = q.shape
+    g = Hq // cache.H
+    Tinv_T = compensation(T_K)
+    out = np.zeros((B, n, Hq, d), dtype=np.float64)
+    for b in range(B):
+        S = int(cache.S[b])
+        for h in range(cache.H):
+            K = cache.keys_hat(b, h)
+            V = cache.values_hat(b, h)
+            for t in range(n):
+                last = S - n + t  # the query's own position: the newest one it may see
+                for j in range(h * g, (h + 1) * g):
+                    qc = Tinv_T[h] @ q[b, t, j].astype(np.float64)
+                    out[b, t, j], _, _ = softmax_attention(qc, K[:last + 1], V[:last + 1], softmax_scale)
     return out

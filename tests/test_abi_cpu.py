@@ -45,6 +45,8 @@ def test_layout_sizes(bnd):
     assert L.state_bytes >= (2 * 64 + 1) * 4
     assert L.split_tokens % 128 == 0 and L.n_splits * L.split_tokens >= L.cap_alloc
     assert L.workspace_bytes > 0
+    # keys canonical, values in the 16-position group layout the header documents
+    assert L.code_order == bnd.CODE_ORDER_VGROUP16 == 1
     cfg4 = bnd.make_config(64, 32, 32, 4, 8192, 4, 64, 16, 1, 0.5, 99.5)
     L4 = bnd.pack_layout(cfg4)
     assert L4.code_bytes == 64 and L4.codes_bytes == 64 * 32 * 8192 * 64

@@ -15,24 +15,6 @@ from tests import harness as H
 pytestmark = pytest.mark.gpu
 
 
-def _oracle_chunk(oc, q, T, scale):
-    """Causal attention of the n newest positions' queries q [B, n, H_q, d] over oc."""
-    B, n, Hq, d = q.shape
-    g = Hq // oc.H
-    tinv_t = oatt.compensation(T)
-    out = np.zeros((B, n, Hq, d))
-    for b in range(B):
-        S = int(oc.S[b])
-        for h in range(oc.H):
-            K, V = oc.keys_hat(b, h), oc.values_hat(b, h)
-            for t in range(n):
-                pos = S - n + t
-                for j in range(h * g, (h + 1) * g):
-                    qc = tinv_t[h] @ q[b, t, j].astype(np.float64)
-                    out[b, t, j], _, _ = oatt.softmax_attention(qc, K[:pos + 1], V[:pos + 1], scale)
-    return out
-
-
 @pytest.mark.parametrize("bits,Hkv,Hq,chunk", [(2, 2, 8, 8), (2, 2, 2, 16), (4, 1, 8, 4), (2, 2, 4, 3)])
 def test_chunk_attention_matches_oracle(bits, Hkv, Hq, chunk):
     B = 2
@@ -57,7 +39,7 @@ def test_chunk_attention_matches_oracle(bits, Hkv, Hq, chunk):
         out = gc.chunk_attn(H.to_dev(q), tinv, scale)
         torch.cuda.synchronize()
         assert gc.status() == 0
-        ref = _oracle_chunk(H.oracle_cache_from_gpu(gc), q, T, scale)
+        ref = oatt.chunk_decode(H.oracle_cache_from_gpu(gc), q, T, scale)
         H.assert_attention_close(out.cpu().numpy(), ref)
         if n == 1:
             dec = gc.decode_attn(H.to_dev(q[:, 0]), tinv, scale)

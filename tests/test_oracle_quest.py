@@ -62,3 +62,30 @@ def test_codes_are_nearest_levels(bits):
     best = dist.min(axis=-1)
     got = np.take_along_axis(dist, c[..., None].astype(np.int64), axis=-1)[..., 0]
     assert np.all(got <= best + 1e-6 * np.abs(s.astype(np.float64))[:, None])
+
+
+def _rms_golden():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "rms_sigma.txt")
+    rows = []
+    for line in open(path):
+        line = line.split("#")[0].split()
+        if line:
+            sig = [int(t, 16) for t in line[:5]]
+            x = np.array([int(t, 16) for t in line[5:]], dtype=np.uint16).view(np.float16)
+            rows.append((sig, x))
+    return rows
+
+
+def test_rms_fp32_summation_order_matches_golden_bits():
+    """sigma in the declared fixed order, bit for bit, against tests/golden/rms_sigma.txt
+    (written by a pure-Python binary32 routine, make_rms_golden.py).  On every stored vector
+    that order gives a different fp32 sigma from a plain left-to-right sum and from three
+    other groupings, so the pin fixes the order, not just the value to an ulp."""
+    rows = _rms_golden()
+    assert len(rows) >= 8
+    xs = np.stack([x for _, x in rows])
+    got = oqt.rms_fp32(xs).astype(np.float32).view(np.uint32)
+    for (sig, _), g in zip(rows, got):
+        assert int(g) == sig[0], (hex(int(g)), hex(sig[0]))
+        assert all(sig[0] != other for other in sig[1:])
