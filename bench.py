@@ -52,6 +52,8 @@ def parse_args():
                    help="only the calibration Gram-matrix measurement (one JSON line)")
     p.add_argument("--prefill-only", action="store_true",
                    help="only the prefill workload's bulk append + decode measurement (one JSON line)")
+    p.add_argument("--decode-only", action="store_true",
+                   help="only the graph-timed decode calls of the 128K and MHA workloads (one JSON line each)")
     return p.parse_args()
 
 
@@ -141,23 +143,24 @@ def code_sha256(paths):
 DECODE_SOURCES = ("decode.cu", "internal.h", "ptx.cuh", "prep.cuh", "qfrag.cuh")
 
 
-def profile_traffic(kernel_file):
-    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if that
-    summary was taken on the current kernel code (its code sha256 is recorded there)."""
+def profile_traffic(workload):
+    """DRAM bytes per launch of the decode call on `workload`, from the machine-readable ncu
+    record profiles/decode_traffic.json (dram__bytes_read.sum + dram__bytes_write.sum of the
+    decode kernels, the command that took it, and the sha256 of the kernel source it was
+    taken on).  Returns (bytes or None, why): None once the kernels have changed since."""
     srcs = [os.path.join(ROOT, "decode_attention_head_b200", "csrc", f) for f in DECODE_SOURCES]
-    path = os.path.join(ROOT, "profiles", kernel_file)
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
-        sha = code_sha256(srcs)
-        info = {}
-        for line in open(path):
-            if ":" in line and line.strip().startswith("- "):
-                k, v = line.strip()[2:].split(":", 1)
-                info[k.strip()] = v.strip().strip("`")
-        if info.get("decode code sha256") != sha:
-            return None
-        return float(info["dram bytes per launch (full workload)"])
-    except Exception:
-        return None
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None, "no ncu record"
+    entry = rec.get("workloads", {}).get(workload)
+    if entry is None:
+        return None, f"no ncu record for {workload}"
+    if rec.get("code_sha256") != code_sha256(srcs):
+        return None, "decode kernels changed since the ncu record was taken"
+    return float(entry["dram_bytes_per_launch"]), "ncu record " + rec.get("taken", "")
 
 
 class ClockSampler:
@@ -206,10 +209,12 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU baseline (oracle)
-def oracle_baseline(wl, target_seconds=12.0, max_steps=400, per_step_budget=None, warmup=0):
+def oracle_baseline(wl, target_seconds=12.0, max_steps=400, per_step_budget=None, warmup=0, layer=0,
+                    barrier=None):
     """Time the CPU oracle on a bounded sample: one (sequence, KV head) unit of `wl` at full
     context, stepping append-1 + decode like the GPU step (after `warmup` untimed steps).
-    Returns (GB/s, cores, sample, steps, seconds)."""
+    `layer` picks the unit's synthetic stream; `barrier` (a process pool's) is waited on
+    just before the timed steps.  Returns (GB/s, cores, sample, steps, seconds)."""
     import numpy as np
     from threadpoolctl import threadpool_limits
 
@@ -223,9 +228,9 @@ def oracle_baseline(wl, target_seconds=12.0, max_steps=400, per_step_budget=None
     extra = max_steps + warmup + 64
     oc = ocache.Cache(1, 1, d, wl.bits, wl.p_lo, wl.p_hi, wl.s_sink, wl.s_keep, wl.s_flush,
                       capacity=S0 + extra, chunk_max=1)
-    T = synth.key_transform(wl, 0, 0).numpy()[None]
-    k = synth.keys(wl, 0, 0, 0, 0, S0 + extra).numpy()
-    v = synth.values(wl, 0, 0, 0, 0, S0 + extra).numpy()
+    T = synth.key_transform(wl, layer, 0).numpy()[None]
+    k = synth.keys(wl, layer, 0, 0, 0, S0 + extra).numpy()
+    v = synth.values(wl, layer, 0, 0, 0, S0 + extra).numpy()
     oc.append(k[None, :S0, None], v[None, :S0, None], T)         # bulk prefill (not timed)
     q_all = np.stack([synth.queries(wl, 0, 0, S0 + i).numpy()[: wl.group] for i in range(8)])
     mirror = StateMirror(synth.scaled(wl, batch=1, n_kv_heads=1, n_q_heads=wl.group), S0, int(oc.S_quant[0]))
@@ -238,6 +243,8 @@ def oracle_baseline(wl, target_seconds=12.0, max_steps=400, per_step_budget=None
             if per_step_budget is None:
                 oatt.decode(oc, q_all[w % 8][None], T, scale)
         mirror = StateMirror(mirror.wl, int(oc.S[0]), int(oc.S_quant[0]))
+        if barrier is not None:
+            barrier.wait()
         t0 = time.perf_counter()
         while steps < max_steps:
             p = S0 + steps
@@ -273,6 +280,44 @@ def oracle_baseline(wl, target_seconds=12.0, max_steps=400, per_step_budget=None
         sample = (f"1 of {units} units, {steps} steps: append 1 token + exact softmax of {wl.group} heads over "
                   f"the newest {per_step_budget} positions (bounded slice of the {wl.context}-position cache)")
     return total_bytes / dt / 1e9, 1, sample, steps, dt
+
+
+def _oracle_worker(args):
+    """One process of the all-cores CPU baseline: the single-unit sample on unit `layer`."""
+    name, layer, steps, barrier = args
+    from decode_attention_head_b200 import synth
+    gbs, _, _, n, dt = oracle_baseline(synth.WORKLOADS[name], target_seconds=1e9, max_steps=steps, layer=layer,
+                                       barrier=barrier)
+    return gbs * dt, dt
+
+
+def cpu_model():
+    """The host CPU's model name (/proc/cpuinfo, as lscpu reports it)."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_baseline_all_cores(wl, steps=40, max_procs=32):
+    """The oracle on every available host core at once: one process per core (up to
+    `max_procs`), each stepping its own independent (sequence, KV head) unit as in
+    oracle_baseline; the processes start their timed steps together (a barrier) and the
+    aggregate is all their bytes over the slowest one's time.  Units are independent, so
+    this is the whole job's CPU throughput on those cores.  Returns (GB/s, processes)."""
+    import multiprocessing as mp
+    n = max(1, min(len(os.sched_getaffinity(0)), max_procs))
+    ctx = mp.get_context("spawn")  # the parent holds a CUDA context: never fork it
+    with ctx.Manager() as mgr:
+        barrier = mgr.Barrier(n)
+        with ctx.Pool(n) as pool:
+            res = pool.map(_oracle_worker, [(wl.name, 100 + i, steps, barrier) for i in range(n)])
+    total = sum(r[0] for r in res)
+    return total * 1e9 / max(r[1] for r in res) / 1e9, n
 
 
 # ------------------------------------------------------------------ GPU run
@@ -521,6 +566,7 @@ def run_gpu(args, rank, world, local_rank):
         del g_e2e
 
     peak, peak_kind = measured_peaks()
+    traffic, traffic_why = profile_traffic(wl.name)
     dec_launch_s = dec_total / K2
     dec_bytes_per_launch = k2_dec_bytes / K2
     achieved = dec_bytes_per_launch / dec_launch_s / 1e9
@@ -559,7 +605,8 @@ def run_gpu(args, rank, world, local_rank):
         "layer_tokens_per_s": round(world * wl.batch * K / t_total, 1),
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": profile_traffic("decode_main_llama3-8b-layer.md"),
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "traffic_source": traffic_why,
             "kernel": "wushkv_decode_attn (decode_prologue + decode_main)", "peak_kind": peak_kind,
         },
         "gpu_launches": 2 * K,  # per timed step: fused append_small + decode_main
@@ -571,6 +618,9 @@ def run_gpu(args, rank, world, local_rank):
     if not args.no_prefill:
         del caches, outs
         torch.cuda.empty_cache()
+        # the long-context and batched decode workloads, graph-timed per launch
+        result["decode_workloads"] = {name: measure_decode(bnd, synth, dev, name, layers)
+                                      for name, layers in DECODE_WORKLOADS}
         result["prefill_append"] = measure_prefill(bnd, synth, dev)
         result["chunk_prefill"] = measure_chunk(bnd, synth, dev)
         result["calibration_gram"] = measure_gram(bnd, synth, dev)
@@ -644,6 +694,82 @@ def measure_prefill(bnd, synth, dev, reps=5):
             "decode_us_at_131072": round(dec_s * 1e6, 2), "decode_gbs": round(dec_bytes / dec_s / 1e9, 2),
             "launch": "eager, 3 append launches (flush_ring, append_bulk, advance_state) + 2 decode launches",
             "reps": reps}
+
+
+DECODE_WORKLOADS = (("qwen3-8b-layer", 8), ("prefill-append-decode", 3), ("mha-32l", 4))
+
+
+def measure_decode(bnd, synth, dev, name, layers, reps=200, warmup=10):
+    """Decode calls of one workload as a serving engine issues them: `layers` layer caches
+    (the workload's shape, filled by bulk appends to its full context, so the quantized
+    region is at its steady state) rotate so that the working set is larger than four times
+    L2; each call is a CUDA graph replay (prologue + main kernel), timed per launch with CUDA
+    events on the launching stream.  The decode never changes the cache, so every call
+    reads the same bytes.  Algorithmic bytes per call: the per-unit costs (codes and (s, z)
+    of the quantized positions, fp16 window rows, q in / out, T_K^{-1})."""
+    import torch
+    wl = synth.WORKLOADS[name] if isinstance(name, str) else name
+    name = wl.name
+    cfg = bnd.config_for_workload(wl, extra_capacity=64)
+    caches, tinvs = [], []
+    for layer in range(layers):
+        c = bnd.KVCache(cfg, device=dev)
+        T = synth.key_transforms(wl, layer)
+        tk = T.to(dev)
+        for s0 in range(0, wl.context, 4096):
+            n = min(4096, wl.context - s0)
+            c.append(synth.bulk_tokens(wl, layer, s0, n, device=dev, which="k"),
+                     synth.bulk_tokens(wl, layer, s0, n, device=dev, which="v"), tk)
+        caches.append(c)
+        tinvs.append(bnd.compensation(T).to(dev))
+    torch.cuda.synchronize()
+    S, Sq = (int(t[0, 0].item()) for t in caches[0].lengths())
+    assert S == wl.context and all(c.status() == 0 for c in caches)
+    q = [synth.bulk_queries(wl, layer, S, device=dev) for layer in range(layers)]
+    outs = [torch.empty(wl.batch, wl.n_q_heads, wl.head_dim, device=dev) for _ in range(layers)]
+    scale = synth.default_softmax_scale(wl.head_dim)
+    stream = torch.cuda.Stream(device=dev)
+    graphs = []
+    with torch.cuda.stream(stream):
+        for c in range(layers):  # one eager call per layer first (kernel attributes outside capture)
+            caches[c].decode_attn(q[c], tinvs[c], scale, out=outs[c], stream=stream)
+        stream.synchronize()
+        for c in range(layers):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                caches[c].decode_attn(q[c], tinvs[c], scale, out=outs[c], stream=stream)
+            graphs.append(g)
+        for j in range(warmup):
+            graphs[j % layers].replay()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        stream.synchronize()
+        for j in range(reps):
+            evs[j].record(stream)
+            graphs[j % layers].replay()
+        evs[reps].record(stream)
+    stream.synchronize()
+    ms = [evs[j].elapsed_time(evs[j + 1]) for j in range(reps)]
+    assert all(c.status() == 0 for c in caches)
+    del graphs
+    t = sum(ms) / len(ms) / 1e3
+    nbytes = StateMirror(wl, S, Sq).decode_bytes()
+    peak, peak_kind = measured_peaks()
+    units_bytes = (bnd.pack_layout(cfg).codes_bytes + bnd.pack_layout(cfg).params_bytes) * 2
+    res = {"workload": name, "batch": wl.batch, "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads,
+           "context": S, "bits": wl.bits, "decode_us_per_launch": round(t * 1e6, 3),
+           "decode_us_median": round(statistics.median(ms) * 1e3, 3), "bytes_per_launch": nbytes,
+           "decode_gbs": round(nbytes / t / 1e9, 2), "frac_measured_hbm": round(nbytes / t / 1e9 / peak, 4),
+           "pct_of_8tbps": round(100 * nbytes / t / 1e9 / NOMINAL_HBM_GBS, 2), "peak_kind": peak_kind,
+           "layers_rotated": layers, "working_set_gb": round(layers * units_bytes / 1e9, 2),
+           "launch": "one CUDA graph per decode call (prologue + main), events per launch", "reps": reps}
+    if wl.n_layers > 1:  # a decode step of the whole model: one call per layer, all layers alike
+        res["model_step_ms"] = round(wl.n_layers * t * 1e3, 3)
+        res["tokens_per_s"] = round(wl.batch / (wl.n_layers * t), 1)
+    else:
+        res["layer_tokens_per_s"] = round(wl.batch / t, 1)
+    del caches, outs
+    torch.cuda.empty_cache()
+    return res
 
 
 def workload_config(wl):
@@ -782,6 +908,16 @@ def main():
         torch.cuda.set_device(dev)
         print(json.dumps(measure_gram(bnd, synth, dev)))
         return 0
+    if args.decode_only:
+        from decode_attention_head_b200 import binding as bnd
+        from decode_attention_head_b200 import build as _build
+        from decode_attention_head_b200 import synth
+        _build.build()
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        for name, layers in DECODE_WORKLOADS:
+            print(json.dumps(measure_decode(bnd, synth, dev, name, layers)), flush=True)
+        return 0
     if args.prefill_only:
         from decode_attention_head_b200 import binding as bnd
         from decode_attention_head_b200 import build as _build
@@ -799,9 +935,15 @@ def main():
     result, wl = run_gpu(args, rank, world, local_rank)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            val, cores, sample, steps, dt = oracle_baseline(wl)
-            result["cpu_baseline"] = {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                                      "sample": sample}
+            val1, _, sample, steps, dt = oracle_baseline(wl)
+            val, cores = oracle_baseline_all_cores(wl)
+            result["cpu_baseline"] = {
+                "value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                "sample": f"{cores} processes, one per core, each stepping its own (sequence, KV head) unit of the "
+                          f"workload at context {wl.context} (append 1 token + decode {wl.group} query heads, 40 "
+                          f"steps, started together); aggregate bytes over the slowest process's time",
+                "single_core": {"value": round(val1, 4), "sample": sample},
+                "cpu_model": cpu_model(), "host_cores": os.cpu_count()}
         else:
             result["cpu_baseline"] = None
         print(json.dumps(result))

@@ -21,7 +21,7 @@ _ERR = {EINVAL: "invalid argument", EUNSUPPORTED: "unsupported configuration", E
         ESINGULAR: "singular key transform", ESCRATCH: "needs more than the static scratch array holds"}
 SYMBOLS = ("wushkv_pack_layout", "wushkv_compensation", "wushkv_hadamard", "wushkv_append", "wushkv_decode_attn",
            "wushkv_chunk_attn", "wushkv_step", "wushkv_step_prep", "wushkv_decode_attn_static",
-           "wushkv_gram_accumulate")
+           "wushkv_gram_accumulate", "wushkv_decode_attn_test_timeout")
 
 
 class Prep(ctypes.Structure):
@@ -85,6 +85,10 @@ def _load() -> ctypes.CDLL:
     lib.wushkv_decode_attn_static.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs), ctypes.c_void_p,
                                               ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p,
                                               ctypes.c_void_p]
+    lib.wushkv_decode_attn_test_timeout.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(CacheBufs),
+                                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                                    ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                                    ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p]
     lib.wushkv_gram_accumulate.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p,
                                            ctypes.c_void_p]
     for name in SYMBOLS:
@@ -277,6 +281,20 @@ class KVCache:
                                              1 if out.dtype == torch.float16 else 0, out.data_ptr(),
                                              _stream_ptr(stream)),
                "wushkv_decode_attn_static")
+        return out
+
+    def decode_attn_test_timeout(self, q: torch.Tensor, t_k_inv: torch.Tensor, softmax_scale: float,
+                                 out: torch.Tensor, withhold_stage: int, wait_limit_cycles: int,
+                                 stream=None) -> torch.Tensor:
+        """The bounded-wait test hook (wushkv_decode_attn_test_timeout): a shortened wait
+        limit and one withheld pipeline stage per work item."""
+        _require_cuda(q, t_k_inv, out)
+        _check(lib.wushkv_decode_attn_test_timeout(ctypes.byref(self.cfg), ctypes.byref(self.bufs), q.data_ptr(),
+                                                   t_k_inv.data_ptr(), float(softmax_scale),
+                                                   1 if out.dtype == torch.float16 else 0, out.data_ptr(),
+                                                   self.workspace.data_ptr(), int(withhold_stage),
+                                                   int(wait_limit_cycles), _stream_ptr(stream)),
+               "wushkv_decode_attn_test_timeout")
         return out
 
     # -- typed views of the buffers (for tests and tools) ------------------------

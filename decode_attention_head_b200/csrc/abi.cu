@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include "internal.h"
 #include "gram.h"
+#include "ptx.cuh"
 #include "qfrag.cuh"
 
 namespace wushkv {
@@ -280,6 +281,8 @@ static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv
   a->gq = d.group;
   a->chunk_n = 0;
   a->chunk_t0 = 0;
+  a->withhold_tile = -1;
+  a->wait_limit = kWaitLimitCycles;
 }
 
 static int check_append(const wushkv_config* cfg, const wushkv_cache* cache, const void* k_new, const void* v_new,
@@ -344,6 +347,24 @@ extern "C" int wushkv_decode_attn(const wushkv_config* cfg, const wushkv_cache* 
   if (rc != WUSHKV_OK) return rc;
   DecodeArgs a;
   fill_decode(cfg, d, cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace, &a);
+  const cudaError_t e = launch_decode(d, cfg->bits, a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA;
+}
+
+extern "C" int wushkv_decode_attn_test_timeout(const wushkv_config* cfg, const wushkv_cache* cache, const void* q,
+                                               const float* t_k_inv, float softmax_scale, int32_t out_fp16,
+                                               void* out, void* workspace, int32_t withhold_stage,
+                                               int64_t wait_limit_cycles, void* stream) {
+  Derived d;
+  int rc = derive(cfg, &d);
+  if (rc != WUSHKV_OK) return rc;
+  rc = check_decode(cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace);
+  if (rc != WUSHKV_OK) return rc;
+  if (withhold_stage < -1 || wait_limit_cycles < 1000 || wait_limit_cycles > kWaitLimitCycles) return WUSHKV_EINVAL;
+  DecodeArgs a;
+  fill_decode(cfg, d, cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace, &a);
+  a.withhold_tile = withhold_stage;
+  a.wait_limit = wait_limit_cycles;
   const cudaError_t e = launch_decode(d, cfg->bits, a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA;
 }

@@ -6,9 +6,11 @@
 // The attention itself is the ordinary wushkv_decode_attn path: this file only supplies
 // its `workspace` argument.  The array is file-scope `static __device__`, so every
 // device that loads the library holds WUSHKV_STATIC_SCRATCH_BYTES of it until the
-// process exits; its device address is looked up once per device with
-// cudaGetSymbolAddress (the host-side name is not a device address).
+// process exits; its device address is looked up with cudaGetSymbolAddress (the
+// host-side name is not a device address) once per CUDA context, on the first call made
+// in that context.
 #include <cmath>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <mutex>
 #include "internal.h"
@@ -17,26 +19,56 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_scratch[WUSHKV_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
+// The array's device address depends on the CUDA context the library's module is loaded
+// in (each device's primary context, or a context the caller created), so it is cached
+// per context: looked up on the first call made in a context and reused afterwards.
+constexpr int kMaxContexts = 64;
 std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_ctx[kMaxContexts] = {};
+void* g_scratch_ptr[kMaxContexts] = {};
+int g_entries = 0;
 
-// Device address of g_scratch on the current device, looked up on the first call made
-// with that device current and cached afterwards.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// The driver's cuCtxGetCurrent, fetched through the runtime (no link against libcuda).
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetCurrentFn>(nullptr);
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
+
+// Device address of g_scratch in the current context.
 cudaError_t scratch_address(void** out) {
   int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = cudaGetDevice(&dev);  // also makes the device's primary context current if none is
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  e = cudaFree(nullptr);                // initialise the context without allocating
+  if (e != cudaSuccess) return e;
+  const CtxGetCurrentFn get = ctx_get_current();
+  CUcontext ctx = nullptr;
+  if (!get || get(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_scratch);
-    if (e != cudaSuccess) return e;
-    if (!p) return cudaErrorInvalidSymbol;
-    g_scratch_ptr[dev] = p;
+  for (int i = 0; i < g_entries; ++i) {
+    if (g_ctx[i] == ctx) {
+      *out = g_scratch_ptr[i];
+      return cudaSuccess;
+    }
   }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_scratch);
+  if (e != cudaSuccess) return e;
+  if (!p) return cudaErrorInvalidSymbol;
+  // a full table (more contexts than any process here creates) overwrites the oldest entry
+  const int slot = g_entries < kMaxContexts ? g_entries++ : 0;
+  g_ctx[slot] = ctx;
+  g_scratch_ptr[slot] = p;
+  *out = p;
   return cudaSuccess;
 }
 
@@ -64,10 +96,9 @@ extern "C" int wushkv_decode_attn_static(const wushkv_config* cfg, const wushkv_
   if (d.ws_total > (size_t)WUSHKV_STATIC_SCRATCH_BYTES) return WUSHKV_ESCRATCH;
   void* ws = nullptr;
   if (scratch_address(&ws) != cudaSuccess) return WUSHKV_ECUDA;
-  // The array keeps whatever the previous call (of any configuration) left in it; the
-  // completion counters of the split merge must start at zero.
-  if (cudaMemsetAsync(static_cast<unsigned char*>(ws) + d.ws_tickets, 0, d.ws_qprime - d.ws_tickets,
-                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return WUSHKV_ECUDA;
+  // The array keeps whatever the previous call (of any configuration) left in it.  Nothing
+  // needs clearing here: the decode's own first kernel (the prologue) resets the split
+  // merge's completion counters on every call, and every other part of the workspace is
+  // written before it is read.
   return wushkv_decode_attn(cfg, cache, q, t_k_inv, softmax_scale, out_fp16, out, ws, stream);
 }

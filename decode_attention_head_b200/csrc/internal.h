@@ -13,8 +13,8 @@ constexpr int kHeadDim = 128;
 constexpr int kTileTokens = 128;      // positions per decode pipeline stage (and cap_alloc granule)
 constexpr int kB200SMs = 148;         // split policy sizes the decode grid for this many SMs
 // Resident decode CTAs per SM the split policy aims at (the kernel's launch bounds hold its
-// registers to this): 8 query heads per KV head need more registers than the others.
-constexpr int decode_ctas_per_sm(int group) { return group == 8 ? 3 : 4; }
+// registers to this; each CTA holds 128 of the SM's 512 tensor-memory columns).
+constexpr int decode_ctas_per_sm(int group) { return group > 0 ? 2 : 2; }
 constexpr int kMaxSplits = 255;       // quantized work items per (sequence, KV head)
 constexpr int kMergeGroup = 16;       // work items merged together at the first merge level
 
@@ -115,6 +115,10 @@ struct DecodeArgs {
   // are [B][chunk_n][H_q][128]; chunk_n = 0 for a one-token decode (gq = G)
   int chunk_n, chunk_t0, gq;
   PrepSpec prep;       // raw q (wushkv_step_prep, bulk route): the prologue normalises and rotates it
+  // bounded waits: the cycle limit after which a wait gives up (STATUS_TIMEOUT), and a test
+  // hook -- the producer never issues stage `withhold_tile` of any item (-1: off)
+  int withhold_tile;
+  long long wait_limit;
 };
 
 // Raise a kernel's dynamic shared-memory limit once per device (a function attribute,

@@ -286,6 +286,21 @@ int wushkv_step_prep(const wushkv_config* cfg, const wushkv_cache* cache, const 
                      int32_t n_new, const void* t_k, const void* q_raw, const float* t_k_inv, float softmax_scale,
                      int32_t out_fp16, void* out, void* workspace, const wushkv_prep* prep, void* stream);
 
+/* Test hook for the bounded waits (not a production entry point; no counterpart in the
+ * method): wushkv_decode_attn with the in-kernel wait limit shortened to wait_limit_cycles
+ * (1000 .. the default of about 2 s of SM clock) and, when withhold_stage >= 0, stage
+ * withhold_stage of every work item's pipeline never issued, so that its consumers give up.
+ * Nothing faults or traps: a wait that gives up sets WUSHKV_STATUS_TIMEOUT, every warp of the
+ * work item leaves its loop, the copies already issued land, the tensor memory is released,
+ * and the item writes no partial result -- the output rows of an affected unit are not
+ * written (they keep whatever the buffer held).  The cache and the workspace are left usable
+ * for the next call.  Returns as wushkv_decode_attn, or WUSHKV_EINVAL for an out-of-range
+ * hook argument. */
+int wushkv_decode_attn_test_timeout(const wushkv_config* cfg, const wushkv_cache* cache, const void* q,
+                                    const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
+                                    void* workspace, int32_t withhold_stage, int64_t wait_limit_cycles,
+                                    void* stream);
+
 /* wushkv_decode_attn with library-owned scratch instead of a caller-allocated workspace.
  * The method has no counterpart of this call: it serves callers that cannot allocate
  * device memory when they decode (a runtime without an allocator, a step that must not

@@ -16,6 +16,8 @@ build.build()
 
 from decode_attention_head_b200 import binding as bnd  # noqa: E402
 from decode_attention_head_b200 import synth  # noqa: E402
+from oracle import attention as oatt  # noqa: E402
+from tests import harness as H  # noqa: E402
 from tests.harness import ATOL  # noqa: E402
 
 pytestmark = pytest.mark.gpu
@@ -27,6 +29,7 @@ def _filled_cache(cfg, n_bulk, n_single, seed):
     wl = synth.WORKLOADS["tiny"]
     t_k = torch.stack([synth.key_transform(wl, seed, h) for h in range(cfg.n_kv_heads)])
     gc = bnd.KVCache(cfg)
+    gc.t_k_host = t_k.numpy()
     t_dev = t_k.cuda()
 
     def tok(n, scale):
@@ -53,11 +56,18 @@ def _static(case, out_dtype):
 
 
 def _compare(case, out, ref):
-    gc = case[0]
+    """The same kernels run on the same inputs with the scratch in another place: the result
+    must be the workspace path's bit for bit (a stale-scratch leak of any size fails), and
+    the oracle's within the attention tolerance."""
+    gc, q = case[0], case[1]
     assert gc.status() == 0
     err = (out.float() - ref.float()).abs().max().item()
     print(f"[no-alloc] units={gc.units} splits={gc.layout.n_splits} dtype={out.dtype} max|diff|={err:.3g}")
     assert np.isfinite(err) and err <= ATOL
+    assert torch.equal(out, ref)
+    if out.dtype == torch.float32:
+        want = oatt.decode(H.oracle_cache_from_gpu(gc), q.cpu().numpy(), gc.t_k_host, SCALE)
+        H.assert_attention_close(out.cpu().numpy(), want)
 
 
 def test_static_scratch_matches_workspace_path():
