@@ -5,7 +5,7 @@
 //
 // Two launches per call:
 //  1. decode_prologue (one 512-thread CTA per (sequence, KV head)): q'_j = T_K^{-T} q_j
-//     for its g query heads in fp32, the query's fixed-point tensor-core operand built
+//     for its g query heads in fp32, the query's fixed-point tensor-core fragments built
 //     from it (qfrag.cuh), and the reset of the unit's completion counters.  It releases
 //     the main kernel at once (programmatic dependent launch), so the main kernel's KV
 //     stream starts while it runs.  (In a fused step, wushkv_step, the append kernel does
@@ -16,34 +16,29 @@
 //     the unit's current quantized region [S_sink, S_quant) (whole 128-position stages)
 //     and of its fp16 window positions (sink [0, S_sink) and recent [S_quant, S)).
 //     The quantized positions stream through shared memory in 128-position stages
-//     (K codes, V codes, K and V (s, z)) via bulk copies on an mbarrier ring.  Ten warps:
-//       producer  one lane issues the stages' bulk copies;
-//       MMA       one lane issues, per stage, the QK^T product on the fifth-generation
-//                 tensor cores: tcgen05.mma kind::i8, M = 128 positions, N = 4 limbs per
-//                 query head, K = 128 masked key codes (u8, in tensor memory) x the
-//                 query's signed 8-bit limbs (shared memory), exact int32 in tensor memory;
-//       position warps (4)  one thread per position: mask the stage's key codes into the
-//                 MMA's A operand (tensor memory), then read their row of q'.c back,
-//                 form the logits log2e*scale*(z*sum(q') + s*sigma*D) (dequantization
-//                 folded), run the online softmax (base 2, a running max that may go
-//                 stale by 2^8) and write the PV weights p*s (fp16 hi + lo) for
-//       value warps (4)  paired one to one with the position warps (the same 32 positions
-//                 of every stage): PV on mma.sync m16n8k16 with the V codes unpacked in
-//                 registers as exact fp16 subnormals, fp32 accumulate; before the stages
-//                 they take the item's share of the fp16 window on an exact scalar path.
+//     (K codes, V codes, K and V (s, z)) via bulk copies on an mbarrier ring: one
+//     producer warp, four consumer warps, 32 positions per consumer warp per stage.
+//     The consumer warps take q' as a 31-bit fixed-point integer split into four signed
+//     8-bit limbs, already laid out as the mma.sync B fragments they need:
+//       QK  : u8 codes x s8 query limbs on tensor cores (mma m16n8k32, exact int32),
+//             logit = log2e*scale*(z*sum(q') + s*sigma*D)  (dequantization folded);
+//       softmax: online, base 2, with a running max that may go stale by 2^8;
+//       PV  : fp16 codes x fp16 (p*s as hi + lo) on tensor cores (mma m16n8k16,
+//             fp32 accumulate), plus sum(p*z) for the zero-point term.
 //     Each item merges its warps and writes (m, l, o); the last item of each group of
 //     items merges the group, the last group merges the groups and writes the output
 //     (atomic counters, nobody waits).
 //
-// Key codes: masking a packed 32-bit word with 0x03030303 << 2m leaves, in each byte, one
-// code times 4^m -- an exact u8 operand; the 4^m is divided out of the query's integer
-// representation.  Value codes: pairs of 16-bit code chunks (one per token) are shifted so
-// that one code sits at bits 4..9 of each half and masked: the half is then the fp16
-// subnormal c * 2^(b-24) (b = 4, 6 or 8, the code's lowest bit), an exact operand whose
-// power-of-two scale is undone once per output row.  Codes are kept high in the subnormal
-// range on purpose: the tensor core aligns a product by the operand's nominal exponent (-14
-// for every subnormal), so each leading zero bit of a subnormal costs one bit of the
-// product's precision inside the MMA; at bits 4..9 at most 6 of 24 are lost.
+// Code unpacking needs no shifts on the key side: masking a packed 32-bit word with
+// 0x03030303 << 2j leaves, in each byte, one code times 4^j -- an exact u8 operand.
+// The key-side scale 4^j is divided out of the query's integer representation.  On
+// the value side, pairs of 16-bit code chunks (one per token) are shifted so that one
+// code sits at bits 4..9 of each half and masked: the half is then the fp16 subnormal
+// c * 2^(b-24) (b = 4, 6 or 8, the code's lowest bit), an exact operand whose
+// power-of-two scale is undone once per output row.  Codes are kept high in the
+// subnormal range on purpose: the tensor core aligns a product by the operand's nominal
+// exponent (-14 for every subnormal), so each leading zero bit of a subnormal costs one
+// bit of the product's precision inside the MMA; at bits 4..9 at most 6 of 24 are lost.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <climits>
@@ -56,18 +51,12 @@
 namespace wushkv {
 namespace {
 
-constexpr int kPosWarps = 4;             // one thread per position of a 128-position stage
-constexpr int kValWarps = 4;             // PV partners of the position warps
-constexpr int kConsumers = 4;            // pseudo-warps per path in the item merge
-constexpr int kProducerWarp = kPosWarps + kValWarps;
-constexpr int kMmaWarp = kProducerWarp + 1;
-constexpr int kThreads = 32 * (kMmaWarp + 1);
-constexpr int kSlice = 32;               // positions per warp pair per stage
+constexpr int kThreads = 160;            // 4 consumer warps + 1 producer warp
+constexpr int kConsumers = 4;
+constexpr int kSlice = 32;               // positions per consumer warp per stage
 constexpr int kPartStride = 132;         // floats per (item, head) partial: m, l, pad, pad, o[128]
 constexpr int kTau = 8;                  // log2 headroom of the stale running max
-constexpr int kQkBufs = 4;               // key operands / QK results in flight (tensor memory)
-constexpr uint32_t kTmemCols = 256;      // 4 key operands (32 columns each) + 4 QK results (16 or 32)
-static_assert(kTileTokens == kPosWarps * kSlice, "a stage holds one slice per warp pair");
+static_assert(kTileTokens == kConsumers * kSlice, "a stage holds one slice per consumer warp");
 
 // 2^n as an fp32 bit pattern, exact for -126 <= n <= 127.
 __device__ __forceinline__ float pow2i(int n) { return __int_as_float((n + 127) << 23); }
@@ -78,6 +67,7 @@ __device__ __forceinline__ float ex2(float x) {  // 2^x (hardware approximation,
   return y;
 }
 
+
 // Row (in units of 128 elements) of query head v (0..G-1) of unit (b, h) in q and out: a
 // one-token decode has its G heads side by side; chunk attention's v is token v / gq of the
 // launch's block of the chunk, head v % gq.
@@ -87,13 +77,10 @@ __device__ __forceinline__ size_t head_row(const DecodeArgs& a, int b, int h, in
   return ((size_t)b * ntok + a.chunk_t0 + t) * a.Hq + (size_t)h * a.gq + hh;
 }
 
-// Stage ring depth: a stage holds its shared-memory slot from the copy's issue until its PV
-// is done (load latency plus three hand-offs), so each CTA keeps as many stages in flight as
-// two CTAs per SM can hold (2-bit: 8 x 9 KB; 4-bit: 5 x 17 KB, 4 at eight query heads).
-template <int BITS, int G>
+template <int BITS>
 struct Cfg {
   static constexpr int CB = 16 * BITS;
-  static constexpr int NSTAGE = BITS == 2 ? 8 : (G == 8 ? 4 : 5);
+  static constexpr int NSTAGE = BITS == 2 ? 4 : 2;  // 4-bit: two 17 KB stages keep four CTAs per SM
   static constexpr int STAGE = kTileTokens * (2 * CB + 8);
 };
 
@@ -194,6 +181,33 @@ __global__ void __launch_bounds__(kPrologueThreads) decode_prologue_kernel(const
                              [] { __syncthreads(); });
 }
 
+// The unit's query fragments and per-head constants (built by the prologue or the fused
+// append, staged in shared memory), loaded by one lane: bq[j][nt][r], and for the lane's
+// logit head t4 + 4*hs the constants log2e*scale*sum(q') (zero-point term) and
+// log2e*scale*sigma.
+template <int G>
+__device__ __forceinline__ void load_query(const uint8_t* qfs, int lane, int t4, uint32_t (&bq)[4][GCfg<G>::NT][2],
+                                           float (&Ah)[GCfg<G>::NHS], float (&Bh)[GCfg<G>::NHS]) {
+  constexpr int NT = GCfg<G>::NT, NHS = GCfg<G>::NHS, FW = GCfg<G>::FW;
+  const uint4* src = reinterpret_cast<const uint4*>(qfs) + lane;
+#pragma unroll
+  for (int m = 0; m < FW / 4; ++m) {
+    const uint4 u = src[32 * m];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int idx = 4 * m + e;
+      bq[(idx >> 1) / NT][(idx >> 1) % NT][idx & 1] = w[e];
+    }
+  }
+  const float* hc = reinterpret_cast<const float*>(qfs + FW * 32 * 4);
+#pragma unroll
+  for (int hs = 0; hs < NHS; ++hs) {
+    Ah[hs] = hc[t4 + 4 * hs];
+    Bh[hs] = hc[8 + t4 + 4 * hs];
+  }
+}
+
 // ---------------------------------------------------------------------------------
 struct Merge {  // per pseudo-warp (0..3 quantized path, 4..7 window path) and head
   float m[8][8], l[8][8], bias[8][8];
@@ -201,57 +215,257 @@ struct Merge {  // per pseudo-warp (0..3 quantized path, 4..7 window path) and h
   float M[8], L[8];   // the item's merged max and denominator per head
 };
 
-// PV weights handed from a position warp to its value warp, per stage (double-buffered):
-// for each of the two 16-position k-blocks, NC columns (G <= 4: heads' hi parts in columns
-// 0..3 and lo parts in 4..7; G = 8: hi in 0..7, lo in 8..15) of eight 32-bit words; word
-// 2 * (r % 4) + (r / 4) % 2 of a column holds block positions r (low half) and r + 8, as the
-// m16n8k16 B fragment of lane (g = column, t4 = r % 4) wants them.  Then a header: a flag
-// and, when it is set, the factor each head's accumulator must first be multiplied by.
-template <int G>
-struct WB {
-  static constexpr int NC = G <= 4 ? 8 : 16;
-  static constexpr int KB = NC * 32 + 32;     // one k-block, padded: conflict-free stores
-  static constexpr int HDR = 2 * KB;          // int flag, pad, float factor[8]
-  static constexpr int BYTES = HDR + 48;
-};
-
 template <int BITS, int G>
 struct Shared {
-  static constexpr int kStages = Cfg<BITS, G>::NSTAGE * Cfg<BITS, G>::STAGE;
+  static constexpr int kStages = Cfg<BITS>::NSTAGE * Cfg<BITS>::STAGE;
   static constexpr int kPv = kConsumers * G * kHeadDim * 4;  // [4][G][128] fp32, reuses the stages
   static constexpr int kArena = kStages > kPv ? kStages : kPv;
-  static constexpr int kWbuf = kPosWarps * 2 * WB<G>::BYTES;
-  static constexpr int kNumBars = 2 * Cfg<BITS, G>::NSTAGE + 2 * kQkBufs + 4 * kPosWarps;
-  static constexpr size_t kFixed = (size_t)kArena + kWbuf + GCfg<G>::QBYTES + kNumBars * 8 + sizeof(Merge) +
-                                   (size_t)kPv + 64;
-  static size_t bytes(int nitems) { return kFixed + (size_t)nitems * G * 4; }
+  static size_t bytes(int nitems) {
+    return (size_t)kArena + 2 * Cfg<BITS>::NSTAGE * 8 + sizeof(Merge) + (size_t)kPv + kQFragBytes +
+           (size_t)nitems * G * 4;
+  }
 };
 
-// One position thread's key record (stage row r) masked into the 32 columns of its tensor
-// memory lane: column c = 8 m + w holds word w & (0x03030303 << 2 m) (2-bit), column
-// c = 16 m + w holds word w & (0x0F0F0F0F << 4 m) (4-bit) -- the K order qfrag.cuh encodes.
-template <int BITS>
-__device__ __forceinline__ void store_key_operand(const uint8_t* st, int r, uint32_t taddr) {
+// Per-warp online-softmax state of the quantized path.
+template <int NHS>
+struct QState {
+  float m[NHS], l[NHS], bias[NHS];
+  float o[8][4];
+  int kacc;
+  float s_lim;
+};
+
+// One consumer warp's 32-position slice of a stage.  FULL: every position is in range.
+template <int BITS, int G, bool FULL>
+__device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, int tpos, int vlo, int vhi,
+                                      const uint32_t (&bq)[4][GCfg<G>::NT][2], const float (&Ah)[GCfg<G>::NHS],
+                                      const float (&Bh)[GCfg<G>::NHS], const bool (&hvalid)[GCfg<G>::NHS],
+                                      QState<GCfg<G>::NHS>& s, int g, int t4) {
+  constexpr int NT = GCfg<G>::NT, NHS = GCfg<G>::NHS;
   constexpr int CB = 16 * BITS;
-  const uint4* rec = reinterpret_cast<const uint4*>(st + r * CB);
-  uint32_t v[32];
-  if (BITS == 2) {
-    const uint4 u0 = rec[0], u1 = rec[1];
-    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+  const uint8_t* kc = st;
+  const uint8_t* vc = st + kTileTokens * CB;
+  const uint32_t* kpar = reinterpret_cast<const uint32_t*>(st + 2 * kTileTokens * CB);
+  const uint32_t* vpar = kpar + kTileTokens;
+
+  // ---- QK^T over two 16-position m-tiles: rows base + 16i + g (+8)
+  int acc[2][NT][4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[8 * m + i] = w[i] & (0x03030303u << (2 * m));
-  } else {
-    const uint4 u0 = rec[0], u1 = rec[1], u2 = rec[2], u3 = rec[3];
-    const uint32_t w[16] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w,
-                            u2.x, u2.y, u2.z, u2.w, u3.x, u3.y, u3.z, u3.w};
+    for (int nt = 0; nt < NT; ++nt) acc[i][nt][0] = acc[i][nt][1] = acc[i][nt][2] = acc[i][nt][3] = 0;
 #pragma unroll
-    for (int m = 0; m < 2; ++m)
+  for (int i = 0; i < 2; ++i) {
+    const int r0 = base + 16 * i + g, r1 = r0 + 8;
+    if (BITS == 2) {
+      const uint2 ka = *reinterpret_cast<const uint2*>(kc + r0 * CB + 8 * t4);
+      const uint2 kb = *reinterpret_cast<const uint2*>(kc + r1 * CB + 8 * t4);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[16 * m + i] = w[i] & (m ? 0xF0F0F0F0u : 0x0F0F0F0Fu);
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t mk = 0x03030303u << (2 * j);
+        const uint32_t A[4] = {ka.x & mk, kb.x & mk, ka.y & mk, kb.y & mk};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[i][nt], A, bq[j][nt]);
+      }
+    } else {
+      const uint4 ka = *reinterpret_cast<const uint4*>(kc + r0 * CB + 16 * t4);
+      const uint4 kb = *reinterpret_cast<const uint4*>(kc + r1 * CB + 16 * t4);
+      const uint32_t kaw[4] = {ka.x, ka.y, ka.z, ka.w};
+      const uint32_t kbw[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t mk = (j & 1) ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
+        const int wa = 2 * (j >> 1);
+        const uint32_t A[4] = {kaw[wa] & mk, kbw[wa] & mk, kaw[wa + 1] & mk, kbw[wa + 1] & mk};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[i][nt], A, bq[j][nt]);
+      }
+    }
   }
-  tmem_st32(taddr, v);
+
+  // ---- logits (base 2) of this lane's 4 positions: rows base + 16i + g + 8u
+  float2 ksz[2][2], vsz[2][2];
+  bool val[2][2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = base + 16 * i + g + 8 * u;
+      ksz[i][u] = __half22float2(u32_as_h2(kpar[r]));
+      vsz[i][u] = __half22float2(u32_as_h2(vpar[r]));
+      val[i][u] = FULL || (tpos + r >= vlo && tpos + r < vhi);
+    }
+  // The running max is kept stale: p = 2^(x - mref) may reach 2^kTau, and only a logit above
+  // mref + kTau (a warp vote) triggers the rescale, so the common path has no reduction.
+  float x[2][2][NHS], alpha[NHS];
+  bool hit = false;
+#pragma unroll
+  for (int hs = 0; hs < NHS; ++hs) {
+    float mx = -CUDART_INF_F;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        // q'.c / sigma = sum_l 256^l D_l; pairs of limbs combine exactly in int32
+        const int d01 = acc[i][hs][2 * u] + 256 * acc[i][hs][2 * u + 1];
+        const int d23 = acc[i][NHS + hs][2 * u] + 256 * acc[i][NHS + hs][2 * u + 1];
+        const float f = fmaf(65536.0f, (float)d23, (float)d01);
+        const float xv = fmaf(Bh[hs] * ksz[i][u].x, f, Ah[hs] * ksz[i][u].y);
+        x[i][u][hs] = (val[i][u] && hvalid[hs]) ? xv : -CUDART_INF_F;
+        mx = fmaxf(mx, x[i][u][hs]);
+      }
+    alpha[hs] = mx;  // lane maximum, reused below
+    hit |= mx > s.m[hs] + kTau;
+  }
+  const bool any_hit = __any_sync(0xffffffffu, hit);
+  if (any_hit) {
+#pragma unroll
+    for (int hs = 0; hs < NHS; ++hs) {
+      float mx = alpha[hs];
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float mn = fmaxf(s.m[hs], mx);
+      alpha[hs] = mn > s.m[hs] ? ex2(s.m[hs] - mn) : 1.0f;
+      s.m[hs] = mn;
+    }
+  }
+  // ---- p*s enters the PV product scaled by 2^kacc: the largest weight of a slice sits below
+  // 2^14 and small weights stay in fp16's normal range; kacc only decreases, and only a
+  // position whose s reaches s_lim = 2^(14 - kTau - kacc) forces a (warp-wide) recomputation
+  bool over = false;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int u = 0; u < 2; ++u) over |= val[i][u] && vsz[i][u].x >= s.s_lim;
+  float fk = 1.0f;
+  if (__any_sync(0xffffffffu, over)) {
+    float smax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) smax = fmaxf(smax, val[i][u] ? vsz[i][u].x : 0.f);
+    smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
+    smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
+    smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
+    if (smax > 0.f) {
+      // p <= 2^kTau, so smax * 2^k < 2^(14 - kTau) keeps p*s*2^k below 2^14
+      const int k = 13 - kTau - (((__float_as_int(smax) >> 23) & 255) - 127);
+      if (k < s.kacc) {
+        fk = pow2i(max(k - s.kacc, -126));
+        s.kacc = k;
+        s.s_lim = pow2i(14 - kTau - k);
+      }
+    }
+  }
+  if (any_hit || fk != 1.0f) {
+    if (!any_hit) {
+#pragma unroll
+      for (int hs = 0; hs < NHS; ++hs) alpha[hs] = 1.0f;
+    }
+    // o columns are heads 2t4, 2t4+1 (lo parts in 4..7 when g <= 4); their alpha lives in
+    // lanes 4g + (head & 3)
+    float ac0 = __shfl_sync(0xffffffffu, alpha[0], 4 * g + ((2 * t4) & 3));
+    float ac1 = __shfl_sync(0xffffffffu, alpha[0], 4 * g + ((2 * t4 + 1) & 3));
+    if (NHS == 2) {
+      const float bc0 = __shfl_sync(0xffffffffu, alpha[NHS - 1], 4 * g + ((2 * t4) & 3));
+      const float bc1 = __shfl_sync(0xffffffffu, alpha[NHS - 1], 4 * g + ((2 * t4 + 1) & 3));
+      if (t4 >= 2) {
+        ac0 = bc0;
+        ac1 = bc1;
+      }
+    }
+    ac0 *= fk;
+    ac1 *= fk;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      s.o[mt][0] *= ac0;
+      s.o[mt][1] *= ac1;
+      s.o[mt][2] *= ac0;
+      s.o[mt][3] *= ac1;
+    }
+#pragma unroll
+    for (int hs = 0; hs < NHS; ++hs) {
+      s.l[hs] *= alpha[hs];
+      s.bias[hs] *= alpha[hs];
+    }
+  }
+  const float wscale = pow2i(s.kacc);
+
+  // ---- PV, one 16-position k-block per m-tile pair i
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    // p*s as an fp16 pair hi + lo (hi = fp16(p*s), lo = fp16(p*s - hi)): the PV product
+    // then carries ~22 bits of p*s, matching the fp32 l it is normalised by
+    uint32_t pk[NHS], pkl[NHS];
+#pragma unroll
+    for (int hs = 0; hs < NHS; ++hs) {
+      const float ms = s.m[hs] == -CUDART_INF_F ? 0.f : s.m[hs];
+      const float p0 = ex2(x[i][0][hs] - ms);
+      const float p1 = ex2(x[i][1][hs] - ms);
+      s.l[hs] += p0 + p1;
+      // masked positions may hold any bits in (s, z): never multiply them
+      const float w0 = val[i][0] ? p0 * vsz[i][0].x * wscale : 0.f;
+      const float w1 = val[i][1] ? p1 * vsz[i][1].x * wscale : 0.f;
+      const float b0 = val[i][0] ? p0 * vsz[i][0].y : 0.f;
+      const float b1 = val[i][1] ? p1 * vsz[i][1].y : 0.f;
+      s.bias[hs] += b0 + b1;
+      const __half2 hi2 = __floats2half2_rn(w0, w1);
+      const float2 hif = __half22float2(hi2);
+      pk[hs] = h2_as_u32(hi2);
+      pkl[hs] = h2_as_u32(__floats2half2_rn(w0 - hif.x, w1 - hif.y));
+    }
+    // B operand: rows k=2t4,2t4+1 <- positions t4, t4+8; k=2t4+8,+9 <- t4+4, t4+12 (of the
+    // block); column n = head n (n < 4 or g == 8); for g <= 4 columns 4..7 carry lo parts
+    const int src0 = 4 * t4 + (g & 3), src1 = 4 * (t4 + 4) + (g & 3);
+    uint32_t pb[2], pbl[2];
+    {
+      const uint32_t h0 = __shfl_sync(0xffffffffu, pk[0], src0);
+      const uint32_t h1 = __shfl_sync(0xffffffffu, pk[0], src1);
+      const uint32_t l0 = __shfl_sync(0xffffffffu, pkl[0], src0);
+      const uint32_t l1 = __shfl_sync(0xffffffffu, pkl[0], src1);
+      if (NHS == 2) {
+        const uint32_t h2 = __shfl_sync(0xffffffffu, pk[NHS - 1], src0);
+        const uint32_t h3 = __shfl_sync(0xffffffffu, pk[NHS - 1], src1);
+        const uint32_t l2 = __shfl_sync(0xffffffffu, pkl[NHS - 1], src0);
+        const uint32_t l3 = __shfl_sync(0xffffffffu, pkl[NHS - 1], src1);
+        pb[0] = g < 4 ? h0 : h2;
+        pb[1] = g < 4 ? h1 : h3;
+        pbl[0] = g < 4 ? l0 : l2;
+        pbl[1] = g < 4 ? l1 : l3;
+      } else {
+        pb[0] = g < 4 ? h0 : l0;
+        pb[1] = g < 4 ? h1 : l1;
+        pbl[0] = pbl[1] = 0u;
+      }
+    }
+    // the V codes of k-block i are one 16-position group in the value layout (vgroup_half):
+    // lane (g, t4) reads the words pairing positions (t4, t4 + 8) and (t4 + 4, t4 + 12) for
+    // its chunks -- four consecutive words, one 16-byte load, the warp's loads contiguous
+    const uint8_t* vgrp = vc + (size_t)(base + 16 * i) * CB;
+    if (BITS == 2) {
+      const uint4 vv = *reinterpret_cast<const uint4*>(vgrp + 64 * g + 16 * t4);
+      const uint32_t xl1 = vv.x, xl2 = vv.y, xh1 = vv.z, xh2 = vv.w;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const uint32_t A[4] = {vcode2(xl1, mt), vcode2(xh1, mt), vcode2(xl2, mt), vcode2(xh2, mt)};
+        mma_f16(s.o[mt], A, pb);
+        if (NHS == 2) mma_f16(s.o[mt], A, pbl);
+      }
+    } else {
+#pragma unroll
+      for (int ws = 0; ws < 2; ++ws) {
+        const uint4 vv = *reinterpret_cast<const uint4*>(vgrp + 512 * ws + 64 * g + 16 * t4);
+        const uint32_t xl1 = vv.x, xl2 = vv.y, xh1 = vv.z, xh2 = vv.w;
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi) {
+          const uint32_t A[4] = {vcode4(xl1, mi), vcode4(xh1, mi), vcode4(xl2, mi), vcode4(xh2, mi)};
+          mma_f16(s.o[4 * ws + mi], A, pb);
+          if (NHS == 2) mma_f16(s.o[4 * ws + mi], A, pbl);
+        }
+      }
+    }
+  }
 }
 
 // fp16 window positions [wbeg, wend) of a unit, positions wbeg + warp, + 4, ...: exact
@@ -473,30 +687,25 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 
 template <int BITS, int G>
 __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_kernel(const DecodeArgs a) {
-  using C = Cfg<BITS, G>;
+  using C = Cfg<BITS>;
   using SM = Shared<BITS, G>;
-  using W = WB<G>;
-  constexpr int NQ = GCfg<G>::NQ, NHS = GCfg<G>::NHS, LBO = GCfg<G>::LBO;
-  constexpr int CB = C::CB, NST = C::NSTAGE;
+  constexpr int NT = GCfg<G>::NT, NHS = GCfg<G>::NHS;
+  constexpr int CB = C::CB;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
   float* pv = reinterpret_cast<float*>(smem);  // [4][G][128], written once the stages are drained
-  uint8_t* wbuf = smem + SM::kArena;           // [4 warp pairs][2 buffers] PV weights
-  uint8_t* qop = wbuf + SM::kWbuf;             // the QK MMA's B operand (query limbs)
-  uint64_t* full = reinterpret_cast<uint64_t*>(qop + GCfg<G>::QBYTES);
-  uint64_t* empty = full + NST;
-  uint64_t* kready = empty + NST;              // [4] key operand of a stage in tensor memory
-  uint64_t* qkdone = kready + kQkBufs;         // [4] its QK product complete
-  uint64_t* wfull = qkdone + kQkBufs;          // [4][2] weights written by position warp w
-  uint64_t* wempty = wfull + 2 * kPosWarps;    // [4][2] ... consumed by value warp w
-  Merge* mg = reinterpret_cast<Merge*>(full + SM::kNumBars);
-  float* wpv = reinterpret_cast<float*>(mg + 1);                // window path [4][G][128]
-  float* wts = wpv + kConsumers * G * kHeadDim;                 // [nitems][G] (last item only)
-  __shared__ uint32_t s_last, s_taddr;
-  __shared__ int s_abort;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kArena);
+  uint64_t* empty = full + C::NSTAGE;
+  Merge* mg = reinterpret_cast<Merge*>(empty + C::NSTAGE);
+  float* wpv = reinterpret_cast<float*>(mg + 1);   // window path [4][G][128]
+  uint8_t* qfs = reinterpret_cast<uint8_t*>(wpv + kConsumers * G * kHeadDim);  // the unit's query fragments
+  float* wts = reinterpret_cast<float*>(qfs + kQFragBytes);  // [nitems][G] (last item only)
+  __shared__ uint32_t s_last;
+  __shared__ int s_abort;  // set by a bounded wait that gave up: every role leaves its loop
   volatile int* abort = &s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
   const int unit = blockIdx.y, item = blockIdx.x;
   const int nitems = a.n_split;
   int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
@@ -542,64 +751,41 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   const int wbeg = min(item * wper, n_win), wend = min(wbeg + wper, n_win);
 
   if (tid == 0) {
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kPosWarps + kValWarps);
-    }
-    for (int b = 0; b < kQkBufs; ++b) {
-      mbar_init(&kready[b], kPosWarps);
-      mbar_init(&qkdone[b], 1);
-    }
-    for (int i = 0; i < 2 * kPosWarps; ++i) {
-      mbar_init(&wfull[i], 1);
-      mbar_init(&wempty[i], 1);
+      mbar_init(&empty[s], kConsumers);
     }
     s_abort = 0;
     fence_mbar_init();
   }
-  for (int i = tid; i < SM::kWbuf / 16; i += kThreads) reinterpret_cast<uint4*>(wbuf)[i] = make_uint4(0, 0, 0, 0);
-  if (warp == kMmaWarp) tmem_alloc(&s_taddr, kTmemCols);
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tbase = s_taddr;
 
-  float o[8][4];  // value warps: the PV accumulators of their 32 positions per stage
+  QState<NHS> qs;
+  bool hvalid[NHS];
 #pragma unroll
-  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  for (int hs = 0; hs < NHS; ++hs) {
+    hvalid[hs] = (G % 4 == 0) || t4 + 4 * hs < G;
+    qs.m[hs] = -CUDART_INF_F;
+    qs.l[hs] = 0.f;
+    qs.bias[hs] = 0.f;
+  }
+  qs.kacc = 64;
+  qs.s_lim = 0.f;  // the first position with s > 0 sets kacc
 
-  if (warp == kProducerWarp) {
+  if (warp == kConsumers) {
     // ---------------- producer: streams the item's tiles; needs nothing from the prologue
-    if (lane == 0) {  // warm L2 with the item's fp16 window rows, read at the end of the item
-      const int s_end = min(wend, n_sink);
-      if (wbeg < s_end) {
-        const size_t row = (size_t)unit * a.sink_dim + wbeg;
-        bulk_prefetch_l2(a.k_sink + row * kHeadDim, (uint32_t)(s_end - wbeg) * kHeadDim * 2);
-        bulk_prefetch_l2(a.v_sink + row * kHeadDim, (uint32_t)(s_end - wbeg) * kHeadDim * 2);
-      }
-      const int rb = max(wbeg, n_sink);
-      if (rb < wend) {
-        const int cnt = wend - rb, slot0 = (r0 + (rb - n_sink)) % a.R;
-        const int first = min(cnt, a.R - slot0);
-        const size_t row = (size_t)unit * a.R;
-        bulk_prefetch_l2(a.k_ring + (row + slot0) * kHeadDim, (uint32_t)first * kHeadDim * 2);
-        bulk_prefetch_l2(a.v_ring + (row + slot0) * kHeadDim, (uint32_t)first * kHeadDim * 2);
-        if (cnt > first) {
-          bulk_prefetch_l2(a.k_ring + row * kHeadDim, (uint32_t)(cnt - first) * kHeadDim * 2);
-          bulk_prefetch_l2(a.v_ring + row * kHeadDim, (uint32_t)(cnt - first) * kHeadDim * 2);
-        }
-      }
-    }
     if (lane == 0 && ntiles > 0) {
       int issued = 0;
       bool waited = !a.fused;  // fused step: tiles below the old S_quant stream at once
       for (int t = 0; t < ntiles; ++t) {
-        const int s = t % NST;
+        const int s = t % C::NSTAGE;
         if (!waited && tile0 + (t + 1) * kTileTokens > sq_stable) {
           griddep_wait();
           waited = true;
         }
-        if (t >= NST && !mbar_wait_abortable(&empty[s], ((t / NST) - 1) & 1, a.status, abort, a.wait_limit)) break;
+        if (t >= C::NSTAGE &&
+            !mbar_wait_abortable(&empty[s], ((t / C::NSTAGE) - 1) & 1, a.status, abort, a.wait_limit))
+          break;
         if (*abort) break;
         if (t == a.withhold_tile) continue;  // test hook: this stage is never issued
         uint8_t* st = stages + s * C::STAGE;
@@ -613,337 +799,90 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
       }
       // every issued copy has landed before the CTA may leave (issued copies always land:
       // they are plain reads of the cache)
-      for (int t = max(0, issued - NST); t < issued; ++t)
-        if (t != a.withhold_tile) mbar_wait(&full[t % NST], (t / NST) & 1, a.status);
+      for (int t = max(0, issued - C::NSTAGE); t < issued; ++t)
+        if (t != a.withhold_tile) mbar_wait(&full[t % C::NSTAGE], (t / C::NSTAGE) & 1, a.status);
     }
-  } else if (warp == kMmaWarp) {
-    // ---------------- tensor-core issue: the query operand into shared memory, then one
-    // QK^T product per stage as soon as the position warps have stored its key operand
-    griddep_wait();  // the operand comes from the prologue (or the fused append)
-    const uint4* src = reinterpret_cast<const uint4*>(a.qfrag + (size_t)unit * kQFragBytes);
-    for (int i = lane; i < GCfg<G>::QBYTES / 16; i += 32) reinterpret_cast<uint4*>(qop)[i] = src[i];
-    fence_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8_u8s8(128, NQ);
-      const uint32_t qaddr = smem_u32(qop);
-      int last[kQkBufs] = {-1, -1, -1, -1};
-      for (int t = 0; t < ntiles; ++t) {
-        const int b = t % kQkBufs;
-        if (!mbar_wait_abortable(&kready[b], (t / kQkBufs) & 1, a.status, abort, a.wait_limit)) break;
-        tc_fence_after();
-        const uint32_t acol = tbase + 32 * b, dcol = tbase + 32 * kQkBufs + NQ * b;
+  } else {
+    // ---------------- consumers
+    // (a) this warp's share of the fp16 window: the first rows are loaded before the wait
+    // for the prologue (they do not depend on it), the rest while the first tiles land
+    WinRows<G> wr;
+    if (a.fused) griddep_wait();  // the window holds the appended tokens
+    window_load<G>(a, unit, wbeg + warp, wend, n_sink, r0, lane, wr);
+    griddep_wait();  // q', the query fragments and the counter resets come from the prologue
+    {  // the unit's query fragments into shared memory while the window share runs
+      constexpr int n16 = GCfg<G>::FW * 8 + 4;
+      const uint8_t* src = a.qfrag + (size_t)unit * kQFragBytes;
+      for (int i = tid; i < n16; i += kConsumers * 32) cp_async16(qfs + 16 * i, src + 16 * i);
+      cp_async_commit();
+    }
+    const int qlim = a.chunk_n > 0 ? S - a.chunk_n + a.chunk_t0 : INT_MAX;
+    window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, wr, mg, wpv, qlim);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_i8_ts(dcol, acol + 8 * kk, smem_desc(qaddr + 2 * kk * LBO, LBO, 128), idesc, kk > 0);
-        mma_commit(&qkdone[b]);
-        last[b] = t;
-      }
-      // no product may still be writing tensor memory when it is released
-      for (int b = 0; b < kQkBufs; ++b)
-        if (last[b] >= 0) mbar_wait(&qkdone[b], (last[b] / kQkBufs) & 1, a.status);
-    }
-  } else if (warp < kPosWarps) {
-    // ---------------- position warps: thread = position r of every stage
-    const int w = warp, r = kSlice * w + lane;
-    const uint32_t lrow = (uint32_t)(kSlice * w) << 16;  // this warp's tensor-memory lanes
-    griddep_wait();  // the per-head constants come from the prologue (or the fused append)
-    const float* hc = reinterpret_cast<const float*>(a.qfrag + (size_t)unit * kQFragBytes + GCfg<G>::QBYTES);
-    float Ah[G], Bh[G], mref[G], lsum[G], bsum[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      Ah[h] = hc[h];
-      Bh[h] = hc[8 + h];
-      mref[h] = -CUDART_INF_F;
-      lsum[h] = 0.f;
-      bsum[h] = 0.f;
-    }
-    int kacc = 64;
-    float s_lim = 0.f;  // the first position with s > 0 sets kacc
-    // Key operands go to tensor-memory buffer u % 4 (free: the product of stage u - 4 that
-    // read it, and wrote the result buffer stage u reuses, was complete and read before this
-    // warp got past stage u - 4).  The stores are asynchronous: those issued at the top of an
-    // iteration complete while the stage's softmax runs, and are handed to the MMA warp
-    // (wait, fence, arrive) only after it.
-    auto store_keys = [&](int u) {
-      store_key_operand<BITS>(stages + (u % NST) * C::STAGE, r, tbase + lrow + 32 * (u % kQkBufs));
-    };
-    auto commit_keys = [&](int u0, int u1) {  // stages [u0, u1) stored: release them to the MMA
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0)
-        for (int u = u0; u < u1; ++u) mbar_arrive(&kready[u % kQkBufs]);
-    };
-    uint32_t dn0[16], dn1[16];  // a stage's QK result, in flight from tensor memory
-    auto load_result = [&](int u) {
-      const uint32_t col = tbase + lrow + 32 * kQkBufs + NQ * (u % kQkBufs);
-      tmem_ld16(col, dn0);
-      if (NQ == 32) tmem_ld16(col + 16, dn1);
-    };
-    auto wait_result = [&]() {
-      tmem_wait_ld16(dn0);
-      if (NQ == 32) tmem_wait_ld16(dn1);
-    };
-    bool have_next = false;  // the result of the stage about to be processed is in flight
-    int staged = 0;  // key operands stored so far: stages [0, staged)
+    for (int mt = 0; mt < 8; ++mt) qs.o[mt][0] = qs.o[mt][1] = qs.o[mt][2] = qs.o[mt][3] = 0.f;
+    // (b) quantized positions
+    cp_async_wait_all();
+    bar_sync(1, kConsumers * 32);  // every consumer thread's copies have landed
+    uint32_t bq[4][NT][2];
+    float Ah[NHS], Bh[NHS];
+    load_query<G>(qfs, lane, t4, bq, Ah, Bh);
+    const int base = kSlice * warp;
     for (int t = 0; t < ntiles; ++t) {
-      const int slot = t % NST, b = t & 1;
-      const uint8_t* st = stages + slot * C::STAGE;
-      if (staged == t) {  // starved: this stage's operand is needed now
-        if (!warp_wait(&full[slot], (t / NST) & 1, a, abort)) break;
-        store_keys(t);
-        commit_keys(t, t + 1);
-        staged = t + 1;
-      }
-      // the operands of the next stages whose data has landed, up to 3 ahead (never waits)
-      const int s0 = staged;
-      while (staged < ntiles && staged <= t + kQkBufs - 1 &&
-             __all_sync(0xffffffffu, mbar_test_wait(&full[staged % NST], (staged / NST) & 1))) {
-        store_keys(staged);
-        ++staged;
-      }
-      // this stage's QK result: loaded ahead during the previous stage when it was ready
-      if (!have_next) {
-        if (!warp_wait(&qkdone[t % kQkBufs], (t / kQkBufs) & 1, a, abort)) break;
-        tc_fence_after();
-        load_result(t);
-      }
-      wait_result();
-      uint32_t dq[NQ];
-#pragma unroll
-      for (int c = 0; c < 16; ++c) dq[c] = dn0[c];
-      if (NQ == 32) {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) dq[(16 + c) % NQ] = dn1[c];
-      }
-      // the next stage's result, if its product is complete, loads while this one's
-      // softmax runs (its key operand was handed over in an earlier iteration)
-      have_next = t + 1 < ntiles && t + 1 < s0 &&
-                  __all_sync(0xffffffffu, mbar_test_wait(&qkdone[(t + 1) % kQkBufs], ((t + 1) / kQkBufs) & 1));
-      if (have_next) {
-        tc_fence_after();
-        load_result(t + 1);
-      }
-      // ---- logits (base 2) of this thread's position, one per head
-      const int pos = tile0 + t * kTileTokens + r;
-      const bool val = pos >= lo && pos < hi;
-      const uint32_t* kpar = reinterpret_cast<const uint32_t*>(st + 2 * kTileTokens * CB);
-      const float2 ksz = __half22float2(u32_as_h2(kpar[r]));
-      const float2 vsz = __half22float2(u32_as_h2(kpar[kTileTokens + r]));
-      float x[G], fac[G];
-      bool hit = false;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        // q'.c / sigma = sum_l 256^l D_l; pairs of limbs combine exactly in int32
-        const int d01 = (int)dq[4 * h] + 256 * (int)dq[4 * h + 1];
-        const int d23 = (int)dq[4 * h + 2] + 256 * (int)dq[4 * h + 3];
-        const float f = fmaf(65536.0f, (float)d23, (float)d01);
-        x[h] = val ? fmaf(Bh[h] * ksz.x, f, Ah[h] * ksz.y) : -CUDART_INF_F;
-        hit |= x[h] > mref[h] + kTau;
-        fac[h] = 1.0f;
-      }
-      // The running max is kept stale: p = 2^(x - mref) may reach 2^kTau, and only a logit
-      // above mref + kTau (a warp vote) triggers the rescale.
-      bool post = false;
-      if (__any_sync(0xffffffffu, hit)) {
-        post = true;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float mx = x[h];
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-          const float mn = fmaxf(mref[h], mx);
-          const float al = mn > mref[h] ? ex2(mref[h] - mn) : 1.0f;
-          mref[h] = mn;
-          lsum[h] *= al;
-          bsum[h] *= al;
-          fac[h] = al;
-        }
-      }
-      // p*s enters the PV product scaled by 2^kacc: the largest weight sits below 2^14 and
-      // small weights stay in fp16's normal range; kacc only decreases, and only a position
-      // whose s reaches s_lim = 2^(14 - kTau - kacc) forces a (warp-wide) recomputation.
-      // Positions outside the item may hold any bits in (s, z): never use them.
-      if (__any_sync(0xffffffffu, val && vsz.x >= s_lim)) {
-        float smax = val ? vsz.x : 0.f;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
-        if (smax > 0.f) {
-          const int k = 13 - kTau - (((__float_as_int(smax) >> 23) & 255) - 127);
-          if (k < kacc) {
-            const float fk = pow2i(max(k - kacc, -126));
-#pragma unroll
-            for (int h = 0; h < G; ++h) fac[h] *= fk;
-            kacc = k;
-            s_lim = pow2i(14 - kTau - k);
-            post = true;
-          }
-        }
-      }
-      const float wscale = pow2i(kacc);
-      // ---- PV weights for the value warp: its buffer b was read by the stage t - 2
-      if (t >= 2 && !warp_wait(&wempty[2 * w + b], ((t >> 1) - 1) & 1, a, abort)) break;
-      uint8_t* wb = wbuf + (2 * w + b) * W::BYTES;
-      const int rr = lane & 15;
-      uint8_t* wcol = wb + (lane >> 4) * W::KB + (2 * (rr & 3) + ((rr >> 2) & 1)) * 4 + (rr >> 3) * 2;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float ms = mref[h] == -CUDART_INF_F ? 0.f : mref[h];
-        const float p = ex2(x[h] - ms);
-        lsum[h] += p;
-        const float wv = val ? p * vsz.x * wscale : 0.f;
-        bsum[h] += val ? p * vsz.y : 0.f;
-        // p*s as an fp16 pair hi + lo: the PV product then carries ~22 bits of p*s,
-        // matching the fp32 l it is normalised by
-        const __half whi = __float2half_rn(wv);
-        const __half wlo = __float2half_rn(wv - __half2float(whi));
-        *reinterpret_cast<__half*>(wcol + h * 32) = whi;
-        *reinterpret_cast<__half*>(wcol + (h + W::NC / 2) * 32) = wlo;
-      }
-      if (lane == 0) {
-        int* hdr = reinterpret_cast<int*>(wb + W::HDR);
-        hdr[0] = post ? 1 : 0;
-        hdr[1] = kacc;
-        if (post) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) reinterpret_cast<float*>(hdr)[2 + h] = fac[h];
-        }
-      }
+      const int s = t % C::NSTAGE;
+      if (!warp_wait(&full[s], (t / C::NSTAGE) & 1, a, abort)) break;
+      const uint8_t* st = stages + s * C::STAGE;
+      const int tpos = tile0 + t * kTileTokens;
+      if (tpos + base >= lo && tpos + base + kSlice <= hi)
+        slice<BITS, G, true>(st, base, tpos, lo, hi, bq, Ah, Bh, hvalid, qs, g, t4);
+      else if (tpos + base + kSlice > lo && tpos + base < hi)
+        slice<BITS, G, false>(st, base, tpos, lo, hi, bq, Ah, Bh, hvalid, qs, g, t4);
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&wfull[2 * w + b]);
-        mbar_arrive(&empty[slot]);  // this warp is done with the stage's key codes and (s, z)
-      }
-      if (staged > s0) commit_keys(s0, staged);
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
-    // l and bias summed over the warp's positions
+    // l and bias summed over the 8 lane groups
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float lv = lsum[h], bv = bsum[h];
+    for (int hs = 0; hs < NHS; ++hs) {
+      float lv = qs.l[hs], bv = qs.bias[hs];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
+      for (int off = 4; off < 32; off <<= 1) {
         lv += __shfl_xor_sync(0xffffffffu, lv, off);
         bv += __shfl_xor_sync(0xffffffffu, bv, off);
       }
-      if (lane == 0) {
-        mg->m[w][h] = mref[h];
-        mg->l[w][h] = lv;
-        mg->bias[w][h] = bv;
-      }
-    }
-  } else {
-    // ---------------- value warps: the fp16 window share, then PV of the paired positions
-    const int w = warp - kPosWarps;
-    const int g = lane >> 2, t4 = lane & 3;
-    griddep_wait();  // the window holds the appended tokens; q' comes from the prologue
-    int kacc = 64;   // the weight scale of the stages seen (the position warp's, via the header)
-    for (int t = 0; t < ntiles; ++t) {
-      const int slot = t % NST, b = t & 1;
-      if (!warp_wait(&full[slot], (t / NST) & 1, a, abort)) break;
-      if (!warp_wait(&wfull[2 * w + b], (t >> 1) & 1, a, abort)) break;
-      const uint8_t* wb = wbuf + (2 * w + b) * W::BYTES;
-      const int* hdr = reinterpret_cast<const int*>(wb + W::HDR);
-      kacc = hdr[1];
-      if (hdr[0]) {  // the running max or the weight scale moved: rescale first
-        const float* fac = reinterpret_cast<const float*>(hdr) + 2;
-        // o columns are heads 2t4, 2t4+1 (G <= 4: lo parts in columns 4..7)
-        const float c0 = fac[NHS == 1 ? (2 * t4) & 3 : 2 * t4];
-        const float c1 = fac[NHS == 1 ? (2 * t4 + 1) & 3 : 2 * t4 + 1];
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          o[mt][0] *= c0;
-          o[mt][1] *= c1;
-          o[mt][2] *= c0;
-          o[mt][3] *= c1;
-        }
-      }
-      const uint8_t* vc = stages + slot * C::STAGE + kTileTokens * CB;
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        // B operand: rows k=2t4,2t4+1 <- positions t4, t4+8; k=2t4+8,+9 <- t4+4, t4+12 (of
-        // the block); column n = the lane group g
-        const uint2 bw = *reinterpret_cast<const uint2*>(wb + i * W::KB + g * 32 + t4 * 8);
-        const uint32_t pb[2] = {bw.x, bw.y};
-        uint32_t pbl[2] = {0u, 0u};
-        if (NHS == 2) {
-          const uint2 bl = *reinterpret_cast<const uint2*>(wb + i * W::KB + (8 + g) * 32 + t4 * 8);
-          pbl[0] = bl.x;
-          pbl[1] = bl.y;
-        }
-        // the V codes of k-block i are one 16-position group in the value layout (vgroup_half):
-        // lane (g, t4) reads the words pairing positions (t4, t4 + 8) and (t4 + 4, t4 + 12) for
-        // its chunks -- four consecutive words, one 16-byte load, the warp's loads contiguous
-        const uint8_t* vgrp = vc + (size_t)(kSlice * w + 16 * i) * CB;
-        if (BITS == 2) {
-          const uint4 vv = *reinterpret_cast<const uint4*>(vgrp + 64 * g + 16 * t4);
-          const uint32_t xl1 = vv.x, xl2 = vv.y, xh1 = vv.z, xh2 = vv.w;
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            const uint32_t A[4] = {vcode2(xl1, mt), vcode2(xh1, mt), vcode2(xl2, mt), vcode2(xh2, mt)};
-            mma_f16(o[mt], A, pb);
-            if (NHS == 2) mma_f16(o[mt], A, pbl);
-          }
-        } else {
-#pragma unroll
-          for (int ws = 0; ws < 2; ++ws) {
-            const uint4 vv = *reinterpret_cast<const uint4*>(vgrp + 512 * ws + 64 * g + 16 * t4);
-            const uint32_t xl1 = vv.x, xl2 = vv.y, xh1 = vv.z, xh2 = vv.w;
-#pragma unroll
-            for (int mi = 0; mi < 4; ++mi) {
-              const uint32_t A[4] = {vcode4(xl1, mi), vcode4(xh1, mi), vcode4(xl2, mi), vcode4(xh2, mi)};
-              mma_f16(o[4 * ws + mi], A, pb);
-              if (NHS == 2) mma_f16(o[4 * ws + mi], A, pbl);
-            }
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&wempty[2 * w + b]);
-        mbar_arrive(&empty[slot]);
+      if (g == 0 && hvalid[hs]) {
+        mg->m[warp][t4 + 4 * hs] = qs.m[hs];
+        mg->l[warp][t4 + 4 * hs] = lv;
+        mg->bias[warp][t4 + 4 * hs] = bv;
       }
     }
     if (NHS == 1) {  // columns 4..7 (lanes t4 = 2, 3) hold the lo parts of heads 0..3
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) o[mt][c] += __shfl_down_sync(0xffffffffu, o[mt][c], 2);
+        for (int c = 0; c < 4; ++c) qs.o[mt][c] += __shfl_down_sync(0xffffffffu, qs.o[mt][c], 2);
     }
-    // every value warp is done with the stages (and every copy has landed: all were
-    // consumed), so the accumulators may go to the stage arena
-    bar_sync(1, kValWarps * 32);
+  }
+  __syncthreads();  // every stage consumed and every copy landed: pv may reuse the stages
+  // a bounded wait gave up (STATUS_TIMEOUT is set): this item's results are incomplete, so
+  // it writes no partial and takes no part in the merge -- the unit's output is not written
+  if (s_abort) return;
+
+  if (warp < kConsumers) {
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
 #pragma unroll
       for (int hi2 = 0; hi2 < 2; ++hi2) {
         int dim, l2s;
         value_row<BITS>(mt, g, hi2, dim, l2s);
-        const float unscale = pow2i(24 - l2s - kacc);
+        const float unscale = pow2i(24 - l2s - qs.kacc);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int hh = 2 * t4 + c;
-          if (hh < G) pv[((size_t)w * G + hh) * kHeadDim + dim] = o[mt][2 * hi2 + c] * unscale;
+          if (hh < G) pv[((size_t)warp * G + hh) * kHeadDim + dim] = qs.o[mt][2 * hi2 + c] * unscale;
         }
       }
     }
-    // the item's share of the fp16 window comes after the stages (its rows were warmed in L2
-    // at the start), so that it never holds up the stage ring
-    WinRows<G> wr;
-    window_load<G>(a, unit, wbeg + w, wend, n_sink, r0, lane, wr);
-    const int qlim = a.chunk_n > 0 ? S - a.chunk_n + a.chunk_t0 : INT_MAX;
-    window_share<G>(a, unit, wbeg, wend, n_sink, r0, w, lane, wr, mg, wpv, qlim);
   }
-  tc_fence_before();
-  __syncthreads();  // every stage consumed, every copy landed, every product complete
-  if (warp == kMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tbase, kTmemCols);
-  }
-  // a bounded wait gave up (STATUS_TIMEOUT is set): this item's results are incomplete, so
-  // it writes no partial and takes no part in the merge -- the unit's output is not written
-  if (s_abort) return;
-
+  __syncthreads();
 
   // ======================= merge the 8 pseudo-warps, write this item's partial: the
   // weights once per (pseudo-warp, head), then the rows

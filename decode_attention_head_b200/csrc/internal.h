@@ -13,8 +13,8 @@ constexpr int kHeadDim = 128;
 constexpr int kTileTokens = 128;      // positions per decode pipeline stage (and cap_alloc granule)
 constexpr int kB200SMs = 148;         // split policy sizes the decode grid for this many SMs
 // Resident decode CTAs per SM the split policy aims at (the kernel's launch bounds hold its
-// registers to this; each CTA holds 128 of the SM's 512 tensor-memory columns).
-constexpr int decode_ctas_per_sm(int group) { return group > 0 ? 2 : 2; }
+// registers to this): 8 query heads per KV head need more registers than the others.
+constexpr int decode_ctas_per_sm(int group) { return group == 8 ? 3 : 4; }
 constexpr int kMaxSplits = 255;       // quantized work items per (sequence, KV head)
 constexpr int kMergeGroup = 16;       // work items merged together at the first merge level
 
