@@ -860,7 +860,7 @@ def measure_gram(bnd, synth, dev, n_seq=4, seq_len=32768, reps=10):
     tokens = n_seq * seq_len
     nbytes = tokens * H * 128 * 2 + H * 128 * 128 * 8 * 2
     peak, peak_kind = measured_peaks()
-    mma_flops = 2 * tokens * H * 10 * 32 * 32  # the 10 blocks of 32 x 32 on and above the diagonal
+    mma_flops = 2 * tokens * H * 128 * 128  # the tensor cores form the whole 128 x 128 tile
     return {"workload": "qwen3-8b calibration keys", "sequences": n_seq, "tokens_per_sequence": seq_len,
             "kv_heads": H, "us": round(t * 1e6, 2), "gbs": round(nbytes / t / 1e9, 2),
             "frac_hbm": round(nbytes / t / 1e9 / peak, 4), "peak_kind": peak_kind,

@@ -6,22 +6,26 @@
 // and value Gram matrices, per KV head).
 //
 // gram[h] += sum_t x[t][h] x[t][h]^T is a dense contraction over tokens (128 x n x 128 per
-// head), run on the tensor cores: mma.sync m16n8k16 with fp16 operands and fp32
-// accumulation (a product of two fp16 values is exact in fp32).
+// head), run on the fifth-generation tensor cores: tcgen05.mma kind::f16, M = N = 128
+// dimensions, K = 16 tokens per instruction, fp16 operands, the whole 128 x 128 fp32 sum in
+// tensor memory (128 lanes x 128 columns).  A product of two fp16 values is exact in fp32.
+//
+// Both operands are the same shared-memory tile: with tokens as the K mode and dimensions
+// as the M (or N) mode, a token's row of 128 dimensions is an MN-major operand row, so no
+// transposition is needed.  The tile is stored in the canonical MN-major 128-byte-swizzled
+// layout: dimensions 0..63 and 64..127 in two regions of [tokens][128 bytes], the 16-byte
+// chunk c of token t at chunk c ^ (t % 8) of its row.  One descriptor serves as A and as B.
 //
 // Work split.  A CTA takes a run of at most kGramTokens consecutive tokens of one head; the
 // run length is chosen so that the grid fills two CTAs per SM when the input allows.  The
-// tokens arrive 64 at a time through a cp.async ring of kGramStages slots, stored as they
-// are in memory (one 256-byte row per token, padded to 272 bytes so that ldmatrix reads
-// are conflict-free).  ldmatrix.trans turns 16 tokens x 16 dimensions into the four words
-// that are at once the A fragment of that dimension block and the B fragments of its two
-// n-tiles.  M is symmetric, so only the 10 blocks of 32 x 32 on and above the diagonal are
-// computed (of 16): each of 5 warps takes two blocks that share their row block, and two
-// such groups of 5 warps take alternate halves of every stage's k-steps.  At the end the
-// two groups add their sums through shared memory, and the CTA adds its fp32 sums into the
-// fp64 Gram matrix with atomics, an off-diagonal block at both (i, j) and (j, i).  A CTA's
-// fp32 sum covers at most kGramTokens tokens, which bounds its rounding error; the fp64
-// additions across CTAs come in no fixed order.
+// tokens arrive 64 at a time through a cp.async ring of kGramStages slots (the rows of one
+// head are n_heads * 256 bytes apart in memory).  One thread issues the four MMAs of a
+// slot and commits them to the slot's mbarrier; the slot is refilled only once they have
+// read it.  At the end the four warps read the sum back from tensor memory (warp w: rows
+// 32 w .. 32 w + 31) and add it into the fp64 Gram matrix with atomics: the entry (i, j),
+// i <= j, at both (i, j) and (j, i), so the result stays exactly symmetric.  A CTA's fp32
+// sum covers at most kGramTokens tokens, which bounds its rounding error; the fp64 additions
+// across CTAs come in no fixed order.
 #include <algorithm>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -33,61 +37,89 @@
 namespace wushkv {
 namespace {
 
-constexpr int kGramGroupWarps = 5;                    // one warp per pair of 32 x 32 blocks
-constexpr int kGramGroupThreads = 32 * kGramGroupWarps;
-constexpr int kGramThreads = 2 * kGramGroupThreads;   // two groups: k-steps {0, 1} and {2, 3} of a stage
-constexpr int kGramStage = 64;                        // tokens per stage
-constexpr int kGramStages = 3;                        // cp.async ring slots
-constexpr int kGramRowBytes = 272;                    // one token's 256 bytes + 16 bytes of padding
-constexpr int kGramSlotBytes = kGramStage * kGramRowBytes;
-constexpr int kGramSmem = kGramStages * kGramSlotBytes;
-static_assert(2 * 32 * kGramGroupThreads * 4 <= kGramSmem, "the group exchange reuses the ring");
+constexpr int kGramThreads = 128;                 // four warps: copies, MMA issue, read-back
+constexpr int kGramStage = 64;                    // tokens per stage (four MMAs of K = 16)
+constexpr int kGramStages = 4;                    // ring slots
+constexpr int kGramRegion = kGramStage * 128;     // bytes of one 64-dimension half of a slot
+constexpr int kGramSlotBytes = 2 * kGramRegion;   // 16 KB
+constexpr int kGramSmem = kGramStages * kGramSlotBytes + 1024;  // + room to align to 1024
+constexpr uint32_t kGramTmemCols = 128;
 
-// Nibble w of a table: the 32-dimension blocks of warp w of a group.  Row block, first and
-// second column block: (0; 0, 1) (0; 2, 3) (1; 1, 2) (3; 1, 3) (2; 2, 3) -- each of the 10
-// unordered pairs {i, j} once.
-constexpr uint32_t kRowBlock = 0x23100u, kColBlock0 = 0x21120u, kColBlock1 = 0x33231u;
-__device__ __forceinline__ int nibble(uint32_t table, int w) { return (table >> (4 * w)) & 15; }
+// kind::f16 with an fp32 accumulator, A and B fp16 and MN-major, M = N = 128.
+constexpr uint32_t kGramIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 15) | (1u << 16) |
+                                ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 
-// Four transposed 8 x 8 fp16 matrices: lanes 8m .. 8m + 7 give the row addresses of matrix m,
-// and lane (g, t4) receives rows 2 t4, 2 t4 + 1 of column g of each.
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
+// D (tensor memory) [+]= A x B with both operands from shared memory; one thread.
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// MN-major, 128-byte-swizzle descriptor of 16 tokens starting at `saddr` (1024-byte aligned):
+// 8-token groups 1024 bytes apart, the two 64-dimension regions kGramRegion bytes apart.
+__device__ __forceinline__ uint64_t gram_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((kGramRegion >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((1024 >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-__global__ void __launch_bounds__(kGramThreads, 2)
+// 32 consecutive columns of this thread's tensor-memory lane, waited for inside the same
+// statement (so that no use of r can be scheduled before the data is there).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kGramThreads)
     gram_kernel(const uint16_t* __restrict__ x, int64_t n_tokens, int n_heads, int64_t cta_tokens,
                 double* __restrict__ gram) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
-  const int grp = warp / kGramGroupWarps, wg = warp % kGramGroupWarps;
+  extern __shared__ uint8_t smem_raw[];
+  // the swizzle pattern repeats every 1024 bytes: slots start on such a boundary
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t done[kGramStages];  // the MMAs that read a slot have completed
+  __shared__ uint32_t s_taddr;
+  __shared__ uint32_t s_status;  // the Gram call has no status word: a wait that gives up (a library bug) lands here
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;
   const int64_t t_begin = (int64_t)blockIdx.x * cta_tokens;
   const int64_t t_end = min(n_tokens, t_begin + cta_tokens);
   const int n_stages = (int)((t_end - t_begin + kGramStage - 1) / kGramStage);
-  const int bi = nibble(kRowBlock, wg);
-  const int bj0 = nibble(kColBlock0, wg), bj1 = nibble(kColBlock1, wg);
-  const uint32_t smem0 = smem_u32(smem);
 
-  // Stage s (tokens t_begin + 64 s ...) into ring slot s % kGramStages: 16-byte copies, one
-  // token row per 16 threads.  Rows past the run are zero-filled, so they add nothing.  One
-  // commit group per call, empty past the last stage.
-  auto issue_stage = [&](int s) {
-    if (s < n_stages) {
-      uint8_t* slot = smem + (s % kGramStages) * kGramSlotBytes;
-      const int64_t t0 = t_begin + (int64_t)s * kGramStage;
+  if (tid == 0) {
+    for (int s = 0; s < kGramStages; ++s) mbar_init(&done[s], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&s_taddr, kGramTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = s_taddr;
+
+  // Stage u (tokens t_begin + 64 u ...) into slot u % kGramStages, once the MMAs of stage
+  // u - kGramStages (the slot's previous user) have read it: 16-byte copies in the swizzled
+  // MN-major layout.  Rows past the run are zero-filled, so they add nothing.  One commit
+  // group per call, empty past the last stage.
+  auto issue_stage = [&](int u) {
+    if (u < n_stages) {
+      const int slot = u % kGramStages;
+      if (u >= kGramStages) mbar_wait(&done[slot], ((u / kGramStages) - 1) & 1, &s_status);
+      uint8_t* base = smem + slot * kGramSlotBytes;
+      const int64_t t0 = t_begin + (int64_t)u * kGramStage;
       for (int i = tid; i < kGramStage * 16; i += kGramThreads) {
         const int r = i >> 4, c = i & 15;
         const int64_t t = t0 + r;
-        uint8_t* dst = slot + r * kGramRowBytes + 16 * c;
+        uint8_t* dst = base + (c >> 3) * kGramRegion + r * 128 + (((c & 7) ^ (r & 7)) << 4);
         if (t < t_end)
           cp_async16(dst, x + (t * n_heads + h) * kHeadDim + 8 * c);
         else
@@ -97,92 +129,50 @@ __global__ void __launch_bounds__(kGramThreads, 2)
     cp_async_commit();
   };
 
-  float acc[2][2][4][4];  // [column block][m-tile][n-tile][C fragment]
-#pragma unroll
-  for (int s = 0; s < 2; ++s)
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[s][mt][nt][i] = 0.f;
-
-#pragma unroll
-  for (int s = 0; s < kGramStages - 1; ++s) issue_stage(s);
-
-  // ldmatrix row address of this lane within a slot: token 16 ks + (lane & 7) + 8 (lane >> 4),
-  // dimensions + 8 ((lane >> 3) & 1): matrices 0..3 are (tokens +0, dims +0), (+0, +8),
-  // (+8, +0), (+8, +8) of a 16 x 16 block, i.e. fragment words f[0] .. f[3].
-  const uint32_t lane_off = ((lane & 7) + 8 * (lane >> 4)) * kGramRowBytes + 16 * ((lane >> 3) & 1);
+  // two stages of copies ahead of the MMAs; a slot is refilled two stages after its MMAs
+  // were issued, so their completion is rarely waited for
+  for (int u = 0; u < kGramStages - 2; ++u) issue_stage(u);
+  const uint32_t smem0 = smem_u32(smem);
   for (int s = 0; s < n_stages; ++s) {
-    cp_async_wait_group<kGramStages - 2>();  // this thread's copies of stage s have landed
-    __syncthreads();                          // everyone's have; everyone is done with stage s - 1
-    issue_stage(s + kGramStages - 1);         // into the slot stage s - 1 used
-    const uint32_t slot = smem0 + (s % kGramStages) * kGramSlotBytes + lane_off;
+    issue_stage(s + kGramStages - 2);
+    asm volatile("cp.async.wait_group %0;" ::"n"(kGramStages - 2) : "memory");  // stage s landed (this thread)
+    fence_async_smem();  // ... and is visible to the tensor core
+    __syncthreads();     // every thread's copies of stage s are in
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t slot = smem0 + (s % kGramStages) * kGramSlotBytes;
 #pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-      const uint32_t rows = slot + (16 * (2 * grp + kk)) * kGramRowBytes;
-      uint32_t fa[2][4];
-      ldsm_x4_trans(fa[0], rows + 32 * (2 * bi));
-      ldsm_x4_trans(fa[1], rows + 32 * (2 * bi + 1));
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
-        const int bj = cb ? bj1 : bj0;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t fb[4];
-          ldsm_x4_trans(fb, rows + 32 * (2 * bj + half));
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int n2 = 0; n2 < 2; ++n2) {
-              const uint32_t b[2] = {fb[n2], fb[n2 + 2]};
-              mma_f16(acc[cb][mt][2 * half + n2], fa[mt], b);
-            }
-        }
+      for (int j = 0; j < kGramStage / 16; ++j) {
+        const uint64_t d = gram_desc(slot + j * 16 * 128);
+        mma_f16_ss(tbase, d, d, kGramIdesc, (s > 0 || j > 0) ? 1u : 0u);
       }
+      mma_commit(&done[s % kGramStages]);
     }
   }
-
-  // The two groups add their sums: group 0 finishes column block 0, group 1 column block 1.
-  cp_async_wait_group<0>();
-  __syncthreads();  // the ring is free
-  float* xch = reinterpret_cast<float*>(smem);  // [2][32][kGramGroupThreads]: block handed over
-  const int gt = tid % kGramGroupThreads;
-  auto put = [&](const float (&a)[2][4][4], int which) {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) xch[(which * 32 + e) * kGramGroupThreads + gt] = a[e >> 4][(e >> 2) & 3][e & 3];
-  };
-  auto take = [&](float (&a)[2][4][4], int which) {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) a[e >> 4][(e >> 2) & 3][e & 3] += xch[(which * 32 + e) * kGramGroupThreads + gt];
-  };
-  if (grp == 0)
-    put(acc[1], 1);
-  else
-    put(acc[0], 0);
-  __syncthreads();
+  // every MMA complete (the last commit covers all of them), then the sum leaves tensor memory
+  mbar_wait(&done[(n_stages - 1) % kGramStages], ((n_stages - 1) / kGramStages) & 1, &s_status);
+  tc_fence_after();
   double* G = gram + (size_t)h * kHeadDim * kHeadDim;
-  auto flush = [&](const float (&a)[2][4][4], int bj) {
+  const int i = 32 * warp + lane;  // this thread's row (tensor-memory lane)
+#pragma unroll 1
+  for (int c = 0; c < kHeadDim / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tbase + ((uint32_t)(32 * warp) << 16) + 32 * c, r);
+    if (32 * c + 31 < i) continue;  // only j >= i: the (j, i) entry gets the same value
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int row = 32 * bi + 16 * mt + g + 8 * (i >> 1);
-          const int col = 32 * bj + 8 * nt + 2 * t4 + (i & 1);
-          const double v = a[mt][nt][i];
-          atomicAdd(G + row * kHeadDim + col, v);
-          if (bi != bj) atomicAdd(G + col * kHeadDim + row, v);
-        }
-  };
-  if (grp == 0) {
-    take(acc[0], 0);
-    flush(acc[0], bj0);
-  } else {
-    take(acc[1], 1);
-    flush(acc[1], bj1);
+    for (int k = 0; k < 32; ++k) {
+      const int j = 32 * c + k;
+      if (j < i) continue;
+      const double v = (double)__uint_as_float(r[k]);
+      atomicAdd(G + i * kHeadDim + j, v);
+      if (j != i) atomicAdd(G + j * kHeadDim + i, v);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kGramTmemCols);
   }
 }
 

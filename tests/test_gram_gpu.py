@@ -1,13 +1,13 @@
 """Calibration Gram matrices on the GPU (wushkv_gram_accumulate) against the oracle's
 float64 sums, through the C ABI.
 
-Tolerance, from the arithmetic.  A CTA sums at most 4096 tokens of one head with mma.sync
-m16n8k16; a product of two fp16 values is exact in fp32.  Each MMA adds 16 products to
+Tolerance, from the arithmetic.  A CTA sums at most 4096 tokens of one head on the tensor
+cores (tcgen05.mma kind::f16, K = 16 tokens per instruction, fp32 accumulator in tensor
+memory); a product of two fp16 values is exact in fp32.  Each MMA adds 16 products to
 its fp32 accumulator C.  Aligning the 17 addends to the largest loses at most one fp32 ulp
 of it per addend, so one MMA errs by at most 17 * 2^-23 * (|C| + sum |a b|) <= 17 * 2^-23 * A,
 with A = sum_t |x_ti| |x_tj| over the CTA's tokens.  Over ceil(T / 16) MMAs that gives
-ceil(T / 16) * 17 * 2^-23 * A.  The kernel splits a CTA's k-steps between two
-accumulators and adds them once at the end, which stays inside this bound.  The fp64
+ceil(T / 16) * 17 * 2^-23 * A.  The fp64
 atomics add a few 2^-53 A more.
 Integer-valued inputs whose partial sums stay below 2^24 are summed exactly, so those
 cases are compared bit for bit: they pin every index of the tiling."""
