@@ -102,6 +102,46 @@ __device__ __forceinline__ uint32_t quantize_one(float v, float zf, float sf, fl
   return static_cast<uint32_t>(c);
 }
 
+// The smallest fp16 x whose code under (s, z) is at least k (1 <= k <= 2^bits - 1), so that
+// code(x) = #{k : x >= X_k}.  code(x) = clamp(rint_even(fl32(fl32(x - z) / s))) is a
+// non-decreasing function of x, so these thresholds give exactly the codes of the reading.
+//  * In t = fl32(x - z): code >= k iff t >= T_k, with T_k = (k - 1/2) s when k is even (the
+//    quotient k - 1/2 is exact and ties round to the even k) and the next fp32 value above
+//    it when k is odd.  (k - 1/2) s is exact in fp32 (at most 16 significant bits).
+//  * In x: fl32(x - z) >= T_k iff the exact x - z reaches the midpoint between T_k and the
+//    fp32 value below it (reaching it exactly counts when T_k's last mantissa bit is even:
+//    the tie rounds to T_k).  x - z is exact in double for fp16 x and z, so the nearest fp16
+//    value to z + mid is checked there and moved by one fp16 step at most.
+// Both facts were checked exhaustively on the CPU (every positive fp16 scale for T_k, every
+// fp16 z against 400 scales and every k <= 15 for X_k).  Returns +inf when no finite x
+// reaches code k.
+__device__ __forceinline__ __half h_step(__half x, int d) {  // the next fp16 value up (d = 1) or down (-1)
+  const int b = __half_as_ushort(x);
+  int key = b >= 0x8000 ? 0xFFFF - b : b + 0x8000;  // fp16 order as an integer order (-0 just below +0)
+  key = min(max(key + d, 0), 0xFFFF);
+  return __ushort_as_half((unsigned short)(key >= 0x8000 ? key - 0x8000 : 0xFFFF - key));
+}
+
+__device__ __forceinline__ __half code_threshold(int k, float sf, float zf) {
+  const float e = __fmul_rn((float)k - 0.5f, sf);
+  const float T = (k & 1) ? __uint_as_float(__float_as_uint(e) + 1u) : e;
+  const double mid = 0.5 * ((double)T + (double)__uint_as_float(__float_as_uint(T) - 1u));
+  const bool incl = (__float_as_uint(T) & 1u) == 0u;
+  const double zd = (double)zf;
+  auto reach = [&](__half x) {
+    const double y = (double)__half2float(x) - zd;
+    return incl ? y >= mid : y > mid;
+  };
+  __half v = __double2half(zd + mid);
+  if (reach(v)) {
+    const __half p = h_step(v, -1);
+    if (reach(p)) v = p;
+  } else {
+    v = h_step(v, 1);
+  }
+  return v;
+}
+
 // Value codes are stored in groups of 16 positions laid out for the decode's PV operand:
 // each 32-bit word pairs the 16-bit chunk c (codes of 16 / BITS consecutive dimensions) of
 // group positions t and t + 8 (t = 0 .. 7; position t in the low half), and the four words
@@ -224,7 +264,20 @@ __device__ __forceinline__ void quantize_row_part(const __half* __restrict__ x, 
   uint32_t w[NW];
 #pragma unroll
   for (int i = 0; i < NW; ++i) w[i] = 0u;
-  if (sf != 0.0f) {
+  if (sf != 0.0f && BITS == 2) {
+    // code = #{k : x >= X_k}, three half2 comparisons per pair of values; 1024 + code is
+    // exact in fp16 and leaves the code in the half's low bits
+    const __half2 x1 = __half2half2(code_threshold(1, sf, zf));
+    const __half2 x2 = __half2half2(code_threshold(2, sf, zf));
+    const __half2 x3 = __half2half2(code_threshold(3, sf, zf));
+    const __half2 k1024 = __float2half2_rn(1024.0f);
+#pragma unroll
+    for (int k = 0; k < H; ++k) {
+      const __half2 c = __hadd2(__hadd2(__hge2(v[k], x1), __hge2(v[k], x2)), __hadd2(__hge2(v[k], x3), k1024));
+      const uint32_t u = h2_as_u32(c);
+      w[k / 8] |= ((u & 3u) | ((u >> 14) & 0xCu)) << (4 * (k % 8));
+    }
+  } else if (sf != 0.0f) {
     const float rcp = __frcp_rn(sf);
 #pragma unroll
     for (int k = 0; k < H; ++k) {
