@@ -273,11 +273,12 @@ __global__ void __launch_bounds__(128) flush_ring_kernel(const AppendArgs a) {
 constexpr int kBulkTile = 64;
 constexpr int kBulkSlab = 256;
 constexpr int kPad = 136;  // halves per padded shared row (272 bytes: conflict-free ldmatrix)
-// value codes of a tile are staged by 16-position group (a 64-token tile spans at most 5);
-// sized per code width so that three CTAs still fit an SM
+// k / v tiles are double-buffered (the next tile's copies land while this one is
+// transformed and quantized); value codes of a tile are staged by 16-position group (a
+// 64-token tile spans at most 5)
 template <int BITS>
 constexpr size_t bulk_smem() {
-  return (size_t)(kHeadDim + 2 * kBulkTile) * kPad * sizeof(__half) + 5 * 16 * 16 * BITS;
+  return (size_t)(kHeadDim + 4 * kBulkTile) * kPad * sizeof(__half) + 5 * 16 * 16 * BITS;
 }
 
 constexpr int kBulkThreads = 256;
@@ -323,12 +324,12 @@ __device__ __forceinline__ uint4 prep_chunk16(uint4 raw, int col, int pos, const
 }
 
 template <int BITS, int NSEL, bool PREP>
-__global__ void __launch_bounds__(kBulkThreads, 3) append_bulk_kernel(const AppendArgs a) {
+__global__ void __launch_bounds__(kBulkThreads, 2) append_bulk_kernel(const AppendArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __half* Ts = reinterpret_cast<__half*>(smem_raw);
-  __half* ks = Ts + kHeadDim * kPad;
-  __half* vs = ks + kBulkTile * kPad;
-  uint8_t* vstg = reinterpret_cast<uint8_t*>(vs + kBulkTile * kPad);  // value groups of the tile
+  __half* const kbuf = Ts + kHeadDim * kPad;               // [2][kBulkTile][kPad]
+  __half* const vbuf = kbuf + 2 * kBulkTile * kPad;        // [2][kBulkTile][kPad]
+  uint8_t* vstg = reinterpret_cast<uint8_t*>(vbuf + 2 * kBulkTile * kPad);  // value groups of the tile
 
   const int unit = blockIdx.y;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
@@ -367,23 +368,48 @@ __global__ void __launch_bounds__(kBulkThreads, 3) append_bulk_kernel(const Appe
   __shared__ double inv_freq[PREP ? 64 : 1];
   if (PREP && tid < 64) inv_freq[tid] = rope_inv_freq(a.prep, tid);
 
-  const int slab0 = blockIdx.x * kBulkSlab;
-  for (int tile0 = slab0; tile0 < min(slab0 + kBulkSlab, a.n_new); tile0 += kBulkTile) {
-    __syncthreads();  // previous tile fully consumed (and T_K stored on the first pass)
+  // tile tile0's k / v rows into buffer `buf` (16-byte asynchronous copies; rows past the
+  // chunk are zero-filled); one commit group per call
+  auto load_tile = [&](int tile0, int buf) {
+    __half* kd = kbuf + buf * kBulkTile * kPad;
+    __half* vd = vbuf + buf * kBulkTile * kPad;
     for (int c = tid; c < kBulkTile * 16; c += kBulkThreads) {
       const int r = c >> 4, col = (c & 15) * 8;
       const int t = tile0 + r;
-      uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
       if (t < a.n_new) {
         const size_t src = (((size_t)b * a.n_new + t) * a.Hkv + h) * kHeadDim + col;
-        kv = *reinterpret_cast<const uint4*>(a.k_new + src);
-        vv = *reinterpret_cast<const uint4*>(a.v_new + src);
+        cp_async16(kd + r * kPad + col, a.k_new + src);
+        cp_async16(vd + r * kPad + col, a.v_new + src);
+      } else {
+        *reinterpret_cast<uint4*>(kd + r * kPad + col) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(vd + r * kPad + col) = make_uint4(0, 0, 0, 0);
       }
-      if (PREP) kv = prep_chunk16(kv, col, S + t, inv_freq, a.prep);
-      *reinterpret_cast<uint4*>(ks + r * kPad + col) = kv;
-      *reinterpret_cast<uint4*>(vs + r * kPad + col) = vv;
     }
-    __syncthreads();
+    cp_async_commit();
+  };
+  const int slab0 = blockIdx.x * kBulkSlab;
+  const int slab_end = min(slab0 + kBulkSlab, a.n_new);
+  if (slab0 < slab_end) load_tile(slab0, 0);
+  int buf = 0;
+  for (int tile0 = slab0; tile0 < slab_end; tile0 += kBulkTile, buf ^= 1) {
+    __syncthreads();  // previous tile fully consumed (and T_K stored on the first pass)
+    __half* const ks = kbuf + buf * kBulkTile * kPad;
+    const __half* const vs = vbuf + buf * kBulkTile * kPad;
+    if (tile0 + kBulkTile < slab_end) {  // the next tile lands while this one is worked on
+      load_tile(tile0 + kBulkTile, buf ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();  // this tile's rows are in
+    if (PREP) {  // raw keys: RMSNorm + RoPE in place, 16 lanes per row
+      for (int c = tid; c < kBulkTile * 16; c += kBulkThreads) {
+        const int r = c >> 4, col = (c & 15) * 8;
+        uint4* kp = reinterpret_cast<uint4*>(ks + r * kPad + col);
+        *kp = prep_chunk16(*kp, col, S + tile0 + r, inv_freq, a.prep);
+      }
+      __syncthreads();
+    }
 
     // GEMM: warp w owns tile rows [16*mw, 16*mw+16) and output columns [64*nw, 64*nw+64)
     // (mw = w % 4, nw = w / 4): C[16][64] = K[16][128] * T^T
