@@ -7,12 +7,9 @@
 // its `workspace` argument.  The array is file-scope `static __device__`, so every
 // device that loads the library holds WUSHKV_STATIC_SCRATCH_BYTES of it until the
 // process exits; its device address is looked up with cudaGetSymbolAddress (the
-// host-side name is not a device address) once per CUDA context, on the first call made
-// in that context.
+// host-side name is not a device address) on every call, in the current CUDA context.
 #include <cmath>
-#include <cuda.h>
 #include <cuda_runtime.h>
-#include <mutex>
 #include "internal.h"
 
 namespace {
@@ -20,54 +17,15 @@ namespace {
 static __device__ __align__(256) unsigned char g_scratch[WUSHKV_STATIC_SCRATCH_BYTES];
 
 // The array's device address depends on the CUDA context the library's module is loaded
-// in (each device's primary context, or a context the caller created), so it is cached
-// per context: looked up on the first call made in a context and reused afterwards.
-constexpr int kMaxContexts = 64;
-std::mutex g_setup_mutex;
-CUcontext g_ctx[kMaxContexts] = {};
-void* g_scratch_ptr[kMaxContexts] = {};
-int g_entries = 0;
-
-using CtxGetCurrentFn = CUresult (*)(CUcontext*);
-
-// The driver's cuCtxGetCurrent, fetched through the runtime (no link against libcuda).
-CtxGetCurrentFn ctx_get_current() {
-  static CtxGetCurrentFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<CtxGetCurrentFn>(nullptr);
-    return reinterpret_cast<CtxGetCurrentFn>(p);
-  }();
-  return fn;
-}
-
-// Device address of g_scratch in the current context.
+// in (each device's primary context, or a context the caller created), so it is looked up
+// on every call, in the context current then: a cache keyed on the context handle could
+// hand out a dead context's address once a destroyed context's handle is reused.  The
+// lookup is a host-side table query; the first one in a context loads the module.
 cudaError_t scratch_address(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);  // also makes the device's primary context current if none is
-  if (e != cudaSuccess) return e;
-  e = cudaFree(nullptr);                // initialise the context without allocating
-  if (e != cudaSuccess) return e;
-  const CtxGetCurrentFn get = ctx_get_current();
-  CUcontext ctx = nullptr;
-  if (!get || get(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  for (int i = 0; i < g_entries; ++i) {
-    if (g_ctx[i] == ctx) {
-      *out = g_scratch_ptr[i];
-      return cudaSuccess;
-    }
-  }
   void* p = nullptr;
-  e = cudaGetSymbolAddress(&p, g_scratch);
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
   if (e != cudaSuccess) return e;
   if (!p) return cudaErrorInvalidSymbol;
-  // a full table (more contexts than any process here creates) overwrites the oldest entry
-  const int slot = g_entries < kMaxContexts ? g_entries++ : 0;
-  g_ctx[slot] = ctx;
-  g_scratch_ptr[slot] = p;
   *out = p;
   return cudaSuccess;
 }

@@ -310,13 +310,13 @@ int wushkv_decode_attn_test_timeout(const wushkv_config* cfg, const wushkv_cache
  * Scratch: a file-scope device array of WUSHKV_STATIC_SCRATCH_BYTES that every GPU
  *   loading the library holds until the process exits.  A configuration whose
  *   layout.workspace_bytes exceeds it returns WUSHKV_ESCRATCH and queues nothing.
- * Set-up: the first call made with a given device current looks up the array's device
- *   address (cudaGetSymbolAddress) and caches it; make that first call before any
- *   stream capture on that device.
- * Sharing: all calls on a device share the one array, which keeps what the last call
- *   left; each call clears the part that must start at zero (a memset queued on
- *   `stream` ahead of the kernels).  Calls whose work overlaps in time (different
- *   streams, or threads without ordering) race on the array: serialise them. */
+ * Set-up: every call looks up the array's device address in the current CUDA context
+ *   (cudaGetSymbolAddress, a host-side query).  The first call in a context may load the
+ *   library's device module: make it before any stream capture in that context.
+ * Sharing: all calls in a context share the one array.  Nothing in it needs clearing:
+ *   the decode's first kernel resets the merge's completion counters on every call and
+ *   every other byte is written before it is read.  Calls whose work overlaps in time
+ *   (different streams, or threads without ordering) race on the array: serialise them. */
 int wushkv_decode_attn_static(const wushkv_config* cfg, const wushkv_cache* cache, const void* q,
                               const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
                               void* stream);
