@@ -607,7 +607,7 @@ def run_gpu(args, rank, world, local_rank):
             "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": traffic,
             "traffic_source": traffic_why,
-            "kernel": "wushkv_decode_attn (decode_prologue + decode_main)", "peak_kind": peak_kind,
+            "kernel": "wushkv_decode_attn (decode_main_kernel)", "peak_kind": peak_kind,
         },
         "gpu_launches": 2 * K,  # per timed step: fused append_small + decode_main
         "clocks": clocks,
@@ -703,10 +703,12 @@ def measure_decode(bnd, synth, dev, name, layers, reps=200, warmup=10):
     """Decode calls of one workload as a serving engine issues them: `layers` layer caches
     (the workload's shape, filled by bulk appends to its full context, so the quantized
     region is at its steady state) rotate so that the working set is larger than four times
-    L2; each call is a CUDA graph replay (prologue + main kernel), timed per launch with CUDA
-    events on the launching stream.  The decode never changes the cache, so every call
-    reads the same bytes.  Algorithmic bytes per call: the per-unit costs (codes and (s, z)
-    of the quantized positions, fp16 window rows, q in / out, T_K^{-1})."""
+    L2; each call is a CUDA graph replay (one kernel), timed per launch with CUDA events on
+    the launching stream.  A second measurement replays one graph holding one call per
+    layer, as a model's decode step issues them (`*_step_graph`: the graph's time over its
+    calls, launch overhead shared).  The decode never changes the cache, so every call reads
+    the same bytes.  Algorithmic bytes per call: the per-unit costs (codes and (s, z) of the
+    quantized positions, fp16 window rows, q in / out, T_K^{-1})."""
     import torch
     wl = synth.WORKLOADS[name] if isinstance(name, str) else name
     name = wl.name
@@ -747,10 +749,24 @@ def measure_decode(bnd, synth, dev, name, layers, reps=200, warmup=10):
             evs[j].record(stream)
             graphs[j % layers].replay()
         evs[reps].record(stream)
+        step = torch.cuda.CUDAGraph()  # one call per layer, back to back
+        with torch.cuda.graph(step, stream=stream):
+            for c in range(layers):
+                caches[c].decode_attn(q[c], tinvs[c], scale, out=outs[c], stream=stream)
+        step_reps = max(reps // layers, 8)
+        for _ in range(3):
+            step.replay()
+        sevs = [torch.cuda.Event(enable_timing=True) for _ in range(step_reps + 1)]
+        stream.synchronize()
+        for j in range(step_reps):
+            sevs[j].record(stream)
+            step.replay()
+        sevs[step_reps].record(stream)
     stream.synchronize()
     ms = [evs[j].elapsed_time(evs[j + 1]) for j in range(reps)]
+    step_ms = [sevs[j].elapsed_time(sevs[j + 1]) / layers for j in range(step_reps)]
     assert all(c.status() == 0 for c in caches)
-    del graphs
+    del graphs, step
     t = sum(ms) / len(ms) / 1e3
     nbytes = StateMirror(wl, S, Sq).decode_bytes()
     peak, peak_kind = measured_peaks()
@@ -761,7 +777,11 @@ def measure_decode(bnd, synth, dev, name, layers, reps=200, warmup=10):
            "decode_gbs": round(nbytes / t / 1e9, 2), "frac_measured_hbm": round(nbytes / t / 1e9 / peak, 4),
            "pct_of_8tbps": round(100 * nbytes / t / 1e9 / NOMINAL_HBM_GBS, 2), "peak_kind": peak_kind,
            "layers_rotated": layers, "working_set_gb": round(layers * units_bytes / 1e9, 2),
-           "launch": "one CUDA graph per decode call (prologue + main), events per launch", "reps": reps}
+           "launch": "one CUDA graph per decode call (one kernel), events per launch", "reps": reps}
+    ts = sum(step_ms) / len(step_ms) / 1e3
+    res.update({"decode_us_per_call_step_graph": round(ts * 1e6, 3), "decode_gbs_step_graph": round(nbytes / ts / 1e9, 2),
+                "frac_measured_hbm_step_graph": round(nbytes / ts / 1e9 / peak, 4),
+                "step_graph": f"one graph of {layers} calls (one per layer cache), events per replay, {step_reps} replays"})
     if wl.n_layers > 1:  # a decode step of the whole model: one call per layer, all layers alike
         res["model_step_ms"] = round(wl.n_layers * t * 1e3, 3)
         res["tokens_per_s"] = round(wl.batch / (wl.n_layers * t), 1)
@@ -830,7 +850,7 @@ def measure_chunk(bnd, synth, dev, n=8, reps=20):
             "append_us": round(app_s * 1e6, 2), "chunk_attn_us": round(att_s * 1e6, 2),
             "passes_over_cache": passes, "chunk_attn_gbs": round(passes * cache_bytes / att_s / 1e9, 2),
             "query_tokens_per_s": round(wl.batch * n / (app_s + att_s), 1),
-            "launch": "eager: 1 append launch + 2 launches per pass (prologue, main)", "reps": reps}
+            "launch": "eager: 1 append launch + 1 decode launch per pass", "reps": reps}
 
 
 def measure_gram(bnd, synth, dev, n_seq=4, seq_len=32768, reps=10):

@@ -54,24 +54,31 @@ int derive(const wushkv_config* cfg, Derived* d) {
   if (d->nsel > 4) return WUSHKV_EUNSUPPORTED;
 
   // decode work split: n_split items per unit, chosen so that units * n_split fills whole
-  // waves of the GPU's CTA slots (the kernel divides each unit's current quantized region
-  // evenly among its items at run time); split_tokens is the per-item bound at capacity
+  // waves of the GPU's CTA slots best (the kernel divides each unit's current quantized
+  // region evenly among its items at run time); an even n_split runs as clusters of two
+  // CTAs (consecutive items), which share the query's preparation and merge their states
+  // before the unit's last merge, and wins a near-tie (within half a percent of fill); on
+  // a tie the smaller n_split wins.  (Clusters of three or more CTAs would leave SMs of a
+  // B200 that no such cluster can be placed on idle.)  split_tokens is the per-item bound
+  // at capacity
   {
     const int slots = kB200SMs * decode_ctas_per_sm(g);
     int n0 = slots / d->units;
     if (n0 < 1) n0 = 1;
-    int best = n0;
-    double best_eff = 0.0;
-    for (int n = n0; n <= n0 + 3 && n <= kMaxSplits; ++n) {
+    if (n0 > kMaxSplits) n0 = kMaxSplits;
+    int best = 1;
+    double best_score = -1.0;
+    for (int n = n0 > 3 ? n0 - 3 : 1; n <= n0 + 3 && n <= kMaxSplits; ++n) {
       const long long items = (long long)d->units * n;
       const long long waves = (items + slots - 1) / slots;
-      const double eff = (double)items / (double)(waves * slots);
-      if (eff > best_eff + 1e-9) {
-        best_eff = eff;
+      const double score = (double)items / (double)(waves * slots) + (n % 2 == 0 ? 0.005 : 0.0);
+      if (score > best_score + 1e-9) {
+        best_score = score;
         best = n;
       }
     }
-    d->n_split = best > kMaxSplits ? kMaxSplits : best;
+    d->n_split = best;
+    d->cluster = best % 2 == 0 ? 2 : 1;
     const int tiles = ceil_div(d->cap_alloc, kTileTokens);
     d->split_tokens = ceil_div(tiles, d->n_split) * kTileTokens;
   }
@@ -83,17 +90,14 @@ int derive(const wushkv_config* cfg, Derived* d) {
   d->ring_bytes = U * (size_t)d->ring * kHeadDim * 2;
   d->state_bytes = round_up((2 * U + 1) * 4, 16);
   size_t off = 0;
-  d->ws_tickets = off;  // unit counters, then group counters
-  off = round_up(off + U * 4 * (1 + (size_t)ceil_div(d->n_split, kMergeGroup)), 256);
+  d->ws_tickets = off;  // unit counters (zero between calls)
+  off = round_up(off + U * 4, 256);
   d->ws_qprime = off;
   off = round_up(off + U * g * kHeadDim * 4, 256);
   d->ws_qfrag = off;
   off = round_up(off + U * kQFragBytes, 256);
-  d->ws_partials = off;
-  off = round_up(off + U * (size_t)d->n_split * g * 132 * 4, 256);
-  const size_t ngroups = (size_t)ceil_div(d->n_split, kMergeGroup);
-  d->ws_gpartials = off;
-  off = round_up(off + U * ngroups * g * 132 * 4, 256);
+  d->ws_partials = off;  // one merged state per cluster
+  off = round_up(off + U * (size_t)(d->n_split / d->cluster) * g * 132 * 4, 256);
   d->ws_total = off;
   return WUSHKV_OK;
 }
@@ -155,6 +159,7 @@ extern "C" int wushkv_pack_layout(const wushkv_config* cfg, wushkv_layout* out) 
   out->chunk_workspace_bytes = chunk_workspace(cfg);
   out->split_tokens = d.split_tokens;
   out->code_order = WUSHKV_CODE_ORDER_VGROUP16;
+  out->decode_cluster = d.cluster;
   return WUSHKV_OK;
 }
 
@@ -231,7 +236,6 @@ static void fill_append(const wushkv_config* cfg, const Derived& d, const wushkv
   a->f_lo = d.f_lo;
   a->f_hi = d.f_hi;
   a->Hq = cfg->n_q_heads;
-  a->ngroups = ceil_div(d.n_split, kMergeGroup);
   a->transform = cfg->transform;
   a->quant_rms = cfg->quantizer == WUSHKV_QUANT_RMS;
   a->rms_kb = (float)(2.0 * (double)cfg->clip_alpha / (double)((1 << cfg->bits) - 1));
@@ -274,7 +278,7 @@ static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv
   a->qprime = reinterpret_cast<float*>(ws + d.ws_qprime);
   a->qfrag = ws + d.ws_qfrag;
   a->partials = reinterpret_cast<float*>(ws + d.ws_partials);
-  a->gpartials = reinterpret_cast<float*>(ws + d.ws_gpartials);
+  a->cluster = d.cluster;
   a->units = d.units;
   a->fused = 0;
   a->n_new = 0;
@@ -401,15 +405,15 @@ static int step_impl(const wushkv_config* cfg, const wushkv_cache* cache, const 
   da.prep = ps;
   cudaError_t e;
   if (n_new <= cfg->chunk_max) {
-    // one kernel appends and prepares the decode (q', counters); the main decode kernel
-    // is its programmatic dependent and waits for it before reading the cache
+    // one kernel appends and prepares the decode (q' and its fragments); the main decode
+    // kernel is its programmatic dependent and waits for it before reading the cache
     aa.defer_state = 1;
     aa.q = da.q;
     aa.t_k_inv = da.t_k_inv;
     aa.qprime = da.qprime;
     aa.qfrag = da.qfrag;
     aa.scale_log2 = da.scale_log2;
-    aa.tickets = da.tickets;
+    aa.qchains = d.cluster;
     e = launch_append_fused(d, cfg->bits, aa, st);
     if (e == cudaSuccess) {
       da.fused = 1;

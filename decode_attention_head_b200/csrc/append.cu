@@ -81,21 +81,19 @@ __device__ void quantize_ring_range(const AppendArgs& a, int unit, int p_begin, 
 
 // ---------------------------------------------------------------------------------
 // q'_j = T_K^{-T} q_j (fp32) of the unit's G query heads into the decode workspace, by the
-// CTA's 128 threads: warp w sums rows [32w, 32w+32) of T_K^{-1} for the four dimensions
-// 4*lane .. 4*lane+3 (all 32 float4 loads in flight at once), the warps' partial sums meet
-// in shared memory.  Also resets the unit's decode completion counters and builds the
-// unit's query fragments for the decode kernel (qfrag.cuh).
+// CTA's 128 threads: thread j loads column j of T_K^{-1} (all 128 rows in flight at once)
+// and sums Tinv[i][j] * q[i] in the chains every decode path takes (qprime_chains, with
+// a.qchains = the decode's cluster size), so that the fused step and a plain decode see the
+// same q'.  Also builds the unit's query fragments for the decode kernel (qfrag.cuh).
 template <int BITS, int G>
 __device__ void prepare_query(const AppendArgs& a, int unit, int tid) {
   __shared__ __align__(16) float qs[G][kHeadDim];
-  __shared__ float red[4][G][kHeadDim];
   const int b = unit / a.Hkv, h = unit % a.Hkv;
   const int warp = tid >> 5, lane = tid & 31;
-  const float4* Ti =
-      reinterpret_cast<const float4*>(a.t_k_inv + ((size_t)h * kHeadDim + 32 * warp) * kHeadDim) + lane;
-  float4 t[32];
+  const float* Tcol = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim + tid;
+  float t[kHeadDim];
 #pragma unroll
-  for (int u = 0; u < 32; ++u) t[u] = __ldg(Ti + (size_t)u * (kHeadDim / 4));
+  for (int i = 0; i < kHeadDim; ++i) t[i] = __ldg(Tcol + (size_t)i * kHeadDim);
   for (int i = tid; i < G * kHeadDim; i += 128)
     qs[i / kHeadDim][i % kHeadDim] = __half2float(a.q[((size_t)b * a.Hq + h * G) * kHeadDim + i]);
   if (a.prep.enabled) {  // raw queries: RMSNorm + RoPE at the query's position, head by head
@@ -109,28 +107,14 @@ __device__ void prepare_query(const AppendArgs& a, int unit, int tid) {
     for (int hh = warp; hh < G; hh += 4) prep_head_warp(qs[hh], a.prep.q_gain, a.prep, qpos, lane);
   }
   bar_sync(2, 128);
+  float acc[G];
+  qprime_chains<G>(t, qs, a.qchains, acc);
+  bar_sync(2, 128);  // every thread has read q
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const float qv = qs[hh][32 * warp + u];
-      acc.x = fmaf(t[u].x, qv, acc.x);
-      acc.y = fmaf(t[u].y, qv, acc.y);
-      acc.z = fmaf(t[u].z, qv, acc.z);
-      acc.w = fmaf(t[u].w, qv, acc.w);
-    }
-    reinterpret_cast<float4*>(red[warp][hh])[lane] = acc;
+    qs[hh][tid] = acc[hh];
+    a.qprime[((size_t)unit * G + hh) * kHeadDim + tid] = acc[hh];
   }
-  bar_sync(2, 128);
-  for (int i = tid; i < G * kHeadDim; i += 128) {
-    const int hh = i / kHeadDim, j = i % kHeadDim;
-    const float v = (red[0][hh][j] + red[1][hh][j]) + (red[2][hh][j] + red[3][hh][j]);
-    qs[hh][j] = v;  // q is no longer read
-    a.qprime[(size_t)unit * G * kHeadDim + i] = v;
-  }
-  for (int i = tid; i < a.ngroups; i += 128) a.tickets[a.B * a.Hkv + (size_t)unit * a.ngroups + i] = 0u;
-  if (tid == 0) a.tickets[unit] = 0u;
   bar_sync(2, 128);
   __shared__ float cred[64];
   build_query_frags<BITS, G>(qs, tid, 128, cred, a.scale_log2, a.qfrag + (size_t)unit * kQFragBytes,
@@ -138,8 +122,8 @@ __device__ void prepare_query(const AppendArgs& a, int unit, int tid) {
 }
 
 // Small append: one 128-thread CTA per (sequence, KV head).  G > 0: the fused step
-// (wushkv_step) also prepares the decode that follows (q', its query fragments and its
-// counters) in a second CTA per unit (blockIdx.y = 1), in parallel with the append and
+// (wushkv_step) also prepares the decode that follows (q' and its query fragments) in a
+// second CTA per unit (blockIdx.y = 1), in parallel with the append and
 // for every unit, including one whose append is refused (its cache is decoded as it
 // stands).  Each role synchronises on its own named barrier (1: append, 2: decode
 // preparation).

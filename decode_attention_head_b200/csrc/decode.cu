@@ -4,30 +4,33 @@
 // §4.4 fp16 sink / recent windows around the quantized middle region).
 //
 // Two launches per call:
-//  1. decode_prologue (one 512-thread CTA per (sequence, KV head)): q'_j = T_K^{-T} q_j
-//     for its g query heads in fp32, the query's fixed-point tensor-core fragments built
-//     from it (qfrag.cuh), and the reset of the unit's completion counters.  It releases
-//     the main kernel at once (programmatic dependent launch), so the main kernel's KV
-//     stream starts while it runs.  (In a fused step, wushkv_step, the append kernel does
-//     this work instead; the main kernel then derives the post-append state itself,
-//     streams the tiles the append cannot touch at once and waits for the append before
-//     reading anything else -- see DecodeArgs::fused.)
-//  2. decode_main: grid (n_split, units).  Work item s of a unit takes the s-th share of
-//     the unit's current quantized region [S_sink, S_quant) (whole 128-position stages)
-//     and of its fp16 window positions (sink [0, S_sink) and recent [S_quant, S)).
-//     The quantized positions stream through shared memory in 128-position stages
-//     (K codes, V codes, K and V (s, z)) via bulk copies on an mbarrier ring: one
-//     producer warp, four consumer warps, 32 positions per consumer warp per stage.
-//     The consumer warps take q' as a 31-bit fixed-point integer split into four signed
-//     8-bit limbs, already laid out as the mma.sync B fragments they need:
+//  1. decode_query (one 128-thread CTA per (sequence, KV head)): q'_j = T_K^{-T} q_j for its
+//     g query heads in fp32 and the query's fixed-point tensor-core fragments built from it
+//     (qfrag.cuh), into the workspace.  It releases the main kernel at once (programmatic
+//     dependent launch), so the main kernel's KV stream starts while it runs.  (In a fused
+//     step, wushkv_step, the append kernel does this work instead; the main kernel then
+//     derives the post-append state itself, streams the tiles the append cannot touch at
+//     once and waits for the append before reading anything else -- see DecodeArgs::fused.)
+//  2. decode_main: grid (n_split, units) in clusters of C (1 or 2) consecutive work items of
+//     a unit.  Work item s of a unit takes the s-th share of the unit's current quantized
+//     region [S_sink, S_quant) (whole 128-position stages) and of its fp16 window positions
+//     (sink [0, S_sink) and recent [S_quant, S)).
+//   * Stream: the quantized positions pass through shared memory in 128-position stages
+//     (K codes, V codes, K and V (s, z)) via bulk copies on an mbarrier ring: one producer
+//     warp, four consumer warps, 32 positions per consumer warp per stage.  The consumer
+//     warps take q' as a 31-bit fixed-point integer split into four signed 8-bit limbs,
+//     laid out as the mma.sync B fragments they need:
 //       QK  : u8 codes x s8 query limbs on tensor cores (mma m16n8k32, exact int32),
 //             logit = log2e*scale*(z*sum(q') + s*sigma*D)  (dequantization folded);
 //       softmax: online, base 2, with a running max that may go stale by 2^8;
 //       PV  : fp16 codes x fp16 (p*s as hi + lo) on tensor cores (mma m16n8k16,
 //             fp32 accumulate), plus sum(p*z) for the zero-point term.
-//     Each item merges its warps and writes (m, l, o); the last item of each group of
-//     items merges the group, the last group merges the groups and writes the output
-//     (atomic counters, nobody waits).
+//   * Merge: each CTA merges its warps into (m, l, o) in its own shared memory; in a
+//     cluster of two, rank 1 stores its state into rank 0's shared memory and rank 0 merges
+//     the two; with one cluster per unit it writes the output, else it writes the
+//     cluster's partial and the last cluster of the unit to finish (an atomic counter that
+//     it then resets to zero, so the workspace needs no clearing between calls) merges them
+//     and writes the output.  Nobody waits on another cluster.
 //
 // Code unpacking needs no shifts on the key side: masking a packed 32-bit word with
 // 0x03030303 << 2j leaves, in each byte, one code times 4^j -- an exact u8 operand.
@@ -125,63 +128,44 @@ __device__ __forceinline__ uint32_t vcode4(uint32_t x, int mi) {
   }
 }
 
-// ---------------------------------------------------------------------------------
-// Prologue: one CTA per unit, 512 threads; thread (part, j) sums 32 of the 128 terms of
-// q'[j] = sum_i Tinv[i][j] q[i], the four parts are added in shared memory, and the CTA
-// then builds the unit's query fragments (qfrag.cuh) for every work item of the unit.
-constexpr int kPrologueThreads = 512;
-
+// The query of a plain decode call, in a kernel of its own: one 128-thread CTA per unit
+// loads column j = thread of T_K^{-1} (all rows in flight at once), forms q' in the chains
+// every path takes (qprime_chains, with the main kernel's cluster size) and the query
+// fragments (qfrag.cuh), into the workspace.  It lets the main kernel launch at once
+// (programmatic dependent launch); the main kernel's KV stream does not wait for it.
 template <int BITS, int G>
-__global__ void __launch_bounds__(kPrologueThreads) decode_prologue_kernel(const DecodeArgs a) {
-  __shared__ __align__(16) float qs[G][kHeadDim];  // q, then q'
-  __shared__ float part[4][G][kHeadDim];
-  __shared__ float red[64];
+__global__ void __launch_bounds__(128) decode_query_kernel(const DecodeArgs a) {
+  __shared__ __align__(16) float qs[G][kHeadDim];
+  __shared__ float red[24];
   griddep_launch();
-  const int unit = blockIdx.x;
+  const int unit = blockIdx.x, tid = threadIdx.x;
   const int b = unit / a.Hkv, h = unit % a.Hkv;
-  const int tid = threadIdx.x, j = tid & (kHeadDim - 1), pt = tid >> 7;
-  const float* Ti = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim + (size_t)(32 * pt) * kHeadDim + j;
-  // all 32 of this thread's T_K^{-1} loads are in flight before q is staged: one round trip
-  float t[32];
+  const float* Tcol = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim + tid;
+  float t[kHeadDim];
 #pragma unroll
-  for (int u = 0; u < 32; ++u) t[u] = __ldg(Ti + (size_t)u * kHeadDim);
-  for (int i = tid; i < G * kHeadDim; i += kPrologueThreads) {
-    const int hh = i / kHeadDim, cc = i % kHeadDim;
-    qs[hh][cc] = __half2float(a.q[head_row(a, b, h, hh) * kHeadDim + cc]);
-  }
-  if (a.prep.enabled) {  // raw queries (fused step, bulk route): RMSNorm + RoPE at position S - 1
+  for (int i = 0; i < kHeadDim; ++i) t[i] = __ldg(Tcol + (size_t)i * kHeadDim);
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) qs[hh][tid] = __half2float(a.q[head_row(a, b, h, hh) * kHeadDim + tid]);
+  if (a.prep.enabled) {  // raw queries (bulk-route step): RMSNorm + RoPE at position S - 1
     __syncthreads();
     const int qpos = max(a.state[2 * unit] - 1, 0);
-    for (int hh = tid >> 5; hh < G; hh += kPrologueThreads / 32)
-      prep_head_warp(qs[hh], a.prep.q_gain, a.prep, qpos, tid & 31);
+    for (int hh = tid >> 5; hh < G; hh += 4) prep_head_warp(qs[hh], a.prep.q_gain, a.prep, qpos, tid & 31);
   }
   __syncthreads();
-  float qp[G];
+  float acc[G];
+  qprime_chains<G>(t, qs, a.cluster, acc);
+  __syncthreads();  // every thread has read q
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh) qp[hh] = 0.f;
-#pragma unroll
-  for (int u = 0; u < 32; ++u)
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) qp[hh] = fmaf(t[u], qs[hh][32 * pt + u], qp[hh]);
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) part[pt][hh][j] = qp[hh];
-  __syncthreads();
-  for (int i = tid; i < G * kHeadDim; i += kPrologueThreads) {
-    const int hh = i / kHeadDim, q = i % kHeadDim;
-    const float v = (part[0][hh][q] + part[1][hh][q]) + (part[2][hh][q] + part[3][hh][q]);
-    qs[hh][q] = v;
-    a.qprime[((size_t)unit * G + hh) * kHeadDim + q] = v;
+  for (int hh = 0; hh < G; ++hh) {
+    qs[hh][tid] = acc[hh];
+    a.qprime[((size_t)unit * G + hh) * kHeadDim + tid] = acc[hh];
   }
-  // completion counters of the unit: its group counters, then the unit counter
-  const int ngroups = (a.n_split + kMergeGroup - 1) / kMergeGroup;
-  for (int i = tid; i < ngroups; i += kPrologueThreads) a.tickets[a.units + (size_t)unit * ngroups + i] = 0u;
-  if (tid == 0) a.tickets[unit] = 0u;
   __syncthreads();
-  build_query_frags<BITS, G>(qs, tid, kPrologueThreads, red, a.scale_log2, a.qfrag + (size_t)unit * kQFragBytes,
+  build_query_frags<BITS, G>(qs, tid, 128, red, a.scale_log2, a.qfrag + (size_t)unit * kQFragBytes,
                              [] { __syncthreads(); });
 }
 
-// The unit's query fragments and per-head constants (built by the prologue or the fused
+// The unit's query fragments and per-head constants (built by the cluster or the fused
 // append, staged in shared memory), loaded by one lane: bq[j][nt][r], and for the lane's
 // logit head t4 + 4*hs the constants log2e*scale*sum(q') (zero-point term) and
 // log2e*scale*sigma.
@@ -209,20 +193,34 @@ __device__ __forceinline__ void load_query(const uint8_t* qfs, int lane, int t4,
 }
 
 // ---------------------------------------------------------------------------------
-struct Merge {  // per pseudo-warp (0..3 quantized path, 4..7 window path) and head
+constexpr int kMaxCluster = 2;   // CTAs per cluster
+
+struct __align__(16) Merge {  // per pseudo-warp (0..3 quantized path, 4..7 window path) and head
   float m[8][8], l[8][8], bias[8][8];
   float e[8][8];      // the pseudo-warps' weights 2^(m - M) in the item's merge
   float M[8], L[8];   // the item's merged max and denominator per head
+  // the cluster's merge (rank 0): the CTAs' weights 2^(m_r - M) and the merged (M, L)
+  float ce[kMaxCluster][8];
+  float cM[8], cL[8];
+  int c_abort;        // some CTA of the cluster gave up on a wait
 };
+static_assert(sizeof(Merge) % 16 == 0, "the regions after the Merge block stay 16-byte aligned");
 
+// Dynamic shared memory of the main kernel, in this order: the stage ring (after the
+// stream: the consumer warps' o [4][G][128], the CTA's merged state o [G][128], m [G], l [G],
+// and the weights of the unit's last merge [n_split][G]), the ring's mbarriers, the Merge
+// block, the window path's o [4][G][128], the query fragments, and the other rank's merged
+// state o [G][128], m [G], l [G], abort word (written by that rank).
 template <int BITS, int G>
 struct Shared {
   static constexpr int kStages = Cfg<BITS>::NSTAGE * Cfg<BITS>::STAGE;
-  static constexpr int kPv = kConsumers * G * kHeadDim * 4;  // [4][G][128] fp32, reuses the stages
-  static constexpr int kArena = kStages > kPv ? kStages : kPv;
-  static size_t bytes(int nitems) {
-    return (size_t)kArena + 2 * Cfg<BITS>::NSTAGE * 8 + sizeof(Merge) + (size_t)kPv + kQFragBytes +
-           (size_t)nitems * G * 4;
+  static constexpr int kPv = kConsumers * G * kHeadDim * 4;
+  static constexpr int kPart = ((G * kHeadDim + 2 * G + 1) * 4 + 15) / 16 * 16;  // o, m, l, abort word
+  static constexpr int kWts = kMaxSplits * G * 4;
+  static constexpr int kArena = kStages;
+  static_assert(kPv + kPart + kWts <= kStages, "the epilogue's buffers fit the drained stage ring");
+  static constexpr size_t bytes() {
+    return (size_t)kArena + 2 * Cfg<BITS>::NSTAGE * 8 + sizeof(Merge) + (size_t)kPv + kQFragBytes + kPart;
   }
 };
 
@@ -506,12 +504,12 @@ __device__ __forceinline__ void window_load(const DecodeArgs& a, int unit, int i
 // one-token decode passes INT_MAX: every cached position is visible).
 template <int G>
 __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, int n_sink, int r0, int warp,
-                             int lane, WinRows<G>& w, Merge* mg, float* wpv, int qlim) {
+                             int lane, WinRows<G>& w, Merge* mg, float* wpv, int qlim, const float* qsrc) {
   constexpr int KB = WinRows<G>::KB;
   float qv[G][4];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
-    const float4 t = *reinterpret_cast<const float4*>(a.qprime + ((size_t)unit * G + hh) * kHeadDim + 4 * lane);
+    const float4 t = *reinterpret_cast<const float4*>(qsrc + hh * kHeadDim + 4 * lane);
     qv[hh][0] = t.x * a.scale_log2;
     qv[hh][1] = t.y * a.scale_log2;
     qv[hh][2] = t.z * a.scale_log2;
@@ -594,86 +592,93 @@ __device__ void window_share(const DecodeArgs& a, int unit, int wbeg, int wend, 
   }
 }
 
-// Merge `count` (<= kMergeMax) consecutive partials (m, l, pad, pad, o[128] per head, base 2, o not
-// yet normalised) of one unit.  dst != nullptr: write the merged partial there; else write
-// the normalised output rows of the unit's G query heads.  wts: shared [count][G].  Lane
-// `it` of the warp of head hh reads partial it's (m, l) in one round trip.
-constexpr int kMergeMax = 16;  // partials one merge level reads at most
-static_assert(kMergeGroup <= kMergeMax && (kMaxSplits + kMergeGroup - 1) / kMergeGroup <= kMergeMax,
-              "a merge level reads at most kMergeMax partials (one per lane of a warp)");
+// Four consecutive output values (fp32, or fp16 when out_fp16) at element offset o of out.
+__device__ __forceinline__ void store_out4(const DecodeArgs& a, size_t o, float4 v) {
+  if (a.out_fp16) {
+    __half2* oh = reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + o);
+    oh[0] = __floats2half2_rn(v.x, v.y);
+    oh[1] = __floats2half2_rn(v.z, v.w);
+  } else {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + o) = v;
+  }
+}
+
+// Merge the `count` (<= kMaxSplits) cluster partials (m, l, pad, pad, o[128] per head,
+// base 2, o not yet normalised) of one unit and write the normalised output rows of its G
+// query heads, summing the partials in their order.  wts: shared [count][G].  The warp of
+// head hh reduces the partials' (m, l) (lane i loads partials i, i + 32, ... at once); thread
+// (head, quad) then sums dimensions 4*quad .. 4*quad+3 of every partial's row, sixteen row
+// loads in flight at a time -- the first sixteen issued before the weights are known, so
+// that their round trip overlaps the (m, l) one.  Every partial is finite (an empty one
+// holds m = -inf, l = 0, o = 0), so no term needs skipping.
+constexpr int kRowBatch = 16;
 template <int G>
-__device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, int count, float* dst,
-                               float* wts) {
+__device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, int count, float* wts) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // thread (hh, quad) takes dimensions 4*quad .. 4*quad+3 of head hh: every partial's row is
-  // loaded at once, the first (head, quad)'s rows before the weights are known, so that
-  // their round trip overlaps the (m, l) one; then they are summed in partial order.  Every
-  // partial is finite (an empty one holds o = 0), so no term needs skipping.
   constexpr int kQuads = kHeadDim / 4;
-  float4 ov[kMergeMax];
-  auto load_rows = [&](int idx) {
+  float4 ov[kRowBatch];
+  auto load_rows = [&](int idx, int i0) {
     const int hh = idx / kQuads, d = 4 * (idx % kQuads);
 #pragma unroll
-    for (int it = 0; it < kMergeMax; ++it)
-      ov[it] = it < count ? __ldcg(reinterpret_cast<const float4*>(src + ((size_t)it * G + hh) * kPartStride + 4 + d))
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kRowBatch; ++u)
+      ov[u] = i0 + u < count
+                  ? __ldcg(reinterpret_cast<const float4*>(src + ((size_t)(i0 + u) * G + hh) * kPartStride + 4 + d))
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
   };
-  if (tid < G * kQuads) load_rows(tid);
+  if (tid < G * kQuads) load_rows(tid, 0);
   for (int hh = warp; hh < G; hh += kThreads / 32) {
-    const bool has = lane < count;
-    float mi = -CUDART_INF_F, li = 0.f;
-    if (has) {
-      mi = __ldcg(src + ((size_t)lane * G + hh) * kPartStride);
-      li = __ldcg(src + ((size_t)lane * G + hh) * kPartStride + 1);
+    // every (m, l) this lane needs in one round trip
+    constexpr int kPer = kMaxSplits / 32;
+    float mi[kPer], li[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int i = lane + 32 * k;
+      mi[k] = -CUDART_INF_F;
+      li[k] = 0.f;
+      if (i < count) {
+        const float* p = src + ((size_t)i * G + hh) * kPartStride;
+        mi[k] = __ldcg(p);
+        li[k] = __ldcg(p + 1);
+      }
     }
-    float M = mi;
+    float M = mi[0];
+#pragma unroll
+    for (int k = 1; k < kPer; ++k) M = fmaxf(M, mi[k]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    const float e = (!has || M == -CUDART_INF_F) ? 0.f : exp2f(mi - M);
-    if (has) wts[lane * G + hh] = e;
-    float L = fmaf(e, li, 0.f);
+    float L = 0.f, e[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      e[k] = (lane + 32 * k < count && M != -CUDART_INF_F) ? exp2f(mi[k] - M) : 0.f;
+      L = fmaf(e[k], li[k], L);
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    __syncwarp();
-    if (dst) {
-      if (lane == 0) {
-        dst[hh * kPartStride + 0] = M;
-        dst[hh * kPartStride + 1] = L;
-      }
-    } else {
-      const float invL = L > 0.f ? 1.0f / L : 0.f;
-      for (int it = lane; it < count; it += 32) wts[it * G + hh] *= invL;
-      if (lane == 0 && !(L > 0.f)) atomicOr(a.status, kStatusEmpty);
-    }
+    const float invL = L > 0.f ? 1.0f / L : 0.f;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k)
+      if (lane + 32 * k < count) wts[(lane + 32 * k) * G + hh] = e[k] * invL;
+    if (lane == 0 && !(L > 0.f)) atomicOr(a.status, kStatusEmpty);
   }
   __syncthreads();
   const int b = unit / a.Hkv, h = unit % a.Hkv;
   for (int idx = tid; idx < G * kQuads; idx += kThreads) {
     const int hh = idx / kQuads, d = 4 * (idx % kQuads);
-    if (idx != tid) load_rows(idx);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < count; i0 += kRowBatch) {
+      if (idx != tid || i0 != 0) load_rows(idx, i0);
 #pragma unroll
-    for (int it = 0; it < kMergeMax; ++it) {
-      if (it < count) {
-        const float w = wts[it * G + hh];
-        acc.x = fmaf(w, ov[it].x, acc.x);
-        acc.y = fmaf(w, ov[it].y, acc.y);
-        acc.z = fmaf(w, ov[it].z, acc.z);
-        acc.w = fmaf(w, ov[it].w, acc.w);
+      for (int u = 0; u < kRowBatch; ++u) {
+        if (i0 + u < count) {
+          const float w = wts[(i0 + u) * G + hh];
+          acc.x = fmaf(w, ov[u].x, acc.x);
+          acc.y = fmaf(w, ov[u].y, acc.y);
+          acc.z = fmaf(w, ov[u].z, acc.z);
+          acc.w = fmaf(w, ov[u].w, acc.w);
+        }
       }
     }
-    if (dst) {
-      *reinterpret_cast<float4*>(dst + hh * kPartStride + 4 + d) = acc;
-    } else {
-      const size_t o = head_row(a, b, h, hh) * kHeadDim + d;
-      if (a.out_fp16) {
-        __half2* oh = reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + o);
-        oh[0] = __floats2half2_rn(acc.x, acc.y);
-        oh[1] = __floats2half2_rn(acc.z, acc.w);
-      } else {
-        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + o) = acc;
-      }
-    }
+    store_out4(a, head_row(a, b, h, hh) * kHeadDim + d, acc);
   }
 }
 
@@ -694,12 +699,15 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
   float* pv = reinterpret_cast<float*>(smem);  // [4][G][128], written once the stages are drained
+  float* cpo = reinterpret_cast<float*>(smem + SM::kPv);  // the CTA's merged o [G][128] (not normalised)
+  float* cpm = cpo + G * kHeadDim;                        // and its m [G], l [G]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kArena);
   uint64_t* empty = full + C::NSTAGE;
   Merge* mg = reinterpret_cast<Merge*>(empty + C::NSTAGE);
   float* wpv = reinterpret_cast<float*>(mg + 1);   // window path [4][G][128]
   uint8_t* qfs = reinterpret_cast<uint8_t*>(wpv + kConsumers * G * kHeadDim);  // the unit's query fragments
-  float* wts = reinterpret_cast<float*>(qfs + kQFragBytes);  // [nitems][G] (last item only)
+  float* srecv = reinterpret_cast<float*>(qfs + kQFragBytes);  // rank 1's merged state (rank 0 only)
+  float* wts = reinterpret_cast<float*>(smem + SM::kPv + SM::kPart);  // [n_split][G] (the last merge only)
   __shared__ uint32_t s_last;
   __shared__ int s_abort;  // set by a bounded wait that gave up: every role leaves its loop
   volatile int* abort = &s_abort;
@@ -708,6 +716,7 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   const int g = lane >> 2, t4 = lane & 3;
   const int unit = blockIdx.y, item = blockIdx.x;
   const int nitems = a.n_split;
+  const int ncta = a.cluster;  // CTAs per cluster (consecutive items of the unit)
   int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
   // fused step: the state read above is the one before the append (that kernel leaves the
   // state words to this one); the append's outcome follows from it as the append derives it
@@ -772,8 +781,10 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   qs.kacc = 64;
   qs.s_lim = 0.f;  // the first position with s > 0 sets kacc
 
+  // With clusters of two, every thread of both CTAs takes the cluster barrier once, on every
+  // path: when rank 1 has stored its merged state into rank 0's shared memory.
   if (warp == kConsumers) {
-    // ---------------- producer: streams the item's tiles; needs nothing from the prologue
+    // ---------------- producer: streams the item's tiles; needs nothing from the query
     if (lane == 0 && ntiles > 0) {
       int issued = 0;
       bool waited = !a.fused;  // fused step: tiles below the old S_quant stream at once
@@ -805,11 +816,11 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   } else {
     // ---------------- consumers
     // (a) this warp's share of the fp16 window: the first rows are loaded before the wait
-    // for the prologue (they do not depend on it), the rest while the first tiles land
+    // for the query (they do not depend on it), the rest while the first tiles land
     WinRows<G> wr;
     if (a.fused) griddep_wait();  // the window holds the appended tokens
     window_load<G>(a, unit, wbeg + warp, wend, n_sink, r0, lane, wr);
-    griddep_wait();  // q', the query fragments and the counter resets come from the prologue
+    griddep_wait();  // q' and the query fragments come from the kernel before
     {  // the unit's query fragments into shared memory while the window share runs
       constexpr int n16 = GCfg<G>::FW * 8 + 4;
       const uint8_t* src = a.qfrag + (size_t)unit * kQFragBytes;
@@ -817,7 +828,8 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
       cp_async_commit();
     }
     const int qlim = a.chunk_n > 0 ? S - a.chunk_n + a.chunk_t0 : INT_MAX;
-    window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, wr, mg, wpv, qlim);
+    window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, wr, mg, wpv, qlim,
+                    a.qprime + (size_t)unit * G * kHeadDim);
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) qs.o[mt][0] = qs.o[mt][1] = qs.o[mt][2] = qs.o[mt][3] = 0.f;
     // (b) quantized positions
@@ -862,9 +874,9 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     }
   }
   __syncthreads();  // every stage consumed and every copy landed: pv may reuse the stages
-  // a bounded wait gave up (STATUS_TIMEOUT is set): this item's results are incomplete, so
-  // it writes no partial and takes no part in the merge -- the unit's output is not written
-  if (s_abort) return;
+  // A CTA whose bounded wait gave up (STATUS_TIMEOUT is set) has incomplete results: it still
+  // takes every step below (the cluster barrier needs it), but its unit's output and state
+  // are not written, so a timeout never produces plausible-looking output.
 
   if (warp < kConsumers) {
 #pragma unroll
@@ -884,8 +896,12 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   }
   __syncthreads();
 
-  // ======================= merge the 8 pseudo-warps, write this item's partial: the
-  // weights once per (pseudo-warp, head), then the rows
+  // ======================= merge the 8 pseudo-warps into the CTA's state (m, l, o): the
+  // weights once per (pseudo-warp, head), then the rows.  Rank 0 of a cluster keeps its
+  // state (cpo, cpm); rank 1 stores its own straight into rank 0's receive buffer.
+  const int rank = ncta > 1 ? (int)cluster_rank() : 0;
+  const int ncl = nitems / ncta;  // clusters of the unit
+  const uint32_t peer = ncta > 1 ? cluster_map(srecv, 0) : 0u;  // rank 0's receive buffer
   if (tid < G) {
     const int hh = tid;
     float M = -CUDART_INF_F;
@@ -898,70 +914,124 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
       mg->e[w][hh] = e;
       L = fmaf(e, mg->l[w][hh], L);
     }
-    mg->M[hh] = M;
-    mg->L[hh] = L;
+    if (rank == 0) {
+      cpm[hh] = M;
+      cpm[G + hh] = L;
+    } else {
+      st_cluster_f32(peer + 4 * (G * kHeadDim + hh), M);
+      st_cluster_f32(peer + 4 * (G * kHeadDim + G + hh), L);
+    }
+  } else if (tid == 32 && rank != 0) {
+    st_cluster_s32(peer + 4 * (G * kHeadDim + 2 * G), s_abort);
   }
   __syncthreads();
-  float* part = a.partials + ((size_t)unit * nitems + item) * G * kPartStride;
-  for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
-    const int hh = idx / kHeadDim, d = idx % kHeadDim;
-    float O = 0.f;
+  for (int q4 = tid; q4 < G * kHeadDim / 4; q4 += kThreads) {
+    const int hh = (4 * q4) / kHeadDim, d = (4 * q4) % kHeadDim;
+    float O[4];
 #pragma unroll
-    for (int w = 0; w < 2 * kConsumers; ++w) {
-      const float ov = w < kConsumers ? pv[((size_t)w * G + hh) * kHeadDim + d]
-                                      : wpv[((size_t)(w - kConsumers) * G + hh) * kHeadDim + d];
-      O = fmaf(mg->e[w][hh], ov + mg->bias[w][hh], O);
+    for (int c = 0; c < 4; ++c) {
+      O[c] = 0.f;
+#pragma unroll
+      for (int w = 0; w < 2 * kConsumers; ++w) {
+        const float ov = w < kConsumers ? pv[((size_t)w * G + hh) * kHeadDim + d + c]
+                                        : wpv[((size_t)(w - kConsumers) * G + hh) * kHeadDim + d + c];
+        O[c] = fmaf(mg->e[w][hh], ov + mg->bias[w][hh], O[c]);
+      }
     }
-    part[hh * kPartStride + 4 + d] = O;
-    if (d == 0) {
-      part[hh * kPartStride + 0] = mg->M[hh];
-      part[hh * kPartStride + 1] = mg->L[hh];
+    const float4 o4 = make_float4(O[0], O[1], O[2], O[3]);
+    if (rank == 0)
+      *reinterpret_cast<float4*>(cpo + 4 * q4) = o4;
+    else
+      st_cluster_f32x4(peer + 16 * q4, o4);
+  }
+  // phase B: rank 0 holds both CTAs' states (rank 1 is done after it)
+  __syncwarp();
+  if (ncta > 1) {
+    cluster_arrive();
+    cluster_wait();
+  } else {
+    __syncthreads();
+  }
+  if (rank != 0) return;
+
+  // ======================= rank 0 merges the cluster's states in rank order
+  const int b = unit / a.Hkv, h = unit % a.Hkv;
+  if (tid < G) {
+    const int hh = tid;
+    const float m0 = cpm[hh], l0 = cpm[G + hh];
+    const float m1 = ncta > 1 ? srecv[G * kHeadDim + hh] : -CUDART_INF_F;
+    const float l1 = ncta > 1 ? srecv[G * kHeadDim + G + hh] : 0.f;
+    const float M = fmaxf(m0, m1);
+    const float e0 = M != -CUDART_INF_F ? exp2f(m0 - M) : 0.f;
+    const float e1 = (M != -CUDART_INF_F && ncta > 1) ? exp2f(m1 - M) : 0.f;
+    mg->ce[0][hh] = e0;
+    mg->ce[1][hh] = e1;
+    mg->cM[hh] = M;
+    mg->cL[hh] = fmaf(e1, l1, e0 * l0);
+  } else if (tid == 32) {
+    mg->c_abort = s_abort | (ncta > 1 ? reinterpret_cast<const int*>(srecv)[G * kHeadDim + 2 * G] : 0);
+  }
+  __syncthreads();
+  const bool c_abort = mg->c_abort != 0;
+  float* part = a.partials + ((size_t)unit * ncl + item / ncta) * G * kPartStride;
+  for (int q4 = tid; q4 < G * kHeadDim / 4; q4 += kThreads) {
+    const int hh = (4 * q4) / kHeadDim, d = (4 * q4) % kHeadDim;
+    const float e0 = mg->ce[0][hh], e1 = mg->ce[1][hh];
+    const float4 v0 = *reinterpret_cast<const float4*>(cpo + 4 * q4);
+    const float4 v1 = ncta > 1 ? *reinterpret_cast<const float4*>(srecv + 4 * q4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 O = make_float4(fmaf(e1, v1.x, e0 * v0.x), fmaf(e1, v1.y, e0 * v0.y), fmaf(e1, v1.z, e0 * v0.z),
+                                 fmaf(e1, v1.w, e0 * v0.w));
+    if (ncl == 1) {  // the unit's only cluster: the output rows
+      if (!c_abort) {
+        const float L = mg->cL[hh];
+        const float invL = L > 0.f ? 1.0f / L : 0.f;
+        if (d == 0 && !(L > 0.f)) atomicOr(a.status, kStatusEmpty);
+        store_out4(a, head_row(a, b, h, hh) * kHeadDim + d, make_float4(O.x * invL, O.y * invL, O.z * invL, O.w * invL));
+      }
+    } else {  // the cluster's partial, for the unit's last merge
+      *reinterpret_cast<float4*>(part + hh * kPartStride + 4 + d) = O;
+      if (d == 0) {
+        part[hh * kPartStride + 0] = mg->cM[hh];
+        part[hh * kPartStride + 1] = mg->cL[hh];
+      }
     }
   }
-  // ======================= two-level merge: the last item of each group of kMergeGroup
-  // items merges the group; the last group to finish merges the groups and writes the
-  // output (atomic counters, nobody waits).  Neither level reads more than a few partials.
-  const int ngroups = (nitems + kMergeGroup - 1) / kMergeGroup;
-  const int grp = item / kMergeGroup;
-  const int g0 = grp * kMergeGroup, gn = min(kMergeGroup, nitems - g0);
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    uint32_t* gt = a.tickets + a.units + (size_t)unit * ngroups + grp;
-    s_last = (atomicAdd(gt, 1u) == (uint32_t)(gn - 1)) ? 1u : 0u;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const float* up = a.partials + ((size_t)unit * nitems + g0) * G * kPartStride;
-  if (ngroups == 1) {
-    merge_partials<G>(a, unit, up, gn, nullptr, wts);
-    if (S_next >= 0 && tid == 0) {  // every item of the unit has read the old state
+  if (ncl == 1) {
+    if (S_next >= 0 && tid == 0 && !c_abort) {  // every item of the unit has read the old state
       a.state[2 * unit] = S_next;
       a.state[2 * unit + 1] = Sq_next;
     }
     return;
   }
-  float* gp = a.gpartials + ((size_t)unit * ngroups + grp) * G * kPartStride;
-  merge_partials<G>(a, unit, up, gn, gp, wts);
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&a.tickets[unit], 1u) == (uint32_t)(ngroups - 1)) ? 1u : 0u;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  merge_partials<G>(a, unit, a.gpartials + (size_t)unit * ngroups * G * kPartStride, ngroups, nullptr, wts);
-  if (S_next >= 0 && tid == 0) {  // every item of the unit has read the old state
-    a.state[2 * unit] = S_next;
-    a.state[2 * unit + 1] = Sq_next;
+
+  // ======================= the unit's last cluster merges the clusters' partials (an
+  // atomic counter, reset by that cluster for the next call; nobody waits).  A cluster that
+  // gave up on a wait adds 2^16 as well, and the last one then writes nothing.
+  __syncthreads();  // the partial is written; thread 0's acquire-release add publishes it
+  if (tid == 0) {
+    const uint32_t inc = mg->c_abort ? 0x10001u : 1u;
+    const uint32_t old = atomic_add_acq_rel(&a.tickets[unit], inc);
+    s_last = ((old & 0xFFFFu) == (uint32_t)(ncl - 1)) ? (((old + inc) >> 16) != 0 ? 2u : 1u) : 0u;
   }
+  __syncthreads();  // (and orders the other clusters' partials before this CTA's reads of them)
+  if (!s_last) return;
+  if (s_last == 1u) {
+    merge_partials<G>(a, unit, a.partials + (size_t)unit * ncl * G * kPartStride, ncl, wts);
+    if (S_next >= 0 && tid == 0) {  // every item of the unit has read the old state
+      a.state[2 * unit] = S_next;
+      a.state[2 * unit + 1] = Sq_next;
+    }
+  }
+  if (tid == 0) a.tickets[unit] = 0u;
 }
 
-// The main kernel as the programmatic dependent of the kernel before it in the stream: it
-// may start before that kernel ends; whatever it reads from it is behind griddepcontrol.wait.
+// One launch of the main kernel, in clusters of d.cluster consecutive work items (no
+// attribute for clusters of one).  `dependent` (the fused step) makes it the programmatic
+// dependent of the kernel before it in the stream, which it may overlap: whatever it reads
+// from that kernel is behind griddepcontrol.wait.
 template <int BITS, int G>
-cudaError_t launch_main_t(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
-  const size_t smem = Shared<BITS, G>::bytes(d.n_split);
+cudaError_t launch_main_t(const Derived& d, const DecodeArgs& a, cudaStream_t st, bool dependent) {
+  constexpr size_t smem = Shared<BITS, G>::bytes();
   cudaError_t e = ensure_smem_attr<decode_main_kernel<BITS, G>>((int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t lc = {};
@@ -969,58 +1039,63 @@ cudaError_t launch_main_t(const Derived& d, const DecodeArgs& a, cudaStream_t st
   lc.blockDim = dim3(kThreads);
   lc.dynamicSmemBytes = smem;
   lc.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (d.cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)d.cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (dependent) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
   lc.attrs = attr;
-  lc.numAttrs = 1;
+  lc.numAttrs = n;
   e = cudaLaunchKernelEx(&lc, decode_main_kernel<BITS, G>, a);
-  if (e != cudaSuccess) {  // without the attribute: plain stream order
+  if (e != cudaSuccess && dependent) {  // without the programmatic dependency: plain stream order
     (void)cudaGetLastError();
-    decode_main_kernel<BITS, G><<<lc.gridDim, kThreads, smem, st>>>(a);
-    e = cudaGetLastError();
+    lc.numAttrs = n - 1;
+    e = cudaLaunchKernelEx(&lc, decode_main_kernel<BITS, G>, a);
   }
   return e;
 }
 
-template <int BITS, int G>
-cudaError_t launch_decode_t(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
-  decode_prologue_kernel<BITS, G><<<d.units, kPrologueThreads, 0, st>>>(a);
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // the main kernel may start before the prologue ends; its consumers wait
-  // (griddepcontrol.wait) for the prologue's results, its producer does not
-  return launch_main_t<BITS, G>(d, a, st);
-}
-
 template <int BITS>
-cudaError_t launch_main_b(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
+cudaError_t launch_main_b(const Derived& d, const DecodeArgs& a, cudaStream_t st, bool dependent) {
   switch (d.group) {
-    case 1: return launch_main_t<BITS, 1>(d, a, st);
-    case 2: return launch_main_t<BITS, 2>(d, a, st);
-    case 4: return launch_main_t<BITS, 4>(d, a, st);
-    default: return launch_main_t<BITS, 8>(d, a, st);
-  }
-}
-
-template <int BITS>
-cudaError_t launch_decode_b(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
-  switch (d.group) {
-    case 1: return launch_decode_t<BITS, 1>(d, a, st);
-    case 2: return launch_decode_t<BITS, 2>(d, a, st);
-    case 4: return launch_decode_t<BITS, 4>(d, a, st);
-    default: return launch_decode_t<BITS, 8>(d, a, st);
+    case 1: return launch_main_t<BITS, 1>(d, a, st, dependent);
+    case 2: return launch_main_t<BITS, 2>(d, a, st, dependent);
+    case 4: return launch_main_t<BITS, 4>(d, a, st, dependent);
+    default: return launch_main_t<BITS, 8>(d, a, st, dependent);
   }
 }
 
 }  // namespace
 
+template <int BITS>
+cudaError_t launch_query_b(const Derived& d, const DecodeArgs& a, cudaStream_t st) {
+  switch (d.group) {
+    case 1: decode_query_kernel<BITS, 1><<<d.units, 128, 0, st>>>(a); break;
+    case 2: decode_query_kernel<BITS, 2><<<d.units, 128, 0, st>>>(a); break;
+    case 4: decode_query_kernel<BITS, 4><<<d.units, 128, 0, st>>>(a); break;
+    default: decode_query_kernel<BITS, 8><<<d.units, 128, 0, st>>>(a); break;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st) {
-  return bits == 2 ? launch_decode_b<2>(d, a, st) : launch_decode_b<4>(d, a, st);
+  // the query kernel, then the main kernel as its programmatic dependent
+  const cudaError_t e = bits == 2 ? launch_query_b<2>(d, a, st) : launch_query_b<4>(d, a, st);
+  if (e != cudaSuccess) return e;
+  return bits == 2 ? launch_main_b<2>(d, a, st, true) : launch_main_b<4>(d, a, st, true);
 }
 
 cudaError_t launch_decode_main(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st) {
-  return bits == 2 ? launch_main_b<2>(d, a, st) : launch_main_b<4>(d, a, st);
+  return bits == 2 ? launch_main_b<2>(d, a, st, true) : launch_main_b<4>(d, a, st, true);
 }
 
 }  // namespace wushkv

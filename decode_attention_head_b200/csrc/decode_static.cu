@@ -6,8 +6,10 @@
 // The attention itself is the ordinary wushkv_decode_attn path: this file only supplies
 // its `workspace` argument.  The array is file-scope `static __device__`, so every
 // device that loads the library holds WUSHKV_STATIC_SCRATCH_BYTES of it until the
-// process exits; its device address is looked up with cudaGetSymbolAddress (the
-// host-side name is not a device address) on every call, in the current CUDA context.
+// process exits.  It starts zero-filled (static storage), as a workspace must before its
+// first use, and every call leaves the decode's completion counters in it at zero again.
+// Its device address is looked up with cudaGetSymbolAddress (the host-side name is not a
+// device address) on every call, in the current CUDA context.
 #include <cmath>
 #include <cuda_runtime.h>
 #include "internal.h"

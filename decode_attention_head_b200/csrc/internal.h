@@ -15,8 +15,7 @@ constexpr int kB200SMs = 148;         // split policy sizes the decode grid for 
 // Resident decode CTAs per SM the split policy aims at (the kernel's launch bounds hold its
 // registers to this): 8 query heads per KV head need more registers than the others.
 constexpr int decode_ctas_per_sm(int group) { return group == 8 ? 3 : 4; }
-constexpr int kMaxSplits = 255;       // quantized work items per (sequence, KV head)
-constexpr int kMergeGroup = 16;       // work items merged together at the first merge level
+constexpr int kMaxSplits = 128;       // work items per (sequence, KV head): at most 16 clusters of 8
 
 struct Derived {
   int units;        // B * H_kv
@@ -29,8 +28,9 @@ struct Derived {
   int i_lo, i_hi;
   float f_lo, f_hi;
   int n_split, split_tokens;
+  int cluster;      // decode CTAs per thread-block cluster (consecutive items of a unit; divides n_split)
   // workspace offsets (bytes)
-  size_t ws_tickets, ws_qprime, ws_qfrag, ws_partials, ws_gpartials, ws_total;
+  size_t ws_tickets, ws_qprime, ws_qfrag, ws_partials, ws_total;
   // cache buffer sizes (bytes)
   size_t codes_bytes, params_bytes, sink_bytes, ring_bytes, state_bytes;
 };
@@ -66,14 +66,14 @@ struct AppendArgs {
   int i_lo, i_hi;
   float f_lo, f_hi;
   // decode preparation fused into a one-token append (wushkv_step): q' = T_K^{-T} q of the
-  // unit's query heads into the decode workspace, and its completion counters reset
+  // unit's query heads and its query fragments into the decode workspace
   const __half* q;
   const float* t_k_inv;
   float* qprime;
   uint8_t* qfrag;      // the unit's query fragments for the decode kernel (qfrag.cuh)
   float scale_log2;    // softmax_scale * log2(e)
-  uint32_t* tickets;
-  int Hq, ngroups;
+  int Hq;
+  int qchains;         // the decode's cluster size: q' is summed in that many row blocks
   PrepSpec prep;  // raw q / k (wushkv_step_prep): RMSNorm + RoPE fused in
   int defer_state;  // 1 (fused step): leave the state words to the decode kernel that follows
   int transform;  // WUSHKV_TRANSFORM_DENSE (t_k) or WUSHKV_TRANSFORM_HADAMARD (in-kernel)
@@ -99,11 +99,11 @@ struct DecodeArgs {
   void* out;
   int out_fp16;
   int units;
-  uint32_t* tickets;   // [units] unit counters, then [units][ngroups] group counters
-  float* qprime;       // [units][G][128] fp32
-  uint8_t* qfrag;      // [units][kQFragBytes]: query fragments and constants (qfrag.cuh)
-  float* partials;     // [units][n_split][G][132]
-  float* gpartials;    // [units][ngroups][G][132]
+  uint32_t* tickets;   // [units] completion counters of the last merge (zero between calls)
+  float* qprime;       // [units][G][128] fp32 (fused step: written by the append kernel)
+  uint8_t* qfrag;      // [units][kQFragBytes]: query fragments and constants (qfrag.cuh; fused step)
+  float* partials;     // [units][n_split / cluster][G][132]: the clusters' merged states
+  int cluster;         // CTAs per cluster
   // fused step (wushkv_step's one-kernel append of n_new tokens runs just before): that
   // kernel leaves the state words alone, so this one reads the pre-append state, derives the
   // post-append (S, S_quant) from it, streams the tiles below the old S_quant before the
@@ -114,7 +114,7 @@ struct DecodeArgs {
   // heads of each of G / gq consecutive chunk tokens, chunk_t0 the first of them; q and out
   // are [B][chunk_n][H_q][128]; chunk_n = 0 for a one-token decode (gq = G)
   int chunk_n, chunk_t0, gq;
-  PrepSpec prep;       // raw q (wushkv_step_prep, bulk route): the prologue normalises and rotates it
+  PrepSpec prep;       // raw q (wushkv_step_prep, bulk route): the kernel normalises and rotates it
   // bounded waits: the cycle limit after which a wait gives up (STATUS_TIMEOUT), and a test
   // hook -- the producer never issues stage `withhold_tile` of any item (-1: off)
   int withhold_tile;
@@ -138,9 +138,9 @@ cudaError_t ensure_smem_attr(int bytes) {
 
 cudaError_t launch_append(const Derived& d, int bits, bool small, const AppendArgs& a, cudaStream_t st);
 cudaError_t launch_decode(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st);
-// wushkv_step's one-token path: the small append fused with the decode prologue (it lets
-// its dependents launch early), then the main decode kernel alone, launched as that
-// kernel's programmatic dependent (it waits for it before reading anything).
+// wushkv_step's one-token path: the small append fused with the decode's query preparation
+// (it lets its dependents launch early), then the main decode kernel, launched as that
+// kernel's programmatic dependent (it waits for it before reading what it writes).
 cudaError_t launch_append_fused(const Derived& d, int bits, const AppendArgs& a, cudaStream_t st);
 cudaError_t launch_decode_main(const Derived& d, int bits, const DecodeArgs& a, cudaStream_t st);
 

@@ -1,8 +1,9 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, bulk (TMA) copies, ldmatrix, warp-level
-// mma, and the fifth-generation tensor-core path (tensor-memory allocation, loads and
-// stores, tcgen05.mma and its commit).  Every wait is bounded: after ~2 s of clock cycles
-// (or a caller-given limit) it gives up and reports, so a library bug can never hang the
-// GPU.
+// mma, thread-block clusters, and the fifth-generation tensor-core path (tensor-memory
+// allocation, loads and stores, tcgen05.mma and its commit).  Every mbarrier wait is
+// bounded: after ~2 s of clock cycles (or a caller-given limit) it gives up and reports,
+// so a copy that never lands cannot hang the GPU.  The cluster barrier has no such limit;
+// kernels that use it reach every one of its phases on every path.
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -108,6 +109,49 @@ __device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t pari
 // Named barrier `id` over `count` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+
+// Thread-block clusters.  A launch attribute sets the cluster's size; the CTAs of a cluster
+// run at the same time and may store into one another's shared memory.  cluster_arrive /
+// cluster_wait are the two halves of the hardware cluster barrier: every thread of every
+// CTA in the cluster must take part (all lanes of a warp together), arrive releases the
+// thread's earlier memory operations and wait acquires those of the other CTAs.  The
+// barrier's wait has no time limit, so a kernel must reach each of them on every path.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
+// The address, in the cluster's shared-memory window, of the variable at `p` in the
+// shared memory of the cluster's CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_map(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_f32x4(uint32_t addr, float4 v) {  // addr 16-byte aligned
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_s32(uint32_t addr, int v) {
+  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// atomicAdd with acquire-release semantics at GPU scope: it publishes every write that
+// happens before it (other threads' ones too, when a CTA barrier orders them before it)
+// and makes every write published by earlier adds visible to what follows it.
+__device__ __forceinline__ uint32_t atomic_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 
 // Programmatic dependent launch: a kernel lets the next kernel in its stream start

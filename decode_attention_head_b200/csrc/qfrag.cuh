@@ -46,18 +46,47 @@ __device__ __forceinline__ void frag_dim(int j, int r, int t4, int byte, int& di
   }
 }
 
-// Build the unit's fragments from q' (fp32 [G][128] in shared memory) with `nthr` threads
-// (tid = 0 .. nthr-1, a multiple of 32, all of them calling; qf 16-byte aligned).  red: shared scratch of
-// 2 * 8 floats.  sync() is the barrier of those threads (a named barrier in a kernel whose
-// other threads do other work).  Per head, one warp reduces max |q'_d / scale_d| and the
-// sum of q' (lane l holds dimensions 4l .. 4l+3; xor-shuffle tree, a fixed order).
+// q' = T_K^{-T} q for thread j's dimension of G query heads, the sums that every path to
+// the decode's query takes: t[i] = Tinv[i][j] (row i of T_K^{-1}, column j), qs the G query
+// rows; one fmaf chain per block of rows -- rows [0, 64) and [64, 128) added in that order
+// when nchains = 2, one chain over all 128 rows when nchains = 1.
+template <int G>
+__device__ __forceinline__ void qprime_chains(const float (&t)[kHeadDim], const float (*qs)[kHeadDim], int nchains,
+                                              float (&acc)[G]) {
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    if (nchains == 2) {
+      float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < kHeadDim / 2; ++i) p0 = fmaf(t[i], qs[hh][i], p0);
+#pragma unroll
+      for (int i = kHeadDim / 2; i < kHeadDim; ++i) p1 = fmaf(t[i], qs[hh][i], p1);
+      acc[hh] = p0 + p1;
+    } else {
+      float p0 = 0.f;
+#pragma unroll
+      for (int i = 0; i < kHeadDim; ++i) p0 = fmaf(t[i], qs[hh][i], p0);
+      acc[hh] = p0;
+    }
+  }
+}
+
+// Build the unit's fragments from q' (fp32 [G][128] in shared memory) with 128 threads
+// (tid = 0 .. 127, all of them calling; out 16-byte aligned).  red: shared scratch of 3 * 8
+// floats.  sync() is the barrier of those threads (a named barrier in a kernel whose other
+// threads do other work).  Per head, one warp reduces max |q'_d / scale_d| and the sum of
+// q' (lane l holds dimensions 4l .. 4l+3; xor-shuffle tree, a fixed order); then thread d
+// takes dimension d of every head: its fixed-point value, its four limbs, and the byte
+// each limb occupies in the fragment words (the inverse of frag_dim), which start zeroed.
 template <int BITS, int G, typename Sync>
 __device__ __forceinline__ void build_query_frags(const float (*qf)[kHeadDim], int tid, int nthr, float* red,
                                                   float scale_log2, uint8_t* out, Sync sync) {
   constexpr int NHS = GCfg<G>::NHS, NT = GCfg<G>::NT, FW = GCfg<G>::FW;
   float* amax_h = red;      // [G]
   float* sum_h = red + 8;   // [G]
+  float* rs_h = red + 16;   // [G]: 1 / sigma
   const int wl = tid & 31;
+  for (int i = tid; i < FW * 8; i += nthr) reinterpret_cast<uint4*>(out)[i] = make_uint4(0u, 0u, 0u, 0u);
   for (int hh = tid >> 5; hh < G; hh += nthr >> 5) {
     const float4 v = *reinterpret_cast<const float4*>(&qf[hh][4 * wl]);
     const float fv[4] = {v.x, v.y, v.z, v.w};
@@ -75,40 +104,48 @@ __device__ __forceinline__ void build_query_frags(const float (*qf)[kHeadDim], i
       sum += __shfl_xor_sync(0xffffffffu, sum, off);
     }
     if (wl == 0) {
+      const float sigma = amax > 0.f ? amax * (1.0f / kQMax) : 1.0f;
       amax_h[hh] = amax;
       sum_h[hh] = sum;
+      rs_h[hh] = 1.0f / sigma;
     }
   }
   sync();
-  uint32_t* words = reinterpret_cast<uint32_t*>(out);
-  for (int w = tid; w < FW * 32; w += nthr) {
-    const int idx = w >> 5, lane = w & 31;  // word idx of lane; idx = (j * NT + nt) * 2 + r
-    const int g = lane >> 2, t4 = lane & 3;
-    const int r = idx & 1, nt = (idx >> 1) % NT, j = (idx >> 1) / NT;
-    const int hh = 4 * (nt % NHS) + (g >> 1);
-    const int limb = 2 * (nt / NHS) + (g & 1);
-    uint32_t word = 0u;
-    if (hh < G) {
-      const float amax = amax_h[hh];
-      const float sigma = amax > 0.f ? amax / kQMax : 1.0f;
-      const float rs = 1.0f / sigma;
+  for (int dim = tid; dim < kHeadDim; dim += nthr) {
+    int j, r, t4, byte;
+    if (BITS == 2) {  // dim = 32*t4 + 16*r + 4*byte + j
+      j = dim & 3;
+      byte = (dim >> 2) & 3;
+      r = (dim >> 4) & 1;
+      t4 = dim >> 5;
+    } else {          // dim = 32*t4 + 8*(2*(j >> 1) + r) + 2*byte + (j & 1)
+      const int rem = dim & 31, w8 = rem >> 3;
+      t4 = dim >> 5;
+      byte = (rem >> 1) & 3;
+      j = 2 * (w8 >> 1) + (rem & 1);
+      r = w8 & 1;
+    }
+    const int l2s = BITS == 2 ? 2 * j : 4 * (j & 1);
+    const float unscale = __int_as_float((127 - l2s) << 23);  // 2^-l2s, exact
 #pragma unroll
-      for (int byte = 0; byte < 4; ++byte) {
-        int dim, l2s;
-        frag_dim<BITS>(j, r, t4, byte, dim, l2s);
-        const int Q = __float2int_rn(qf[hh][dim] * (rs / float(1 << l2s)));
-        // balanced base-256 digits, each in [-128, 127]
-        const int L0 = ((Q + 128) & 255) - 128;
-        const int Q1 = (Q - L0) >> 8;
-        const int L1 = ((Q1 + 128) & 255) - 128;
-        const int Q2 = (Q1 - L1) >> 8;
-        const int L2 = ((Q2 + 128) & 255) - 128;
-        const int L3 = (Q2 - L2) >> 8;
-        const int L = limb == 0 ? L0 : limb == 1 ? L1 : limb == 2 ? L2 : L3;
-        word |= (uint32_t)(L & 255) << (8 * byte);
+    for (int hh = 0; hh < G; ++hh) {
+      const int Q = __float2int_rn(qf[hh][dim] * (rs_h[hh] * unscale));
+      // balanced base-256 digits, each in [-128, 127]
+      int L[4];
+      L[0] = ((Q + 128) & 255) - 128;
+      const int Q1 = (Q - L[0]) >> 8;
+      L[1] = ((Q1 + 128) & 255) - 128;
+      const int Q2 = (Q1 - L[1]) >> 8;
+      L[2] = ((Q2 + 128) & 255) - 128;
+      L[3] = (Q2 - L[2]) >> 8;
+      const int hs = hh >> 2, hq = hh & 3;
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        const int nt = (l >> 1) * NHS + hs, g = 2 * hq + (l & 1);
+        const int lane = 4 * g + t4, idx = (j * NT + nt) * 2 + r;
+        out[(((idx >> 2) * 32 + lane) * 4 + (idx & 3)) * 4 + byte] = (uint8_t)(L[l] & 255);
       }
     }
-    words[((idx >> 2) * 32 + lane) * 4 + (idx & 3)] = word;
   }
   float* hc = reinterpret_cast<float*>(out + FW * 32 * 4);
   for (int i = tid; i < 16; i += nthr) {
@@ -119,7 +156,7 @@ __device__ __forceinline__ void build_query_frags(const float (*qf)[kHeadDim], i
         v = scale_log2 * sum_h[hh];
       } else {
         const float amax = amax_h[hh];
-        v = scale_log2 * (amax > 0.f ? amax / kQMax : 1.0f);
+        v = scale_log2 * (amax > 0.f ? amax * (1.0f / kQMax) : 1.0f);
       }
     }
     hc[i] = v;

@@ -117,7 +117,7 @@ typedef struct wushkv_layout {
   size_t ring_bytes;      /* each of k_ring, v_ring: fp16 [B][H_kv][ring_slots][128] */
   size_t state_bytes;     /* int32 [B*H_kv][2] = (S, S_quant) per (sequence, KV head), then the
                              status word; zero it to start from an empty cache */
-  size_t workspace_bytes; /* wushkv_decode_attn scratch; no initialisation needed */
+  size_t workspace_bytes; /* wushkv_decode_attn scratch; zero-fill it once before its first use */
   int32_t cap_alloc;      /* capacity rounded up to a multiple of 128 */
   int32_t ring_slots;     /* s_keep + s_flush - 1 + chunk_max; position p lives in slot p % ring_slots */
   int32_t code_bytes;     /* 128 * bits / 8 bytes of packed codes per token and head */
@@ -126,7 +126,8 @@ typedef struct wushkv_layout {
                              kernel splits each sequence's current length evenly among the
                              n_splits items, in whole multiples of 128) */
   int32_t code_order;     /* how the packed codes are ordered (WUSHKV_CODE_ORDER_*) */
-  size_t chunk_workspace_bytes; /* wushkv_chunk_attn scratch (no initialisation needed) */
+  size_t chunk_workspace_bytes; /* wushkv_chunk_attn scratch (zero-fill it once before its first use) */
+  int32_t decode_cluster; /* decode CTAs per thread-block cluster (1 or 2; divides n_splits) */
 } wushkv_layout;
 
 /* Device pointers of one layer's cache.
@@ -219,8 +220,10 @@ int wushkv_append(const wushkv_config* cfg, const wushkv_cache* cache, const voi
  * t_k_inv:  device fp32 [H_kv][128][128], T_K^{-1} row-major (see wushkv_compensation).
  * softmax_scale: logits are softmax_scale * q.k (1/sqrt(128) for standard attention).
  * out_fp16: 0 -> out is fp32 [B][H_q][128]; 1 -> fp16.
- * workspace: device scratch of layout.workspace_bytes (no initialisation needed; calls that
- *   share one workspace must not overlap in time).
+ * workspace: device scratch of layout.workspace_bytes.  Zero-fill it once before its first
+ *   use (cudaMemset): it holds the completion counters of the decode's last merge, which
+ *   every call leaves at zero again -- also a call that gave up on a wait.  Calls that
+ *   share one workspace must not overlap in time.
  * out[b][j] = sum_p softmax_p(softmax_scale * q'_j . khat_p) vhat_p over p < S, with
  *   q'_j = T_K^{-T} q_j, khat_p / vhat_p the stored fp16 k'/v in the windows and
  *   z + s*code in the quantized region.  S == 0 gives zeros and WUSHKV_STATUS_EMPTY.
@@ -252,7 +255,8 @@ int wushkv_step(const wushkv_config* cfg, const wushkv_cache* cache, const void*
  * S - n_q + t) sees positions 0 .. S - n_q + t.
  * q:   device fp16 [B][n_q][H_q][128] (after head-norm and RoPE); out: [B][n_q][H_q][128],
  *      fp32 or fp16 (out_fp16); t_k_inv, softmax_scale as in wushkv_decode_attn.
- * workspace: layout.chunk_workspace_bytes (no initialisation needed).
+ * workspace: layout.chunk_workspace_bytes, zero-filled once before its first use (as for
+ *   wushkv_decode_attn; the same buffer may serve both).
  * The chunk's queries share passes over the cache in blocks of up to 8 / g tokens.
  * Returns WUSHKV_OK, WUSHKV_EINVAL (also n_q < 1 or n_q > chunk_max), WUSHKV_EUNSUPPORTED
  * or WUSHKV_ECUDA. */
@@ -313,10 +317,11 @@ int wushkv_decode_attn_test_timeout(const wushkv_config* cfg, const wushkv_cache
  * Set-up: every call looks up the array's device address in the current CUDA context
  *   (cudaGetSymbolAddress, a host-side query).  The first call in a context may load the
  *   library's device module: make it before any stream capture in that context.
- * Sharing: all calls in a context share the one array.  Nothing in it needs clearing:
- *   the decode's first kernel resets the merge's completion counters on every call and
- *   every other byte is written before it is read.  Calls whose work overlaps in time
- *   (different streams, or threads without ordering) race on the array: serialise them. */
+ * Sharing: all calls in a context share the one array.  It starts zero-filled (a device
+ *   array of the module) and every call leaves the merge's completion counters in it at
+ *   zero again; every other byte is written before it is read.  Calls whose work overlaps
+ *   in time (different streams, or threads without ordering) race on the array: serialise
+ *   them. */
 int wushkv_decode_attn_static(const wushkv_config* cfg, const wushkv_cache* cache, const void* q,
                               const float* t_k_inv, float softmax_scale, int32_t out_fp16, void* out,
                               void* stream);

@@ -168,3 +168,21 @@ def test_binding_refuses_host_tensors(bnd):
     bnd._require_cuda(None)
     with pytest.raises(bnd.WushKVError, match="CUDA"):
         bnd._require_cuda(None, torch.zeros(1))
+
+
+def test_decode_split_policy(bnd):
+    """The decode's work split: n_split items per (sequence, KV head) filling the B200's
+    CTA slots (148 SMs, 4 CTAs each, 3 for 8 query heads per KV head), in clusters of two
+    consecutive items when n_split is even, never more than 128 items."""
+    from decode_attention_head_b200 import synth
+    expect = {"llama3-8b-layer": (9, 1), "qwen3-8b-layer": (74, 2), "mha-32l": (2, 2),
+              "prefill-append-decode": (13, 1), "tiny": (128, 2)}
+    for name, wl in synth.WORKLOADS.items():
+        L = bnd.pack_layout(bnd.config_for_workload(wl, extra_capacity=64))
+        assert (L.n_splits, L.decode_cluster) == expect[name], name
+    for B, Hkv, Hq in [(1, 1, 1), (1, 8, 64), (3, 8, 32), (16, 8, 32), (64, 32, 32), (256, 8, 8)]:
+        L = bnd.pack_layout(bnd.make_config(B, Hkv, Hq, 2, 4096, 4, 32, 16, 1))
+        slots = 148 * (3 if Hq // Hkv == 8 else 4)
+        assert 1 <= L.n_splits <= 128 and L.decode_cluster == (2 if L.n_splits % 2 == 0 else 1)
+        if B * Hkv * L.n_splits > slots:  # more than one wave only when one item per unit overfills it
+            assert L.n_splits <= 4

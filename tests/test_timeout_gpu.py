@@ -3,8 +3,9 @@
 wushkv_decode_attn_test_timeout shortens the decode kernel's wait limit and withholds the
 issue of one pipeline stage (the copy is never started, so no copy is in flight when a
 warp gives up).  The call must return, the status word must carry STATUS_TIMEOUT, no
-output row may be written (an aborted work item takes no part in the merge), and the next
-ordinary call on the same cache and workspace must be exact again.
+output row may be written (an aborted work item's cluster writes no output), the
+workspace's completion counters must be back at zero, and the next ordinary call on the
+same cache and workspace must be exact again.
 """
 import numpy as np
 import pytest
@@ -39,12 +40,16 @@ def test_withheld_stage_times_out_cleanly(bits, g):
     torch.cuda.synchronize()
     assert gc.status() & bnd.STATUS_TIMEOUT
     assert torch.isnan(out).all(), "an aborted call must not write plausible-looking output"
+    # the workspace's completion counters (its first 4 * units bytes) are back at zero: the
+    # next call needs no clearing
+    assert not gc.workspace[:4 * gc.units].any()
 
     gc.state[2 * gc.units] = 0  # clear the status word (after the (S, S_quant) pairs)
     again = gc.decode_attn(q, tinv, scale)
     torch.cuda.synchronize()
     assert gc.status() == 0
     assert torch.equal(again, ref)
+    assert not gc.workspace[:4 * gc.units].any()
 
 
 def test_hook_arguments_are_checked():
