@@ -22,8 +22,9 @@
 // head are n_heads * 256 bytes apart in memory).  One thread issues the four MMAs of a
 // slot and commits them to the slot's mbarrier; the slot is refilled only once they have
 // read it.  At the end the four warps read the sum back from tensor memory (warp w: rows
-// 32 w .. 32 w + 31) and add it into the fp64 Gram matrix with atomics: the entry (i, j),
-// i <= j, at both (i, j) and (j, i), so the result stays exactly symmetric.  A CTA's fp32
+// 32 w .. 32 w + 31) into a shared-memory tile and add it into the fp64 Gram matrix with
+// atomics, row by row with consecutive columns across a warp's lanes (coalesced): the entry
+// (i, j), i <= j, at both (i, j) and (j, i), the same value at both.  A CTA's fp32
 // sum covers at most kGramTokens tokens, which bounds its rounding error; the fp64 additions
 // across CTAs come in no fixed order.
 #include <algorithm>
@@ -42,7 +43,9 @@ constexpr int kGramStage = 64;                    // tokens per stage (four MMAs
 constexpr int kGramStages = 4;                    // ring slots
 constexpr int kGramRegion = kGramStage * 128;     // bytes of one 64-dimension half of a slot
 constexpr int kGramSlotBytes = 2 * kGramRegion;   // 16 KB
-constexpr int kGramSmem = kGramStages * kGramSlotBytes + 1024;  // + room to align to 1024
+constexpr int kGramPitch = kHeadDim + 1;         // floats per row of the read-back tile (no bank conflicts)
+static_assert(kHeadDim * kGramPitch * 4 <= kGramStages * kGramSlotBytes + 2048, "the read-back tile fits");
+constexpr int kGramSmem = kGramStages * kGramSlotBytes + 1024 + 2048;  // + room to align to 1024, + tile pitch
 constexpr uint32_t kGramTmemCols = 128;
 
 // kind::f16 with an fp32 accumulator, A and B fp16 and MN-major, M = N = 128.
@@ -150,26 +153,37 @@ __global__ void __launch_bounds__(kGramThreads)
     }
   }
   // every MMA complete (the last commit covers all of them), then the sum leaves tensor memory
+  // into a [128][129] fp32 tile over the drained slots (warp w: rows 32 w .. 32 w + 31)
   mbar_wait(&done[(n_stages - 1) % kGramStages], ((n_stages - 1) / kGramStages) & 1, &s_status);
   tc_fence_after();
-  double* G = gram + (size_t)h * kHeadDim * kHeadDim;
+  float* tile = reinterpret_cast<float*>(smem);
   const int i = 32 * warp + lane;  // this thread's row (tensor-memory lane)
 #pragma unroll 1
   for (int c = 0; c < kHeadDim / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + ((uint32_t)(32 * warp) << 16) + 32 * c, r);
-    if (32 * c + 31 < i) continue;  // only j >= i: the (j, i) entry gets the same value
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const int j = 32 * c + k;
-      if (j < i) continue;
-      const double v = (double)__uint_as_float(r[k]);
-      atomicAdd(G + i * kHeadDim + j, v);
-      if (j != i) atomicAdd(G + j * kHeadDim + i, v);
-    }
+    for (int k = 0; k < 32; ++k) tile[i * kGramPitch + 32 * c + k] = __uint_as_float(r[k]);
   }
   tc_fence_before();
   __syncthreads();
+  // G[r][c] += the CTA's (min(r, c), max(r, c)) entry, the same value at (r, c) and (c, r): a warp
+  // takes a row, its lanes 32 consecutive columns, so every fp64 atomic instruction covers
+  // 256 contiguous bytes
+  // (the CTAs of a head start at different rows, so that they do not all add into the same
+  // lines at the same time)
+  double* G = gram + (size_t)h * kHeadDim * kHeadDim;
+  const int shift = (int)((blockIdx.x * 8u) & (kHeadDim - 1));
+#pragma unroll 1
+  for (int r0 = warp; r0 < kHeadDim; r0 += kGramThreads / 32) {
+    const int row = (r0 + shift) & (kHeadDim - 1);
+#pragma unroll
+    for (int q = 0; q < kHeadDim / 32; ++q) {
+      const int col = 32 * q + lane;
+      const float v = col >= row ? tile[row * kGramPitch + col] : tile[col * kGramPitch + row];
+      atomicAdd(G + row * kHeadDim + col, (double)v);
+    }
+  }
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, kGramTmemCols);
