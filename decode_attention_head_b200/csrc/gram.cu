@@ -18,16 +18,19 @@
 //
 // Work split.  A CTA takes a run of at most kGramTokens consecutive tokens of one head; the
 // run length is chosen so that the grid fills two CTAs per SM when the input allows.  The
-// tokens arrive 64 at a time through a cp.async ring of kGramStages slots (the rows of one
-// head are n_heads * 256 bytes apart in memory).  One thread issues the four MMAs of a
-// slot and commits them to the slot's mbarrier; the slot is refilled only once they have
-// read it.  At the end the four warps read the sum back from tensor memory (warp w: rows
+// tokens arrive 64 at a time through a ring of kGramStages slots, each filled by two TMA
+// tile copies (a 3-D tensor map over [tokens][heads][128 dims], boxes of 64 dimensions x 1
+// head x 64 tokens, 128-byte swizzle: the copies write the MN-major layout above, and zero
+// past the last token).  One thread issues the copies, another the four MMAs of a slot,
+// which it commits to the slot's mbarrier; the slot is refilled only once they have read
+// it.  At the end the four warps read the sum back from tensor memory (warp w: rows
 // 32 w .. 32 w + 31) into a shared-memory tile and add it into the fp64 Gram matrix with
 // atomics, row by row with consecutive columns across a warp's lanes (coalesced): the entry
 // (i, j), i <= j, at both (i, j) and (j, i), the same value at both.  A CTA's fp32
 // sum covers at most kGramTokens tokens, which bounds its rounding error; the fp64 additions
 // across CTAs come in no fixed order.
 #include <algorithm>
+#include <cuda.h>  // CUtensorMap and its enums (the encoder is fetched through the runtime)
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -84,12 +87,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
+// One 3-D TMA tile copy (no multicast) into shared memory, completing on an mbarrier:
+// coordinates (dimension, head, token) of the box's first element.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __global__ void __launch_bounds__(kGramThreads)
-    gram_kernel(const uint16_t* __restrict__ x, int64_t n_tokens, int n_heads, int64_t cta_tokens,
+    gram_kernel(const __grid_constant__ CUtensorMap map, int64_t n_tokens, int64_t cta_tokens,
                 double* __restrict__ gram) {
   extern __shared__ uint8_t smem_raw[];
   // the swizzle pattern repeats every 1024 bytes: slots start on such a boundary
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t full[kGramStages];  // a slot's tokens have landed
   __shared__ __align__(8) uint64_t done[kGramStages];  // the MMAs that read a slot have completed
   __shared__ uint32_t s_taddr;
   __shared__ uint32_t s_status;  // the Gram call has no status word: a wait that gives up (a library bug) lands here
@@ -100,7 +114,10 @@ __global__ void __launch_bounds__(kGramThreads)
   const int n_stages = (int)((t_end - t_begin + kGramStage - 1) / kGramStage);
 
   if (tid == 0) {
-    for (int s = 0; s < kGramStages; ++s) mbar_init(&done[s], 1);
+    for (int s = 0; s < kGramStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&done[s], 1);
+    }
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&s_taddr, kGramTmemCols);
@@ -109,52 +126,49 @@ __global__ void __launch_bounds__(kGramThreads)
   tc_fence_after();
   const uint32_t tbase = s_taddr;
 
-  // Stage u (tokens t_begin + 64 u ...) into slot u % kGramStages, once the MMAs of stage
-  // u - kGramStages (the slot's previous user) have read it: 16-byte copies in the swizzled
-  // MN-major layout.  Rows past the run are zero-filled, so they add nothing.  One commit
-  // group per call, empty past the last stage.
-  auto issue_stage = [&](int u) {
-    if (u < n_stages) {
+  if (tid == 0) {
+    // producer: stage u (tokens t_begin + 64 u ...) into slot u % kGramStages once the MMAs
+    // of stage u - kGramStages (the slot's previous user) have read it.  Tokens past the
+    // run belong to the next CTA only where the run is a whole number of stages, so a
+    // partial stage exists only at the tensor's end, where the copy fills zeros.
+    int issued = 0;
+    for (int u = 0; u < n_stages; ++u) {
       const int slot = u % kGramStages;
-      if (u >= kGramStages) mbar_wait(&done[slot], ((u / kGramStages) - 1) & 1, &s_status);
+      if (u >= kGramStages && !mbar_wait(&done[slot], ((u / kGramStages) - 1) & 1, &s_status)) break;
       uint8_t* base = smem + slot * kGramSlotBytes;
-      const int64_t t0 = t_begin + (int64_t)u * kGramStage;
-      for (int i = tid; i < kGramStage * 16; i += kGramThreads) {
-        const int r = i >> 4, c = i & 15;
-        const int64_t t = t0 + r;
-        uint8_t* dst = base + (c >> 3) * kGramRegion + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-        if (t < t_end)
-          cp_async16(dst, x + (t * n_heads + h) * kHeadDim + 8 * c);
-        else
-          *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-      }
+      const int z = (int)(t_begin + (int64_t)u * kGramStage);
+      mbar_expect_tx(&full[slot], kGramSlotBytes);
+      tma_load_3d(base, &map, 0, h, z, &full[slot]);
+      tma_load_3d(base + kGramRegion, &map, 64, h, z, &full[slot]);
+      issued = u + 1;
     }
-    cp_async_commit();
-  };
-
-  // two stages of copies ahead of the MMAs; a slot is refilled two stages after its MMAs
-  // were issued, so their completion is rarely waited for
-  for (int u = 0; u < kGramStages - 2; ++u) issue_stage(u);
-  const uint32_t smem0 = smem_u32(smem);
-  for (int s = 0; s < n_stages; ++s) {
-    issue_stage(s + kGramStages - 2);
-    asm volatile("cp.async.wait_group %0;" ::"n"(kGramStages - 2) : "memory");  // stage s landed (this thread)
-    fence_async_smem();  // ... and is visible to the tensor core
-    __syncthreads();     // every thread's copies of stage s are in
-    if (tid == 0) {
+    // every issued copy has landed before the CTA may leave (they are plain reads of x)
+    for (int u = max(0, issued - kGramStages); u < issued; ++u)
+      mbar_wait(&full[u % kGramStages], (u / kGramStages) & 1, &s_status);
+  } else if (tid == 32) {
+    // MMA issue: four K = 16 slices of each slot, committed to the slot's `done`
+    const uint32_t smem0 = smem_u32(smem);
+    for (int s = 0; s < n_stages; ++s) {
+      const int slot = s % kGramStages;
+      if (!mbar_wait(&full[slot], (s / kGramStages) & 1, &s_status)) break;
       tc_fence_after();
-      const uint32_t slot = smem0 + (s % kGramStages) * kGramSlotBytes;
+      const uint32_t a = smem0 + slot * kGramSlotBytes;
 #pragma unroll
       for (int j = 0; j < kGramStage / 16; ++j) {
-        const uint64_t d = gram_desc(slot + j * 16 * 128);
+        const uint64_t d = gram_desc(a + j * 16 * 128);
         mma_f16_ss(tbase, d, d, kGramIdesc, (s > 0 || j > 0) ? 1u : 0u);
       }
-      mma_commit(&done[s % kGramStages]);
+      mma_commit(&done[slot]);
     }
   }
-  // every MMA complete (the last commit covers all of them), then the sum leaves tensor memory
-  // into a [128][129] fp32 tile over the drained slots (warp w: rows 32 w .. 32 w + 31)
-  mbar_wait(&done[(n_stages - 1) % kGramStages], ((n_stages - 1) / kGramStages) & 1, &s_status);
+  // every MMA complete (the last commit covers all of them; the MMA thread waits for it --
+  // a thread that had not followed the barrier's phases could not), then the sum leaves
+  // tensor memory into a [128][129] fp32 tile over the drained slots (warp w: rows 32 w ..
+  // 32 w + 31)
+  if (tid == 32 && n_stages > 0)
+    mbar_wait(&done[(n_stages - 1) % kGramStages], ((n_stages - 1) / kGramStages) & 1, &s_status);
+  tc_fence_before();
+  __syncthreads();
   tc_fence_after();
   float* tile = reinterpret_cast<float*>(smem);
   const int i = 32 * warp + lane;  // this thread's row (tensor-memory lane)
@@ -190,20 +204,57 @@ __global__ void __launch_bounds__(kGramThreads)
   }
 }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's cuTensorMapEncodeTiled, fetched through the runtime (no link against libcuda).
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
 }  // namespace
 
 cudaError_t launch_gram(const uint16_t* x, int64_t n_tokens, int n_heads, double* gram, cudaStream_t st) {
-  // Runs per head for two CTAs per SM, each a whole number of stages and at most kGramTokens.
-  const int64_t runs = std::max<int64_t>(1, (2 * kB200SMs + n_heads - 1) / n_heads);
-  int64_t cta_tokens = (n_tokens + runs - 1) / runs;
-  cta_tokens = (cta_tokens + kGramStage - 1) / kGramStage * kGramStage;
-  cta_tokens = std::min<int64_t>(std::max<int64_t>(cta_tokens, kGramStage), kGramTokens);
-  const int64_t chunks = (n_tokens + cta_tokens - 1) / cta_tokens;
-  const cudaError_t e = ensure_smem_attr<gram_kernel>(kGramSmem);
+  const EncodeTiledFn encode = encode_tiled();
+  if (!encode) return cudaErrorNotSupported;
+  cudaError_t e = ensure_smem_attr<gram_kernel>(kGramSmem);
   if (e != cudaSuccess) return e;
-  gram_kernel<<<dim3((unsigned)chunks, (unsigned)n_heads), kGramThreads, kGramSmem, st>>>(x, n_tokens, n_heads,
-                                                                                        cta_tokens, gram);
-  return cudaGetLastError();
+  // windows of at most 2^30 tokens (a tensor map's token coordinate is a 32-bit integer)
+  constexpr int64_t kWindow = int64_t(1) << 30;
+  for (int64_t w0 = 0; w0 < n_tokens; w0 += kWindow) {
+    const int64_t nw = std::min(kWindow, n_tokens - w0);
+    // runs per head for two CTAs per SM, each a whole number of stages and at most kGramTokens
+    const int64_t runs = std::max<int64_t>(1, (2 * kB200SMs + n_heads - 1) / n_heads);
+    int64_t cta_tokens = (nw + runs - 1) / runs;
+    cta_tokens = (cta_tokens + kGramStage - 1) / kGramStage * kGramStage;
+    cta_tokens = std::min<int64_t>(std::max<int64_t>(cta_tokens, kGramStage), kGramTokens);
+    const int64_t chunks = (nw + cta_tokens - 1) / cta_tokens;
+    // [tokens][heads][128] fp16: dimension fastest, then head, then token
+    CUtensorMap map;
+    const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)n_heads, (cuuint64_t)nw};
+    const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)n_heads * kHeadDim * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kGramStage};
+    const cuuint32_t estrides[3] = {1, 1, 1};
+    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+               const_cast<uint16_t*>(x + w0 * n_heads * kHeadDim), dims, strides, box, estrides,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    gram_kernel<<<dim3((unsigned)chunks, (unsigned)n_heads), kGramThreads, kGramSmem, st>>>(map, nw, cta_tokens,
+                                                                                          gram);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace wushkv

@@ -56,6 +56,15 @@ def test_integer_inputs_bit_exact(n):
     np.testing.assert_array_equal(got, ocal.gram(x))
 
 
+@pytest.mark.parametrize("heads,n", [(1, 80000), (3, 50000), (8, 40000)])
+def test_integer_inputs_long_runs_bit_exact(heads, n):
+    """Runs of 5 to 17 stages of 64 tokens per CTA: every slot of the copy ring is reused."""
+    rng = np.random.default_rng(n + heads)
+    x = rng.integers(-8, 9, size=(n, heads, 128)).astype(np.float16)  # |partial sums| <= 64 * 4096 < 2^24
+    got = _gpu_gram(x).cpu().numpy()
+    np.testing.assert_array_equal(got, ocal.gram(x))
+
+
 def test_single_token_is_exact_outer_product():
     rng = np.random.default_rng(3)
     x = (rng.standard_normal((1, 2, 128)) * 3).astype(np.float16)
