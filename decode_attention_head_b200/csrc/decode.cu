@@ -18,8 +18,9 @@
 //   * Stream: the quantized positions pass through shared memory in 128-position stages
 //     (K codes, V codes, K and V (s, z)) via bulk copies on an mbarrier ring: one producer
 //     warp, four consumer warps, 32 positions per consumer warp per stage.  The consumer
-//     warps take q' as a 31-bit fixed-point integer split into four signed 8-bit limbs,
-//     laid out as the mma.sync B fragments they need:
+//     warps take q' as a 31-bit fixed-point integer split into four signed 8-bit limbs
+//     (23-bit, three limbs, for eight query heads per KV head), laid out as the mma.sync B
+//     fragments they need:
 //       QK  : u8 codes x s8 query limbs on tensor cores (mma m16n8k32, exact int32),
 //             logit = log2e*scale*(z*sum(q') + s*sigma*D)  (dequantization folded);
 //       softmax: online, base 2, with a running max that may go stale by 2^8;
@@ -306,7 +307,12 @@ __device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, 
       for (int u = 0; u < 2; ++u) {
         // q'.c / sigma = sum_l 256^l D_l; pairs of limbs combine exactly in int32
         const int d01 = acc[i][hs][2 * u] + 256 * acc[i][hs][2 * u + 1];
-        const int d23 = acc[i][NHS + hs][2 * u] + 256 * acc[i][NHS + hs][2 * u + 1];
+        // limbs 2 and 3; with three limbs limb 2 alone, in n-tile 2 column 2 t4 + hs
+        int d23;
+        if constexpr (GCfg<G>::LIMBS == 4)
+          d23 = acc[i][NHS + hs][2 * u] + 256 * acc[i][NHS + hs][2 * u + 1];
+        else
+          d23 = acc[i][NT - 1][2 * u + hs];
         const float f = fmaf(65536.0f, (float)d23, (float)d01);
         const float xv = fmaf(Bh[hs] * ksz[i][u].x, f, Ah[hs] * ksz[i][u].y);
         x[i][u][hs] = (val[i][u] && hvalid[hs]) ? xv : -CUDART_INF_F;

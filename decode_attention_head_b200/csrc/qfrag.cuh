@@ -9,22 +9,29 @@
 // Those digits are laid out as the mma.sync m16n8k32 B fragments of the consumer warps:
 // lane (g, t4) holds, for k-step j, n-tile nt and register r, the four bytes = limb
 // 2*(nt / NHS) + (g & 1) of head 4*(nt % NHS) + (g >> 1) at the four dimensions that its
-// key-code register carries.  The fragments are built once per (sequence, KV head) -- by
-// the decode prologue, or by the fused append of a decode step -- and every work item of
-// the unit loads them as they are.
+// key-code register carries.  With eight query heads per KV head the query takes three
+// limbs instead (sigma = max / 2^22, a 23-bit fixed point): n-tiles 0 and 1 hold limbs 0
+// and 1 of heads 0..3 and 4..7 as above, n-tile 2 holds limb 2 of all eight, column g
+// belonging to head (g >> 1) + 4 (g & 1) -- so that the lane that holds a head's limbs 0
+// and 1 in its accumulator also holds its limb 2 -- and each slice issues 24 QK MMAs
+// instead of 32.  The fragments are built once per (sequence, KV head) -- by the decode's
+// query kernel, or by the fused append of a decode step -- and every work item of the unit
+// loads them as they are.
 #pragma once
 #include <cstdint>
 #include "internal.h"
 
 namespace wushkv {
 
-constexpr float kQMax = 1073741824.0f;  // |fixed-point query| <= 2^30; four signed 8-bit limbs hold +-2.1e9
-
 template <int G>
 struct GCfg {
   static constexpr int NHS = G <= 4 ? 1 : 2;  // head sets handled per lane
-  static constexpr int NT = 2 * NHS;          // QK n-tiles: limbs {0,1} then {2,3} per head set
+  static constexpr int LIMBS = G <= 4 ? 4 : 3;  // signed 8-bit limbs of the fixed-point query
+  // QK n-tiles: limbs {0,1} then {2,3} per head set; three limbs: {0,1} per head set, then limb 2
+  static constexpr int NT = LIMBS == 4 ? 2 * NHS : 3;
   static constexpr int FW = 4 * NT * 2;       // fragment words per lane: [k-step][n-tile][reg]
+  // |fixed-point query| bound: four limbs hold +-2.1e9, three +-8.4e6
+  static constexpr float QMAX = LIMBS == 4 ? 1073741824.0f : 4194304.0f;
 };
 
 // Per-unit layout of the fragments in the decode workspace: FW/4 uint4 per lane stored as
@@ -104,7 +111,7 @@ __device__ __forceinline__ void build_query_frags(const float (*qf)[kHeadDim], i
       sum += __shfl_xor_sync(0xffffffffu, sum, off);
     }
     if (wl == 0) {
-      const float sigma = amax > 0.f ? amax * (1.0f / kQMax) : 1.0f;
+      const float sigma = amax > 0.f ? amax * (1.0f / GCfg<G>::QMAX) : 1.0f;
       amax_h[hh] = amax;
       sum_h[hh] = sum;
       rs_h[hh] = 1.0f / sigma;
@@ -130,18 +137,20 @@ __device__ __forceinline__ void build_query_frags(const float (*qf)[kHeadDim], i
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
       const int Q = __float2int_rn(qf[hh][dim] * (rs_h[hh] * unscale));
-      // balanced base-256 digits, each in [-128, 127]
+      // balanced base-256 digits, each in [-128, 127] (with three limbs the top one is the
+      // rest, |Q2| <= 64)
       int L[4];
       L[0] = ((Q + 128) & 255) - 128;
       const int Q1 = (Q - L[0]) >> 8;
       L[1] = ((Q1 + 128) & 255) - 128;
       const int Q2 = (Q1 - L[1]) >> 8;
-      L[2] = ((Q2 + 128) & 255) - 128;
+      L[2] = GCfg<G>::LIMBS == 4 ? ((Q2 + 128) & 255) - 128 : Q2;
       L[3] = (Q2 - L[2]) >> 8;
       const int hs = hh >> 2, hq = hh & 3;
 #pragma unroll
-      for (int l = 0; l < 4; ++l) {
-        const int nt = (l >> 1) * NHS + hs, g = 2 * hq + (l & 1);
+      for (int l = 0; l < GCfg<G>::LIMBS; ++l) {
+        const bool top3 = GCfg<G>::LIMBS == 3 && l == 2;  // n-tile 2: column 2 hq + hs
+        const int nt = top3 ? 2 : (l >> 1) * NHS + hs, g = top3 ? 2 * hq + hs : 2 * hq + (l & 1);
         const int lane = 4 * g + t4, idx = (j * NT + nt) * 2 + r;
         out[(((idx >> 2) * 32 + lane) * 4 + (idx & 3)) * 4 + byte] = (uint8_t)(L[l] & 255);
       }
@@ -156,7 +165,7 @@ __device__ __forceinline__ void build_query_frags(const float (*qf)[kHeadDim], i
         v = scale_log2 * sum_h[hh];
       } else {
         const float amax = amax_h[hh];
-        v = scale_log2 * (amax > 0.f ? amax * (1.0f / kQMax) : 1.0f);
+        v = scale_log2 * (amax > 0.f ? amax * (1.0f / GCfg<G>::QMAX) : 1.0f);
       }
     }
     hc[i] = v;
