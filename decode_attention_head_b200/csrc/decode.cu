@@ -307,9 +307,12 @@ __device__ __forceinline__ void slice(const uint8_t* __restrict__ st, int base, 
       for (int u = 0; u < 2; ++u) {
         // q'.c / sigma = sum_l 256^l D_l; pairs of limbs combine exactly in int32
         const int d01 = acc[i][hs][2 * u] + 256 * acc[i][hs][2 * u + 1];
-        // limbs 2 and 3; with three limbs limb 2 alone, in n-tile 2 column 2 t4 + hs
+        // limbs 2 and 3; with three limbs limb 2 alone, in n-tile 2 column 2 t4 + hs; with one
+        // query head, the next lane's pair (t4 = 1 holds limbs 2 and 3 of the head at t4 = 0)
         int d23;
-        if constexpr (GCfg<G>::LIMBS == 4)
+        if constexpr (G == 1)
+          d23 = __shfl_xor_sync(0xffffffffu, d01, 1);
+        else if constexpr (GCfg<G>::LIMBS == 4)
           d23 = acc[i][NHS + hs][2 * u] + 256 * acc[i][NHS + hs][2 * u + 1];
         else
           d23 = acc[i][NT - 1][2 * u + hs];

@@ -14,7 +14,9 @@
 // and 1 of heads 0..3 and 4..7 as above, n-tile 2 holds limb 2 of all eight, column g
 // belonging to head (g >> 1) + 4 (g & 1) -- so that the lane that holds a head's limbs 0
 // and 1 in its accumulator also holds its limb 2 -- and each slice issues 24 QK MMAs
-// instead of 32.  The fragments are built once per (sequence, KV head) -- by the decode's
+// instead of 32.  With one query head per KV head a single n-tile holds its four limbs in
+// columns 0..3 (lane t4 = 0 gets limbs 0 and 1 in its accumulator, lane t4 = 1 limbs 2 and
+// 3, combined by one shuffle): 8 QK MMAs per slice instead of 16.  The fragments are built once per (sequence, KV head) -- by the decode's
 // query kernel, or by the fused append of a decode step -- and every work item of the unit
 // loads them as they are.
 #pragma once
@@ -27,8 +29,9 @@ template <int G>
 struct GCfg {
   static constexpr int NHS = G <= 4 ? 1 : 2;  // head sets handled per lane
   static constexpr int LIMBS = G <= 4 ? 4 : 3;  // signed 8-bit limbs of the fixed-point query
-  // QK n-tiles: limbs {0,1} then {2,3} per head set; three limbs: {0,1} per head set, then limb 2
-  static constexpr int NT = LIMBS == 4 ? 2 * NHS : 3;
+  // QK n-tiles: limbs {0,1} then {2,3} per head set; three limbs: {0,1} per head set, then
+  // limb 2; one query head: its four limbs in columns 0..3 of a single n-tile
+  static constexpr int NT = G == 1 ? 1 : LIMBS == 4 ? 2 * NHS : 3;
   static constexpr int FW = 4 * NT * 2;       // fragment words per lane: [k-step][n-tile][reg]
   // |fixed-point query| bound: four limbs hold +-2.1e9, three +-8.4e6
   static constexpr float QMAX = LIMBS == 4 ? 1073741824.0f : 4194304.0f;
@@ -150,7 +153,8 @@ __device__ __forceinline__ void build_query_frags(const float (*qf)[kHeadDim], i
 #pragma unroll
       for (int l = 0; l < GCfg<G>::LIMBS; ++l) {
         const bool top3 = GCfg<G>::LIMBS == 3 && l == 2;  // n-tile 2: column 2 hq + hs
-        const int nt = top3 ? 2 : (l >> 1) * NHS + hs, g = top3 ? 2 * hq + hs : 2 * hq + (l & 1);
+        const int nt = G == 1 ? 0 : top3 ? 2 : (l >> 1) * NHS + hs;
+        const int g = G == 1 ? l : top3 ? 2 * hq + hs : 2 * hq + (l & 1);
         const int lane = 4 * g + t4, idx = (j * NT + nt) * 2 + r;
         out[(((idx >> 2) * 32 + lane) * 4 + (idx & 3)) * 4 + byte] = (uint8_t)(L[l] & 255);
       }
