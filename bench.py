@@ -410,6 +410,12 @@ def run_gpu(args, rank, world, local_rank):
         for c in range(L):
             caches[c].step(k_pool[c % P], v_pool[c % P], tks[c], q_pool[c % P], tinvs[c], scale, out=outs[c],
                            stream=stream)
+    # the decode calls alone, all L layers in one graph (the roofline's kernel duration: the
+    # graph launch is shared by L calls; the decode leaves the caches unchanged)
+    g_dec_all = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_dec_all, stream=stream):
+        for c in range(L):
+            caches[c].decode_attn(q_pool[c % P], tinvs[c], scale, out=outs[c], stream=stream)
     # capture does not execute; the state mirrors stay in step with the device state
 
     def step_graphs(n, first):
@@ -474,9 +480,20 @@ def run_gpu(args, rank, world, local_rank):
     with torch.cuda.stream(stream):
         split_graphs(K2, first2, evs)
     stream.synchronize()
+    R3 = max(K2 // L, 3)
+    evs3 = [torch.cuda.Event(enable_timing=True) for _ in range(R3 + 1)]
+    with torch.cuda.stream(stream):
+        g_dec_all.replay()
+        for j in range(R3):
+            evs3[j].record(stream)
+            g_dec_all.replay()
+        evs3[R3].record(stream)
+    stream.synchronize()
     clocks = sampler.stop()
     dec_ms = [evs[2 * j + 1].elapsed_time(evs[2 * j + 2]) for j in range(K2)]
     app_ms = [evs[2 * j].elapsed_time(evs[2 * j + 1]) for j in range(K2)]
+    dec_all_ms = [evs3[j].elapsed_time(evs3[j + 1]) for j in range(R3)]
+    dec_all_bytes = sum(mirrors[c].decode_bytes() for c in range(L))
     k2_app_bytes, k2_dec_bytes = 0, 0
     for j in range(K2):
         c = (first2 + j) % L
@@ -485,8 +502,8 @@ def run_gpu(args, rank, world, local_rank):
     status = [cch.status() for cch in caches]
     assert all(s == 0 for s in status), status
 
-    t_total, dec_total, app_total = max_over_ranks([t_total_ms / 1e3, sum(dec_ms) / 1e3, sum(app_ms) / 1e3], dev,
-                                                   world)
+    t_total, dec_total, app_total, dec_all_total = max_over_ranks(
+        [t_total_ms / 1e3, sum(dec_ms) / 1e3, sum(app_ms) / 1e3, sum(dec_all_ms) / 1e3], dev, world)
 
     # ---- end to end through the public API: pinned host inputs in, result out, every step.
     # Per layer step: one host->device copy of that step's k, v and q (packed in one pinned
@@ -567,9 +584,11 @@ def run_gpu(args, rank, world, local_rank):
 
     peak, peak_kind = measured_peaks()
     traffic, traffic_why = profile_traffic(wl.name)
-    dec_launch_s = dec_total / K2
-    dec_bytes_per_launch = k2_dec_bytes / K2
+    # the roofline's kernel duration: the decode calls of all layers in one graph, per call
+    dec_launch_s = dec_all_total / (R3 * L)
+    dec_bytes_per_launch = dec_all_bytes / L
     achieved = dec_bytes_per_launch / dec_launch_s / 1e9
+    own_graph_s = dec_total / K2  # the same call as a graph of its own (its launch unshared)
     total_bytes = step_app_bytes + step_dec_bytes
     value = job_throughput(world, total_bytes, t_total)
     result = {
@@ -593,13 +612,17 @@ def run_gpu(args, rank, world, local_rank):
             "launch": "one CUDA graph per model decode step: wushkv_step (append fused with decode) of "
                       "each rotated layer in turn; per-layer graphs where K does not fill a whole step",
             "per_kernel_timing": "append and decode as separate calls, events per launch, "
-                                 "min(K, 4000) more steps of the same workload",
+                                 "min(K, 4000) more steps of the same workload; the roofline's decode "
+                                 "duration from a graph of the decode calls of all layers (events per "
+                                 "replay, per call = replay time / layers)",
             "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
         },
         "decode_attn_gbs": round(achieved, 2),
         "decode_pct_of_measured_hbm": round(100 * achieved / peak, 2),
         "decode_pct_of_8tbps": round(100 * achieved / NOMINAL_HBM_GBS, 2),
         "decode_us_per_launch": round(dec_launch_s * 1e6, 3),
+        "decode_us_per_launch_own_graph": round(own_graph_s * 1e6, 3),
+        "decode_gbs_own_graph": round(k2_dec_bytes / K2 / own_graph_s / 1e9, 2),
         "append_gbs": round(k2_app_bytes / app_total / 1e9, 2),
         "append_us_per_launch": round(app_total / K2 * 1e6, 3),
         "layer_tokens_per_s": round(world * wl.batch * K / t_total, 1),
@@ -614,7 +637,7 @@ def run_gpu(args, rank, world, local_rank):
         "e2e": e2e,
     }
     # release graphs before the process group goes away
-    del g_step, g_app, g_dec
+    del g_step, g_app, g_dec, g_dec_all
     if not args.no_prefill:
         del caches, outs
         torch.cuda.empty_cache()
