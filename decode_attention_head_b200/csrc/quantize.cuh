@@ -216,10 +216,32 @@ __device__ __forceinline__ void quantize_row_part(const __half* __restrict__ x, 
     a[j] = pinf;
     b[j] = ninf;
   }
+  // Pairs of values first: of each pair (v[2m], v[2m+1]) only the smaller can be among the
+  // NSEL smallest unless its partner is too, so at most NSEL / 2 pair maxima are among them
+  // (and at most NSEL / 2 pair minima among the NSEL largest).  The minima go through the
+  // NSEL-list of the smallest and the maxima through an (NSEL / 2)-list, and the other way
+  // round for the largest; the short lists join the long ones at the end.  Exact, with 3.5
+  // instead of 5 min / max per value for NSEL = 3.
+  constexpr int NB = NSEL / 2;
+  __half2 a2[NB], b2[NB];
 #pragma unroll
-  for (int i = 0; i < H; ++i) {
-    insert_small<NSEL>(a, v[i]);
-    insert_large<NSEL>(b, v[i]);
+  for (int j = 0; j < NB; ++j) {
+    a2[j] = pinf;
+    b2[j] = ninf;
+  }
+  static_assert(H % 2 == 0, "values come in pairs of half2");
+#pragma unroll
+  for (int i = 0; i < H; i += 2) {
+    const __half2 lo = __hmin2(v[i], v[i + 1]), hi = __hmax2(v[i], v[i + 1]);
+    insert_small<NSEL>(a, lo);
+    insert_large<NSEL>(b, hi);
+    insert_small<NB>(a2, hi);
+    insert_large<NB>(b2, lo);
+  }
+#pragma unroll
+  for (int j = 0; j < NB; ++j) {
+    insert_small<NSEL>(a, a2[j]);
+    insert_large<NSEL>(b, b2[j]);
   }
   float lo_s[NSEL], lo_t[NSEL], hi_s[NSEL], hi_t[NSEL];
 #pragma unroll
