@@ -287,17 +287,25 @@ __device__ __forceinline__ void quantize_row_part(const __half* __restrict__ x, 
 #pragma unroll
   for (int i = 0; i < NW; ++i) w[i] = 0u;
   if (sf != 0.0f && BITS == 2) {
-    // code = #{k : x >= X_k}, three half2 comparisons per pair of values; 1024 + code is
-    // exact in fp16 and leaves the code in the half's low bits
+    // code = #{k : x >= X_k}, three half2 comparison masks per pair of values.  The masks are
+    // nested (X_1 <= X_2 <= X_3), so the code's bit 1 is the second mask and its bit 0 is
+    // (m1 & ~m2) | m3; four pairs' bits are gathered in one word (values 2k at bits 4j,
+    // 4j + 1 of the low half, values 2k + 1 in the high half) and folded into 16 code bits.
     const __half2 x1 = __half2half2(code_threshold(1, sf, zf));
     const __half2 x2 = __half2half2(code_threshold(2, sf, zf));
     const __half2 x3 = __half2half2(code_threshold(3, sf, zf));
-    const __half2 k1024 = __float2half2_rn(1024.0f);
+    static_assert(H % 4 == 0, "four pairs per gathered word");
 #pragma unroll
-    for (int k = 0; k < H; ++k) {
-      const __half2 c = __hadd2(__hadd2(__hge2(v[k], x1), __hge2(v[k], x2)), __hadd2(__hge2(v[k], x3), k1024));
-      const uint32_t u = h2_as_u32(c);
-      w[k / 8] |= ((u & 3u) | ((u >> 14) & 0xCu)) << (4 * (k % 8));
+    for (int k0 = 0; k0 < H; k0 += 4) {
+      uint32_t u = 0u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t m1 = __hge2_mask(v[k0 + j], x1), m2 = __hge2_mask(v[k0 + j], x2);
+        const uint32_t m3 = __hge2_mask(v[k0 + j], x3);
+        const uint32_t b0 = (m1 & ~m2) | m3;
+        u |= ((b0 & 0x00010001u) | (m2 & 0x00020002u)) << (4 * j);
+      }
+      w[k0 / 8] |= ((u | (u >> 14)) & 0xFFFFu) << (16 * ((k0 / 4) & 1));
     }
   } else if (sf != 0.0f) {
     const float rcp = __frcp_rn(sf);
