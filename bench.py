@@ -54,6 +54,8 @@ def parse_args():
                    help="only the prefill workload's bulk append + decode measurement (one JSON line)")
     p.add_argument("--decode-only", action="store_true",
                    help="only the graph-timed decode calls of the 128K and MHA workloads (one JSON line each)")
+    p.add_argument("--chunk-only", action="store_true",
+                   help="only the chunked-prefill measurement on the Llama-3-8B layer (one JSON line)")
     return p.parse_args()
 
 
@@ -826,8 +828,9 @@ def workload_config(wl):
 def measure_chunk(bnd, synth, dev, n=8, reps=20):
     """Chunked prefill on the Llama-3-8B-shaped layer: an n-token chunk appended to a cache of
     32,768 - n positions (the decode-time append path), then its n queries attending
-    causally (wushkv_chunk_attn: ng = 8 / g tokens per pass over the cache).  Repeated from
-    the same state, each timed with CUDA events."""
+    causally (wushkv_chunk_attn: blocks of ng = 8 / g tokens, whose query heads share the
+    per-position work; the blocks run side by side in one launch pair, each streaming the
+    cache).  Repeated from the same state, each timed with CUDA events."""
     import torch
     wl = synth.WORKLOADS["llama3-8b-layer"]
     base = wl.context - n
@@ -867,13 +870,16 @@ def measure_chunk(bnd, synth, dev, n=8, reps=20):
     app_s = sum(app_ms) / len(app_ms) / 1e3
     S1, Sq1 = (int(t[0, 0].item()) for t in c.lengths())
     ng = max(1, 8 // wl.group)
-    passes = (n + ng - 1) // ng
+    blocks = (n + ng - 1) // ng
     cache_bytes = StateMirror(wl, S1, Sq1).decode_bytes()
     return {"workload": wl.name, "chunk_tokens": n, "cached_before": base,
             "append_us": round(app_s * 1e6, 2), "chunk_attn_us": round(att_s * 1e6, 2),
-            "passes_over_cache": passes, "chunk_attn_gbs": round(passes * cache_bytes / att_s / 1e9, 2),
+            "blocks": blocks, "cache_bytes": cache_bytes,
+            "chunk_attn_gbs": round(blocks * cache_bytes / att_s / 1e9, 2),
             "query_tokens_per_s": round(wl.batch * n / (app_s + att_s), 1),
-            "launch": "eager: 1 append launch + 1 decode launch per pass", "reps": reps}
+            "launch": "eager: 1 append launch, then 1 launch pair (query + main kernel) whose grid "
+                      "holds the %d blocks side by side; chunk_attn_gbs counts the cache once per "
+                      "block" % blocks, "reps": reps}
 
 
 def measure_gram(bnd, synth, dev, n_seq=4, seq_len=32768, reps=10):
@@ -969,6 +975,15 @@ def main():
         torch.cuda.set_device(dev)
         for name, layers in DECODE_WORKLOADS:
             print(json.dumps(measure_decode(bnd, synth, dev, name, layers)), flush=True)
+        return 0
+    if args.chunk_only:
+        from decode_attention_head_b200 import binding as bnd
+        from decode_attention_head_b200 import build as _build
+        from decode_attention_head_b200 import synth
+        _build.build()
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        print(json.dumps(measure_chunk(bnd, synth, dev)))
         return 0
     if args.prefill_only:
         from decode_attention_head_b200 import binding as bnd

@@ -16,7 +16,17 @@ namespace wushkv {
 static inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 static inline size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 
-int derive(const wushkv_config* cfg, Derived* d) {
+// Chunk attention runs up to this many blocks of chunk tokens in one launch, as that many
+// virtual units per cache unit (and never more virtual units than a grid column holds).
+constexpr int kMaxPasses = 32;
+static int max_passes(const wushkv_config* cfg, long long units) {
+  long long p = kMaxPasses;
+  if (cfg->chunk_max < p) p = cfg->chunk_max;
+  if (65535 / units < p) p = 65535 / units;
+  return p < 1 ? 1 : (int)p;
+}
+
+int derive(const wushkv_config* cfg, Derived* d, long long ticket_units) {
   if (!cfg || !d) return WUSHKV_EINVAL;
   if (cfg->head_dim != kHeadDim) return WUSHKV_EUNSUPPORTED;
   if (cfg->bits != 2 && cfg->bits != 4) return WUSHKV_EUNSUPPORTED;
@@ -90,8 +100,12 @@ int derive(const wushkv_config* cfg, Derived* d) {
   d->ring_bytes = U * (size_t)d->ring * kHeadDim * 2;
   d->state_bytes = round_up((2 * U + 1) * 4, 16);
   size_t off = 0;
-  d->ws_tickets = off;  // unit counters (zero between calls)
-  off = round_up(off + U * 4, 256);
+  // unit counters (zero between calls): one per virtual unit of the largest chunk-attention
+  // launch, in every layout, so that decode, step and chunk calls may share one workspace --
+  // no call writes anything but zeros into another call's counters
+  if (ticket_units < 0) ticket_units = (long long)U * max_passes(cfg, (long long)U);
+  d->ws_tickets = off;
+  off = round_up(off + (size_t)ticket_units * 4, 256);
   d->ws_qprime = off;
   off = round_up(off + U * g * kHeadDim * 4, 256);
   d->ws_qfrag = off;
@@ -114,7 +128,7 @@ static bool cache_ok(const wushkv_cache* c) {
 
 using namespace wushkv;
 
-// Largest power of two ng with ng * g <= 8 and ng <= n: the chunk tokens one launch of
+// Largest power of two ng with ng * g <= 8 and ng <= n: the chunk tokens one block of
 // chunk attention takes (as ng * g query heads per KV head).
 static int chunk_block(int g, int n) {
   int ng = 1;
@@ -122,20 +136,46 @@ static int chunk_block(int g, int n) {
   return ng;
 }
 
-// The decode derivation for a launch of chunk attention over ng tokens.
-static int derive_chunk(const wushkv_config* cfg, int ng, Derived* d) {
+// The decode derivation for a launch of chunk attention over np blocks of ng tokens: the
+// query heads per KV head of one block, and np virtual units per cache unit (passed to the
+// split policy and the workspace layout as np times the batch).
+static int derive_chunk(const wushkv_config* cfg, int ng, int np, Derived* d) {
   wushkv_config c2 = *cfg;
   c2.n_q_heads = cfg->n_kv_heads * (cfg->n_q_heads / cfg->n_kv_heads) * ng;
-  return derive(&c2, d);
+  c2.batch = cfg->batch * np;
+  const long long units = (long long)cfg->batch * cfg->n_kv_heads;
+  return derive(&c2, d, units * max_passes(cfg, units));
 }
 
-// Workspace of wushkv_chunk_attn: the largest any of its launches needs.
+// The launches of chunk attention over the chunk tokens [t0, n): the first takes the whole
+// blocks of the largest size that fits, up to kMaxPasses of them (and no more virtual units
+// than a grid column holds), all in one grid -- their passes over the cache run side by side,
+// so the blocks of a unit read each stage at about the same time; what is left takes the
+// next launch, and so on.
+static void chunk_launch(int g, int units, int n, int t0, int* ng, int* np) {
+  *ng = chunk_block(g, n - t0);
+  int p = (n - t0) / *ng;
+  const int grid_cap = 65535 / units > 1 ? 65535 / units : 1;
+  if (p > kMaxPasses) p = kMaxPasses;
+  if (p > grid_cap) p = grid_cap;
+  *np = p;
+}
+
+// Workspace of wushkv_chunk_attn: the largest any of its launches needs, over every chunk
+// length up to chunk_max (lengths above (kMaxPasses + 1) * 8 repeat launches of shorter ones).
 static size_t chunk_workspace(const wushkv_config* cfg) {
   const int g = cfg->n_q_heads / cfg->n_kv_heads;
+  const int units = cfg->batch * cfg->n_kv_heads;
+  const int nmax = cfg->chunk_max < (kMaxPasses + 1) * 8 ? cfg->chunk_max : (kMaxPasses + 1) * 8;
   size_t best = 0;
-  for (int n = 1; n <= cfg->chunk_max && n <= 8; n *= 2) {
-    Derived d;
-    if (derive_chunk(cfg, chunk_block(g, n), &d) == WUSHKV_OK && d.ws_total > best) best = d.ws_total;
+  for (int n = 1; n <= nmax; ++n) {
+    for (int t0 = 0; t0 < n;) {
+      int ng, np;
+      chunk_launch(g, units, n, t0, &ng, &np);
+      Derived d;
+      if (derive_chunk(cfg, ng, np, &d) == WUSHKV_OK && d.ws_total > best) best = d.ws_total;
+      t0 += ng * np;
+    }
   }
   return best;
 }
@@ -285,6 +325,7 @@ static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv
   a->gq = d.group;
   a->chunk_n = 0;
   a->chunk_t0 = 0;
+  a->npass = 1;
   a->withhold_tile = -1;
   a->wait_limit = kWaitLimitCycles;
 }
@@ -453,22 +494,27 @@ extern "C" int wushkv_chunk_attn(const wushkv_config* cfg, const wushkv_cache* c
   rc = check_decode(cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace);
   if (rc != WUSHKV_OK) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // blocks of ng tokens, each one launch pair whose ng * g query heads per KV head share
-  // one pass over the cache
+  // blocks of ng tokens (ng * g query heads per KV head share one pass over the cache); one
+  // launch pair takes np blocks as np virtual units per cache unit
   for (int t0 = 0; t0 < n_q;) {
-    const int ng = chunk_block(d.group, n_q - t0);
+    int ng, np;
+    chunk_launch(d.group, d.units, n_q, t0, &ng, &np);
     Derived d2;
-    rc = derive_chunk(cfg, ng, &d2);
+    rc = derive_chunk(cfg, ng, np, &d2);
     if (rc != WUSHKV_OK) return rc;
     DecodeArgs a;
     fill_decode(cfg, d2, cache, q, t_k_inv, softmax_scale, out_fp16, out, workspace, &a);
+    a.B = cfg->batch;  // the cache's units, not the virtual ones
+    a.units = d.units;
+    a.status = reinterpret_cast<uint32_t*>(cache->state + 2 * (size_t)d.units);
     a.Hq = cfg->n_q_heads;
     a.gq = d.group;
     a.chunk_n = n_q;
     a.chunk_t0 = t0;
+    a.npass = np;
     const cudaError_t e = launch_decode(d2, cfg->bits, a, st);
     if (e != cudaSuccess) return WUSHKV_ECUDA;
-    t0 += ng;
+    t0 += ng * np;
   }
   return WUSHKV_OK;
 }

@@ -73,12 +73,21 @@ __device__ __forceinline__ float ex2(float x) {  // 2^x (hardware approximation,
 
 
 // Row (in units of 128 elements) of query head v (0..G-1) of unit (b, h) in q and out: a
-// one-token decode has its G heads side by side; chunk attention's v is token v / gq of the
-// launch's block of the chunk, head v % gq.
-__device__ __forceinline__ size_t head_row(const DecodeArgs& a, int b, int h, int v) {
+// one-token decode has its G heads side by side; chunk attention's v is token t0 + v / gq
+// of the chunk (t0: the first token of the virtual unit's block), head v % gq.
+__device__ __forceinline__ size_t head_row(const DecodeArgs& a, int b, int h, int t0, int v) {
   const int t = v / a.gq, hh = v - t * a.gq;
   const int ntok = a.chunk_n > 0 ? a.chunk_n : 1;
-  return ((size_t)b * ntok + a.chunk_t0 + t) * a.Hq + (size_t)h * a.gq + hh;
+  return ((size_t)b * ntok + t0 + t) * a.Hq + (size_t)h * a.gq + hh;
+}
+
+// Virtual unit vu of a launch (a grid row): its cache unit (sequence, KV head) and the first
+// chunk token of its block (chunk attention takes npass blocks of G / gq tokens per launch;
+// npass = 1 and t0 = 0 otherwise).
+template <int G>
+__device__ __forceinline__ void virtual_unit(const DecodeArgs& a, int vu, int& unit, int& t0) {
+  unit = vu / a.npass;
+  t0 = a.chunk_t0 + (vu - unit * a.npass) * (G / a.gq);
 }
 
 template <int BITS>
@@ -139,14 +148,16 @@ __global__ void __launch_bounds__(128) decode_query_kernel(const DecodeArgs a) {
   __shared__ __align__(16) float qs[G][kHeadDim];
   __shared__ float red[24];
   griddep_launch();
-  const int unit = blockIdx.x, tid = threadIdx.x;
+  const int vu = blockIdx.x, tid = threadIdx.x;
+  int unit, t0;
+  virtual_unit<G>(a, vu, unit, t0);
   const int b = unit / a.Hkv, h = unit % a.Hkv;
   const float* Tcol = a.t_k_inv + (size_t)h * kHeadDim * kHeadDim + tid;
   float t[kHeadDim];
 #pragma unroll
   for (int i = 0; i < kHeadDim; ++i) t[i] = __ldg(Tcol + (size_t)i * kHeadDim);
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh) qs[hh][tid] = __half2float(a.q[head_row(a, b, h, hh) * kHeadDim + tid]);
+  for (int hh = 0; hh < G; ++hh) qs[hh][tid] = __half2float(a.q[head_row(a, b, h, t0, hh) * kHeadDim + tid]);
   if (a.prep.enabled) {  // raw queries (bulk-route step): RMSNorm + RoPE at position S - 1
     __syncthreads();
     const int qpos = max(a.state[2 * unit] - 1, 0);
@@ -159,10 +170,10 @@ __global__ void __launch_bounds__(128) decode_query_kernel(const DecodeArgs a) {
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
     qs[hh][tid] = acc[hh];
-    a.qprime[((size_t)unit * G + hh) * kHeadDim + tid] = acc[hh];
+    a.qprime[((size_t)vu * G + hh) * kHeadDim + tid] = acc[hh];
   }
   __syncthreads();
-  build_query_frags<BITS, G>(qs, tid, 128, red, a.scale_log2, a.qfrag + (size_t)unit * kQFragBytes,
+  build_query_frags<BITS, G>(qs, tid, 128, red, a.scale_log2, a.qfrag + (size_t)vu * kQFragBytes,
                              [] { __syncthreads(); });
 }
 
@@ -613,7 +624,8 @@ __device__ __forceinline__ void store_out4(const DecodeArgs& a, size_t o, float4
 }
 
 // Merge the `count` (<= kMaxSplits) cluster partials (m, l, pad, pad, o[128] per head,
-// base 2, o not yet normalised) of one unit and write the normalised output rows of its G
+// base 2, o not yet normalised) of one virtual unit (cache unit `unit`, chunk block at t0)
+// and write the normalised output rows of its G
 // query heads, summing the partials in their order.  wts: shared [count][G].  The warp of
 // head hh reduces the partials' (m, l) (lane i loads partials i, i + 32, ... at once); thread
 // (head, quad) then sums dimensions 4*quad .. 4*quad+3 of every partial's row, row_batch
@@ -625,7 +637,7 @@ __device__ __forceinline__ void store_out4(const DecodeArgs& a, size_t o, float4
 template <int G>
 __host__ __device__ constexpr int row_batch() { return 16; }
 template <int G>
-__device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, int count, float* wts) {
+__device__ void merge_partials(const DecodeArgs& a, int unit, int t0, const float* src, int count, float* wts) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int kQuads = kHeadDim / 4;
   constexpr int kRowBatch = row_batch<G>();
@@ -691,7 +703,7 @@ __device__ void merge_partials(const DecodeArgs& a, int unit, const float* src, 
         }
       }
     }
-    store_out4(a, head_row(a, b, h, hh) * kHeadDim + d, acc);
+    store_out4(a, head_row(a, b, h, t0, hh) * kHeadDim + d, acc);
   }
 }
 
@@ -723,11 +735,15 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   float* wts = reinterpret_cast<float*>(smem + SM::kPv + SM::kPart);  // [n_split][G] (the last merge only)
   __shared__ uint32_t s_last;
   __shared__ int s_abort;  // set by a bounded wait that gave up: every role leaves its loop
+  __shared__ int s_vu[3];  // vu, unit, t0 for the epilogue (kept out of the stream's registers)
   volatile int* abort = &s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t4 = lane & 3;
-  const int unit = blockIdx.y, item = blockIdx.x;
+  int vu = blockIdx.y;  // virtual unit: workspace index
+  const int item = blockIdx.x;
+  int unit, t0;         // its cache unit and chunk block
+  virtual_unit<G>(a, vu, unit, t0);
   const int nitems = a.n_split;
   const int ncta = a.cluster;  // CTAs per cluster (consecutive items of the unit)
   int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
@@ -778,6 +794,9 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
       mbar_init(&empty[s], kConsumers);
     }
     s_abort = 0;
+    s_vu[0] = vu;
+    s_vu[1] = unit;
+    s_vu[2] = t0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -836,13 +855,13 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     griddep_wait();  // q' and the query fragments come from the kernel before
     {  // the unit's query fragments into shared memory while the window share runs
       constexpr int n16 = GCfg<G>::FW * 8 + 4;
-      const uint8_t* src = a.qfrag + (size_t)unit * kQFragBytes;
+      const uint8_t* src = a.qfrag + (size_t)vu * kQFragBytes;
       for (int i = tid; i < n16; i += kConsumers * 32) cp_async16(qfs + 16 * i, src + 16 * i);
       cp_async_commit();
     }
-    const int qlim = a.chunk_n > 0 ? S - a.chunk_n + a.chunk_t0 : INT_MAX;
+    const int qlim = a.chunk_n > 0 ? S - a.chunk_n + t0 : INT_MAX;
     window_share<G>(a, unit, wbeg, wend, n_sink, r0, warp, lane, wr, mg, wpv, qlim,
-                    a.qprime + (size_t)unit * G * kHeadDim);
+                    a.qprime + (size_t)vu * G * kHeadDim);
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) qs.o[mt][0] = qs.o[mt][1] = qs.o[mt][2] = qs.o[mt][3] = 0.f;
     // (b) quantized positions
@@ -912,6 +931,9 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   // ======================= merge the 8 pseudo-warps into the CTA's state (m, l, o): the
   // weights once per (pseudo-warp, head), then the rows.  Rank 0 of a cluster keeps its
   // state (cpo, cpm); rank 1 stores its own straight into rank 0's receive buffer.
+  vu = s_vu[0];
+  unit = s_vu[1];
+  t0 = s_vu[2];
   const int rank = ncta > 1 ? (int)cluster_rank() : 0;
   const int ncl = nitems / ncta;  // clusters of the unit
   const uint32_t peer = ncta > 1 ? cluster_map(srecv, 0) : 0u;  // rank 0's receive buffer
@@ -986,7 +1008,7 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   }
   __syncthreads();
   const bool c_abort = mg->c_abort != 0;
-  float* part = a.partials + ((size_t)unit * ncl + item / ncta) * G * kPartStride;
+  float* part = a.partials + ((size_t)vu * ncl + item / ncta) * G * kPartStride;
   for (int q4 = tid; q4 < G * kHeadDim / 4; q4 += kThreads) {
     const int hh = (4 * q4) / kHeadDim, d = (4 * q4) % kHeadDim;
     const float e0 = mg->ce[0][hh], e1 = mg->ce[1][hh];
@@ -999,7 +1021,8 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
         const float L = mg->cL[hh];
         const float invL = L > 0.f ? 1.0f / L : 0.f;
         if (d == 0 && !(L > 0.f)) atomicOr(a.status, kStatusEmpty);
-        store_out4(a, head_row(a, b, h, hh) * kHeadDim + d, make_float4(O.x * invL, O.y * invL, O.z * invL, O.w * invL));
+        store_out4(a, head_row(a, b, h, t0, hh) * kHeadDim + d,
+                   make_float4(O.x * invL, O.y * invL, O.z * invL, O.w * invL));
       }
     } else {  // the cluster's partial, for the unit's last merge
       *reinterpret_cast<float4*>(part + hh * kPartStride + 4 + d) = O;
@@ -1023,19 +1046,19 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   __syncthreads();  // the partial is written; thread 0's acquire-release add publishes it
   if (tid == 0) {
     const uint32_t inc = mg->c_abort ? 0x10001u : 1u;
-    const uint32_t old = atomic_add_acq_rel(&a.tickets[unit], inc);
+    const uint32_t old = atomic_add_acq_rel(&a.tickets[vu], inc);
     s_last = ((old & 0xFFFFu) == (uint32_t)(ncl - 1)) ? (((old + inc) >> 16) != 0 ? 2u : 1u) : 0u;
   }
   __syncthreads();  // (and orders the other clusters' partials before this CTA's reads of them)
   if (!s_last) return;
   if (s_last == 1u) {
-    merge_partials<G>(a, unit, a.partials + (size_t)unit * ncl * G * kPartStride, ncl, wts);
+    merge_partials<G>(a, unit, t0, a.partials + (size_t)vu * ncl * G * kPartStride, ncl, wts);
     if (S_next >= 0 && tid == 0) {  // every item of the unit has read the old state
       a.state[2 * unit] = S_next;
       a.state[2 * unit + 1] = Sq_next;
     }
   }
-  if (tid == 0) a.tickets[unit] = 0u;
+  if (tid == 0) a.tickets[vu] = 0u;
 }
 
 // One launch of the main kernel, in clusters of d.cluster consecutive work items (no

@@ -36,7 +36,9 @@ struct Derived {
 };
 
 // Validates cfg and fills d; returns WUSHKV_OK / WUSHKV_EINVAL / WUSHKV_EUNSUPPORTED.
-int derive(const wushkv_config* cfg, Derived* d);
+// ticket_units: completion counters to reserve at the start of the workspace (-1: those
+// of cfg's own largest chunk-attention launch, which every layout of cfg reserves alike).
+int derive(const wushkv_config* cfg, Derived* d, long long ticket_units = -1);
 
 // The flush under length L of a (sequence, KV head) whose quantized region ends at Sq:
 // lo0 = max(Sq, S_sink); e = L - S_keep - lo0; e >= S_flush -> nf = floor(e / S_flush) *
@@ -99,10 +101,11 @@ struct DecodeArgs {
   void* out;
   int out_fp16;
   int units;
-  uint32_t* tickets;   // [units] completion counters of the last merge (zero between calls)
-  float* qprime;       // [units][G][128] fp32 (fused step: written by the append kernel)
-  uint8_t* qfrag;      // [units][kQFragBytes]: query fragments and constants (qfrag.cuh; fused step)
-  float* partials;     // [units][n_split / cluster][G][132]: the clusters' merged states
+  // workspace, per virtual unit (units * npass of them; see chunk attention below)
+  uint32_t* tickets;   // [vu] completion counters of the last merge (zero between calls)
+  float* qprime;       // [vu][G][128] fp32 (fused step: written by the append kernel)
+  uint8_t* qfrag;      // [vu][kQFragBytes]: query fragments and constants (qfrag.cuh; fused step)
+  float* partials;     // [vu][n_split / cluster][G][132]: the clusters' merged states
   int cluster;         // CTAs per cluster
   // fused step (wushkv_step's one-kernel append of n_new tokens runs just before): that
   // kernel leaves the state words alone, so this one reads the pre-append state, derives the
@@ -111,9 +114,13 @@ struct DecodeArgs {
   // the new state once every item of the unit has read the old one (the final merge).
   int fused, n_new;
   // chunk attention (wushkv_chunk_attn): the kernel's G query heads per unit are gq real
-  // heads of each of G / gq consecutive chunk tokens, chunk_t0 the first of them; q and out
-  // are [B][chunk_n][H_q][128]; chunk_n = 0 for a one-token decode (gq = G)
-  int chunk_n, chunk_t0, gq;
+  // heads of each of G / gq consecutive chunk tokens; q and out are [B][chunk_n][H_q][128];
+  // chunk_n = 0 for a one-token decode (gq = G).  One launch takes npass such blocks of
+  // tokens, starting at chunk token chunk_t0: its grid has a virtual unit vu = unit * npass
+  // + pass for each (cache unit, block), with the workspace (tickets, q', fragments,
+  // partials) indexed by vu and the cache by unit; block `pass` starts at chunk token
+  // chunk_t0 + pass * G / gq.  npass = 1 outside chunk attention.
+  int chunk_n, chunk_t0, gq, npass;
   PrepSpec prep;       // raw q (wushkv_step_prep, bulk route): the kernel normalises and rotates it
   // bounded waits: the cycle limit after which a wait gives up (STATUS_TIMEOUT), and a test
   // hook -- the producer never issues stage `withhold_tile` of any item (-1: off)

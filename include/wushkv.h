@@ -256,8 +256,12 @@ int wushkv_step(const wushkv_config* cfg, const wushkv_cache* cache, const void*
  * q:   device fp16 [B][n_q][H_q][128] (after head-norm and RoPE); out: [B][n_q][H_q][128],
  *      fp32 or fp16 (out_fp16); t_k_inv, softmax_scale as in wushkv_decode_attn.
  * workspace: layout.chunk_workspace_bytes, zero-filled once before its first use (as for
- *   wushkv_decode_attn; the same buffer may serve both).
- * The chunk's queries share passes over the cache in blocks of up to 8 / g tokens.
+ *   wushkv_decode_attn; one buffer of the larger size may serve both, and wushkv_step:
+ *   every layout of a configuration keeps its completion counters in the same leading
+ *   bytes, which every call leaves at zero).
+ * The chunk's queries take blocks of up to 8 / g tokens (their query heads share the
+ * kernel's per-position work); one launch pair runs up to 32 equal blocks side by side, as
+ * separate grid rows of each (sequence, KV head) that stream its cache at the same time.
  * Returns WUSHKV_OK, WUSHKV_EINVAL (also n_q < 1 or n_q > chunk_max), WUSHKV_EUNSUPPORTED
  * or WUSHKV_ECUDA. */
 int wushkv_chunk_attn(const wushkv_config* cfg, const wushkv_cache* cache, const void* q, int32_t n_q,

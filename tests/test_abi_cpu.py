@@ -186,3 +186,21 @@ def test_decode_split_policy(bnd):
         assert 1 <= L.n_splits <= 128 and L.decode_cluster == (2 if L.n_splits % 2 == 0 else 1)
         if B * Hkv * L.n_splits > slots:  # more than one wave only when one item per unit overfills it
             assert L.n_splits <= 4
+
+
+def test_workspace_counters_cover_every_chunk_launch(bnd):
+    """Every layout of a configuration reserves the same leading completion counters: one per
+    virtual unit of its largest chunk-attention launch (up to 32 blocks of chunk tokens per
+    (sequence, KV head), no more than chunk_max, and no more grid rows than 65535), so that
+    decode, step and chunk calls can share one workspace.  The decode layout grows by exactly
+    that reservation as chunk_max grows; the rest of it does not depend on chunk_max."""
+    def up(x):
+        return (x + 255) // 256 * 256
+    for B, Hkv, Hq in [(8, 8, 32), (2, 2, 8), (1, 1, 8), (600, 64, 64)]:
+        U = B * Hkv
+        base = bnd.pack_layout(bnd.make_config(B, Hkv, Hq, 2, 4096, 4, 32, 16, 1))
+        for cmax in (2, 8, 40):
+            L = bnd.pack_layout(bnd.make_config(B, Hkv, Hq, 2, 4096, 4, 32, 16, cmax))
+            mp = max(1, min(32, cmax, 65535 // U))
+            assert L.workspace_bytes - base.workspace_bytes == up(4 * U * mp) - up(4 * U), (B, Hkv, cmax)
+            assert L.chunk_workspace_bytes >= L.workspace_bytes

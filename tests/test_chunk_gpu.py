@@ -15,7 +15,20 @@ from tests import harness as H
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("bits,Hkv,Hq,chunk", [(2, 2, 8, 8), (2, 2, 2, 16), (4, 1, 8, 4), (2, 2, 4, 3)])
+def ticket_words(cfg, B, Hkv):
+    """The completion counters at the start of every workspace layout: one per virtual unit
+    of the largest chunk-attention launch (blocks of chunk tokens run as up to 32 grid rows
+    per (sequence, KV head))."""
+    units = B * Hkv
+    return units * max(1, min(32, cfg.chunk_max, 65535 // units))
+
+
+# chunk lengths cover one block per launch, several equal blocks in one launch (8 tokens at
+# g = 4: four blocks of two; 16 at g = 1: two blocks of eight; 4 at g = 8: four blocks of
+# one), ragged remainders taking further launches (7 at g = 4: three blocks of two, then
+# one token), and more blocks than one launch takes (40 at g = 8: 32 blocks, then 8)
+@pytest.mark.parametrize("bits,Hkv,Hq,chunk", [(2, 2, 8, 8), (2, 2, 2, 16), (4, 1, 8, 4), (2, 2, 4, 3),
+                                               (2, 1, 8, 40)])
 def test_chunk_attention_matches_oracle(bits, Hkv, Hq, chunk):
     B = 2
     cfg = bnd.make_config(B, Hkv, Hq, bits, 3000, 4, 32, 16, chunk)
@@ -39,11 +52,18 @@ def test_chunk_attention_matches_oracle(bits, Hkv, Hq, chunk):
         out = gc.chunk_attn(H.to_dev(q), tinv, scale)
         torch.cuda.synchronize()
         assert gc.status() == 0
+        # every counter is back at zero, for the next call of any kind on this workspace
+        nt = ticket_words(cfg, B, Hkv)
+        assert torch.count_nonzero(gc.workspace[:4 * nt]).item() == 0
         ref = oatt.chunk_decode(H.oracle_cache_from_gpu(gc), q, T, scale)
         H.assert_attention_close(out.cpu().numpy(), ref)
+        dec = gc.decode_attn(H.to_dev(q[:, -1]), tinv, scale)  # same workspace, other layout
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(gc.workspace[:4 * nt]).item() == 0
         if n == 1:
-            dec = gc.decode_attn(H.to_dev(q[:, 0]), tinv, scale)
             assert torch.equal(dec, out[:, 0])
+        else:  # the chunk's last token sees the whole cache, as a decode of its query does
+            H.assert_attention_close(dec.cpu().numpy(), ref[:, -1])
 
 
 def test_chunk_attention_rejects_oversized_chunk():
