@@ -121,48 +121,29 @@ __device__ void prepare_query(const AppendArgs& a, int unit, int tid) {
                              [] { bar_sync(2, 128); });
 }
 
-// Small append: one 128-thread CTA per (sequence, KV head).  G > 0: the fused step
-// (wushkv_step) also prepares the decode that follows (q' and its query fragments) in a
-// second CTA per unit (blockIdx.y = 1), in parallel with the append and
-// for every unit, including one whose append is refused (its cache is decoded as it
-// stands).  Each role synchronises on its own named barrier (1: append, 2: decode
-// preparation).
-template <int BITS, int NSEL, int G>
-__global__ void __launch_bounds__(128) append_small_kernel(const AppendArgs a) {
-  const int unit = blockIdx.x;
-  const int b = unit / a.Hkv, h = unit % a.Hkv;
-  if (G > 0) {
-    griddep_launch();  // the decode kernel may launch now; it waits for this whole grid
-    // the fused step leaves the state words to the decode kernel (defer_state), so the two
-    // roles need not order their reads of them
-    if (blockIdx.y == 1) {
-      prepare_query<BITS, (G > 0 ? G : 1)>(a, unit, threadIdx.x);
-      return;
+// Row r (= the thread) of k' = T_K k in fp32: its 256-byte row of T_K (tr, fp16) against the
+// key staged in shared memory, in four interleaved partial sums added at the end.
+__device__ __forceinline__ float key_row(const uint4 (&tr)[kHeadDim / 8], const float* ks) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < kHeadDim / 8; ++i) {
+    const uint32_t w[4] = {tr[i].x, tr[i].y, tr[i].z, tr[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 tf = __half22float2(u32_as_h2(w[e]));
+      acc[e] = fmaf(tf.x, ks[8 * i + 2 * e], acc[e]);
+      acc[e] = fmaf(tf.y, ks[8 * i + 2 * e + 1], acc[e]);
     }
-    // the unit's key transform into L2 while the state is read (the rows are loaded below)
-    if (threadIdx.x == 0 && a.transform == WUSHKV_TRANSFORM_DENSE)
-      bulk_prefetch_l2(a.t_k + (size_t)h * kHeadDim * kHeadDim, kHeadDim * kHeadDim * 2);
   }
-  const int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
-  const bool valid = state_ok(S, Sq, a);
-  const bool fits = valid && S + a.n_new <= a.cap;
-  if (!valid) {
-    if (threadIdx.x == 0) atomicOr(a.status, kStatusBadState);
-    return;
-  }
-  if (!fits) {
-    if (threadIdx.x == 0) atomicOr(a.status, kStatusOverflow);
-    return;
-  }
-  // 1. the flush that closes the previous chunk (entries still in the ring)
-  const FlushPlan fp = flush_plan(Sq, S, a);
-  quantize_ring_range<BITS, NSEL>(a, unit, fp.lo0, fp.lo0 + fp.nf, threadIdx.x, 128);
-  bar_sync(1, 128);  // ring slots are read above before new tokens may reuse them below
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
 
-  // 2. new tokens: k' = fp16_rn(T_K k) (fp32 accumulation), v as given.  Thread r owns
-  // output row r: its 256-byte row of T_K is loaded once (16 x 16 B in flight), the
-  // token's key is staged in shared memory as fp32.
-  __shared__ float ks[kHeadDim];
+// The small append's new tokens, one after another: k' = fp16_rn(T_K k) (fp32 accumulation;
+// or the Walsh-Hadamard transform), v as given, into the sink or the ring.  Thread r owns
+// output row r: its row of T_K is loaded once (16 x 16 B in flight); the token's key is
+// staged in shared memory (ks) as fp32, after RMSNorm + RoPE at its position when the step
+// takes raw keys.  All 128 threads of the CTA take part (named barrier 1).
+__device__ void append_tokens(const AppendArgs& a, int unit, int b, int h, int S, float* ks) {
   __shared__ float hs[kHeadDim];  // Hadamard butterflies across warps
   const int r = threadIdx.x;
   const bool hadamard = a.transform == WUSHKV_TRANSFORM_HADAMARD;
@@ -211,20 +192,85 @@ __global__ void __launch_bounds__(128) append_small_kernel(const AppendArgs a) {
       }
       kdst[r] = __float2half_rn(y * 0.08838834764831845f);
     } else {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four interleaved partial sums, added at the end
-#pragma unroll
-      for (int i = 0; i < kHeadDim / 8; ++i) {
-        const uint32_t w[4] = {tr[i].x, tr[i].y, tr[i].z, tr[i].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 tf = __half22float2(u32_as_h2(w[e]));
-          acc[e] = fmaf(tf.x, ks[8 * i + 2 * e], acc[e]);
-          acc[e] = fmaf(tf.y, ks[8 * i + 2 * e + 1], acc[e]);
-        }
-      }
-      kdst[r] = __float2half_rn((acc[0] + acc[1]) + (acc[2] + acc[3]));
+      kdst[r] = __float2half_rn(key_row(tr, ks));
     }
     bar_sync(1, 128);  // ks is rewritten by the next token
+  }
+}
+
+// Small append: one 128-thread CTA per (sequence, KV head).  G > 0: the fused step
+// (wushkv_step) also prepares the decode that follows (q' and its query fragments) in a
+// second CTA per unit (blockIdx.y = 1), in parallel with the append and
+// for every unit, including one whose append is refused (its cache is decoded as it
+// stands).  Each role synchronises on its own named barrier (1: append, 2: decode
+// preparation).
+template <int BITS, int NSEL, int G>
+__global__ void __launch_bounds__(128) append_small_kernel(const AppendArgs a) {
+  const int unit = blockIdx.x;
+  const int b = unit / a.Hkv, h = unit % a.Hkv;
+  if (G > 0) {
+    griddep_launch();  // the decode kernel may launch now; it waits for this whole grid
+    // the fused step leaves the state words to the decode kernel (defer_state), so the two
+    // roles need not order their reads of them
+    if (blockIdx.y == 1) {
+      prepare_query<BITS, (G > 0 ? G : 1)>(a, unit, threadIdx.x);
+      return;
+    }
+  }
+  __shared__ float ks[kHeadDim];  // the token's key (fp32), for the transform
+  const int r = threadIdx.x;
+  // One post-RoPE token under a dense transform (a decode step): k' = T_K k needs nothing
+  // from the state, so it is formed first -- thread r loads its row of T_K and the token --
+  // and the state read, the flush and the stores follow.  Same arithmetic as the general
+  // path below.
+  const bool early = a.n_new == 1 && !a.prep.enabled && a.transform == WUSHKV_TRANSFORM_DENSE;
+  float k_early = 0.f;
+  uint4 v_early = make_uint4(0u, 0u, 0u, 0u);
+  if (early) {
+    const size_t src = ((size_t)b * a.Hkv + h) * kHeadDim;
+    uint4 tr[kHeadDim / 8];
+    const uint4* Trow = reinterpret_cast<const uint4*>(a.t_k + ((size_t)h * kHeadDim + r) * kHeadDim);
+#pragma unroll
+    for (int i = 0; i < kHeadDim / 8; ++i) tr[i] = Trow[i];
+    ks[r] = __half2float(a.k_new[src + r]);
+    if (r < kHeadDim / 8) v_early = reinterpret_cast<const uint4*>(a.v_new + src)[r];
+    bar_sync(1, 128);
+    k_early = key_row(tr, ks);
+  } else if (G > 0 && threadIdx.x == 0 && a.transform == WUSHKV_TRANSFORM_DENSE) {
+    // the unit's key transform into L2 while the state is read (the rows are loaded below)
+    bulk_prefetch_l2(a.t_k + (size_t)h * kHeadDim * kHeadDim, kHeadDim * kHeadDim * 2);
+  }
+  const int S = a.state[2 * unit], Sq = a.state[2 * unit + 1];
+  const bool valid = state_ok(S, Sq, a);
+  const bool fits = valid && S + a.n_new <= a.cap;
+  if (!valid) {
+    if (threadIdx.x == 0) atomicOr(a.status, kStatusBadState);
+    return;
+  }
+  if (!fits) {
+    if (threadIdx.x == 0) atomicOr(a.status, kStatusOverflow);
+    return;
+  }
+  // 1. the flush that closes the previous chunk (entries still in the ring)
+  const FlushPlan fp = flush_plan(Sq, S, a);
+  quantize_ring_range<BITS, NSEL>(a, unit, fp.lo0, fp.lo0 + fp.nf, threadIdx.x, 128);
+  bar_sync(1, 128);  // ring slots are read above before new tokens may reuse them below
+
+  // 2. the new tokens
+  if (early) {  // the one formed above
+    __half* kdst;
+    __half* vdst;
+    if (S < a.s_sink) {
+      kdst = a.k_sink + ((size_t)unit * a.sink_dim + S) * kHeadDim;
+      vdst = a.v_sink + ((size_t)unit * a.sink_dim + S) * kHeadDim;
+    } else {
+      kdst = a.k_ring + ((size_t)unit * a.R + S % a.R) * kHeadDim;
+      vdst = a.v_ring + ((size_t)unit * a.R + S % a.R) * kHeadDim;
+    }
+    kdst[r] = __float2half_rn(k_early);
+    if (r < kHeadDim / 8) reinterpret_cast<uint4*>(vdst)[r] = v_early;
+  } else {
+    append_tokens(a, unit, b, h, S, ks);
   }
   // 3. state (a fused step's decode kernel writes it instead, once it has read the old one)
   if (threadIdx.x == 0 && !a.defer_state) {
