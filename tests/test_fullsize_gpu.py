@@ -124,3 +124,37 @@ def test_full_size_workload_sampled_units(name):
         ref = oatt.decode(gu, q[b:b + 1, h * g:(h + 1) * g].cpu().numpy(), Tn[h:h + 1],
                           synth.default_softmax_scale(wl.head_dim))[0]
         H.assert_attention_close(out[b, h * g:(h + 1) * g].cpu().numpy(), ref)
+
+
+def test_full_size_chunk_attention_sampled_units():
+    """Chunked prefill at the Llama-3-8B layer's full size, in the launch configuration the
+    benchmark times: an 8-token chunk appended (decode-time path) onto 32,760 cached
+    positions, its 8 queries attending causally in one launch pair (4 blocks of 2 tokens side
+    by side).  Each sampled unit's 8 x 4 query rows are checked against the oracle's causal
+    chunk attention over the GPU's own cache of that unit."""
+    wl = synth.WORKLOADS["llama3-8b-layer"]
+    n = 8
+    dev = torch.device("cuda")
+    cfg = bnd.config_for_workload(wl, extra_capacity=64, chunk_max=n)
+    T = synth.key_transforms(wl, 0)
+    tk, tinv = T.to(dev), bnd.compensation(T).to(dev)
+    gc = bnd.KVCache(cfg, device=dev)
+    base = wl.context - n
+    for s0 in range(0, base, 4096):
+        m = min(4096, base - s0)
+        gc.append(synth.bulk_tokens(wl, 0, s0, m, device=dev, which="k"),
+                  synth.bulk_tokens(wl, 0, s0, m, device=dev, which="v"), tk)
+    gc.append(synth.bulk_tokens(wl, 0, base, n, device=dev, which="k"),
+              synth.bulk_tokens(wl, 0, base, n, device=dev, which="v"), tk)
+    q = torch.stack([synth.bulk_queries(wl, 0, base + t, device=dev) for t in range(n)], dim=1).contiguous()
+    scale = synth.default_softmax_scale(wl.head_dim)
+    out = gc.chunk_attn(q, tinv, scale)
+    torch.cuda.synchronize()
+    assert gc.status() == 0
+    assert (gc.lengths()[0] == wl.context).all()
+    Tn = T.numpy()
+    g = wl.group
+    for b, h in _samples(wl):
+        gu = _unit_cache_from_gpu(gc, b, h, Tn[h])
+        ref = oatt.chunk_decode(gu, q[b:b + 1, :, h * g:(h + 1) * g].cpu().numpy(), Tn[h:h + 1], scale)[0]
+        H.assert_attention_close(out[b, :, h * g:(h + 1) * g].cpu().numpy(), ref)
