@@ -48,7 +48,8 @@ class Layout(ctypes.Structure):
                 ("state_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t),
                 ("cap_alloc", ctypes.c_int32), ("ring_slots", ctypes.c_int32), ("code_bytes", ctypes.c_int32),
                 ("n_splits", ctypes.c_int32), ("split_tokens", ctypes.c_int32), ("code_order", ctypes.c_int32),
-                ("chunk_workspace_bytes", ctypes.c_size_t), ("decode_cluster", ctypes.c_int32)]
+                ("chunk_workspace_bytes", ctypes.c_size_t), ("decode_cluster", ctypes.c_int32),
+                ("decode_interleave", ctypes.c_int32)]
 
 
 class CacheBufs(ctypes.Structure):

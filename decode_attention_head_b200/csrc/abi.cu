@@ -89,6 +89,9 @@ int derive(const wushkv_config* cfg, Derived* d, long long ticket_units) {
     }
     d->n_split = best;
     d->cluster = best % 2 == 0 ? 2 : 1;
+    // a unit whose items fill a quarter of a round of CTAs or more (one sequence at long
+    // context) would otherwise sit in the rounds an SM receives last, which run slowest
+    d->interleave = best * 4 >= kB200SMs ? 1 : 0;
     const int tiles = ceil_div(d->cap_alloc, kTileTokens);
     d->split_tokens = ceil_div(tiles, d->n_split) * kTileTokens;
   }
@@ -200,6 +203,7 @@ extern "C" int wushkv_pack_layout(const wushkv_config* cfg, wushkv_layout* out) 
   out->split_tokens = d.split_tokens;
   out->code_order = WUSHKV_CODE_ORDER_VGROUP16;
   out->decode_cluster = d.cluster;
+  out->decode_interleave = d.interleave;
   return WUSHKV_OK;
 }
 
@@ -319,6 +323,7 @@ static void fill_decode(const wushkv_config* cfg, const Derived& d, const wushkv
   a->qfrag = ws + d.ws_qfrag;
   a->partials = reinterpret_cast<float*>(ws + d.ws_partials);
   a->cluster = d.cluster;
+  a->interleave = d.interleave;
   a->units = d.units;
   a->fused = 0;
   a->n_new = 0;

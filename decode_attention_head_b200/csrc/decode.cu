@@ -12,7 +12,10 @@
 //     derives the post-append state itself, streams the tiles the append cannot touch at
 //     once and waits for the append before reading anything else -- see DecodeArgs::fused.)
 //  2. decode_main: grid (n_split, units) in clusters of C (1 or 2) consecutive work items of
-//     a unit.  Work item s of a unit takes the s-th share of the unit's current quantized
+//     a unit (with many items per unit the grid's clusters interleave the units instead, in
+//     linear order, so that every unit has items in every round of CTAs an SM receives: the
+//     rounds dispatched last run slowest, and a unit confined to them finished last).  Work
+//     item s of a unit takes the s-th share of the unit's current quantized
 //     region [S_sink, S_quant) (whole 128-position stages) and of its fp16 window positions
 //     (sink [0, S_sink) and recent [S_quant, S)).
 //   * Stream: the quantized positions pass through shared memory in 128-position stages
@@ -735,13 +738,21 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   float* wts = reinterpret_cast<float*>(smem + SM::kPv + SM::kPart);  // [n_split][G] (the last merge only)
   __shared__ uint32_t s_last;
   __shared__ int s_abort;  // set by a bounded wait that gave up: every role leaves its loop
-  __shared__ int s_vu[3];  // vu, unit, t0 for the epilogue (kept out of the stream's registers)
+  __shared__ int s_vu[4];  // vu, unit, t0, item for the epilogue (kept out of the stream's registers)
   volatile int* abort = &s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t4 = lane & 3;
-  int vu = blockIdx.y;  // virtual unit: workspace index
-  const int item = blockIdx.x;
+  // virtual unit (workspace index) and work item of this CTA
+  int vu, item;  // (both re-read from shared memory for the epilogue)
+  if (a.interleave) {
+    const int lin = blockIdx.y * gridDim.x + blockIdx.x, cl = lin / a.cluster;
+    vu = cl % gridDim.y;
+    item = (cl / gridDim.y) * a.cluster + lin % a.cluster;
+  } else {
+    vu = blockIdx.y;
+    item = blockIdx.x;
+  }
   int unit, t0;         // its cache unit and chunk block
   virtual_unit<G>(a, vu, unit, t0);
   const int nitems = a.n_split;
@@ -797,6 +808,7 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
     s_vu[0] = vu;
     s_vu[1] = unit;
     s_vu[2] = t0;
+    s_vu[3] = item;
     fence_mbar_init();
   }
   __syncthreads();
@@ -934,6 +946,7 @@ __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(G)) decode_main_k
   vu = s_vu[0];
   unit = s_vu[1];
   t0 = s_vu[2];
+  item = s_vu[3];
   const int rank = ncta > 1 ? (int)cluster_rank() : 0;
   const int ncl = nitems / ncta;  // clusters of the unit
   const uint32_t peer = ncta > 1 ? cluster_map(srecv, 0) : 0u;  // rank 0's receive buffer

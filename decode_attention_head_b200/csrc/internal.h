@@ -29,6 +29,7 @@ struct Derived {
   float f_lo, f_hi;
   int n_split, split_tokens;
   int cluster;      // decode CTAs per thread-block cluster (consecutive items of a unit; divides n_split)
+  int interleave;   // 1: the decode grid's consecutive clusters belong to different units
   // workspace offsets (bytes)
   size_t ws_tickets, ws_qprime, ws_qfrag, ws_partials, ws_total;
   // cache buffer sizes (bytes)
@@ -107,6 +108,10 @@ struct DecodeArgs {
   uint8_t* qfrag;      // [vu][kQFragBytes]: query fragments and constants (qfrag.cuh; fused step)
   float* partials;     // [vu][n_split / cluster][G][132]: the clusters' merged states
   int cluster;         // CTAs per cluster
+  // 1: cluster c of the grid (in linear order) is cluster c / U of unit c % U (U = gridDim.y),
+  // so that every unit has work items in every round of CTAs an SM receives; 0: grid row =
+  // unit, column = item
+  int interleave;
   // fused step (wushkv_step's one-kernel append of n_new tokens runs just before): that
   // kernel leaves the state words alone, so this one reads the pre-append state, derives the
   // post-append (S, S_quant) from it, streams the tiles below the old S_quant before the

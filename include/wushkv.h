@@ -128,6 +128,7 @@ typedef struct wushkv_layout {
   int32_t code_order;     /* how the packed codes are ordered (WUSHKV_CODE_ORDER_*) */
   size_t chunk_workspace_bytes; /* wushkv_chunk_attn scratch (zero-fill it once before its first use) */
   int32_t decode_cluster; /* decode CTAs per thread-block cluster (1 or 2; divides n_splits) */
+  int32_t decode_interleave; /* 1: the decode grid interleaves the units (n_splits >= 37) */
 } wushkv_layout;
 
 /* Device pointers of one layer's cache.

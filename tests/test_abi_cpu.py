@@ -180,6 +180,10 @@ def test_decode_split_policy(bnd):
     for name, wl in synth.WORKLOADS.items():
         L = bnd.pack_layout(bnd.config_for_workload(wl, extra_capacity=64))
         assert (L.n_splits, L.decode_cluster) == expect[name], name
+        # the grid interleaves the units where a unit's items fill a quarter of a round of
+        # CTAs (148 SMs): here the Qwen3-8B layer's one sequence and the tiny parity case
+        assert L.decode_interleave == (1 if L.n_splits * 4 >= 148 else 0), name
+        assert L.decode_interleave == (name in ("qwen3-8b-layer", "tiny")), name
     for B, Hkv, Hq in [(1, 1, 1), (1, 8, 64), (3, 8, 32), (16, 8, 32), (64, 32, 32), (256, 8, 8)]:
         L = bnd.pack_layout(bnd.make_config(B, Hkv, Hq, 2, 4096, 4, 32, 16, 1))
         slots = 148 * (3 if Hq // Hkv == 8 else 4)
