@@ -54,6 +54,8 @@ def parse_args():
                    help="only the prefill workload's bulk append + decode measurement (one JSON line)")
     p.add_argument("--decode-only", action="store_true",
                    help="only the graph-timed decode calls of the 128K and MHA workloads (one JSON line each)")
+    p.add_argument("--decode-workload", default=None,
+                   help="with --decode-only: only this one of the decode workloads")
     p.add_argument("--chunk-only", action="store_true",
                    help="only the chunked-prefill measurement on the Llama-3-8B layer (one JSON line)")
     return p.parse_args()
@@ -974,7 +976,8 @@ def main():
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
         for name, layers in DECODE_WORKLOADS:
-            print(json.dumps(measure_decode(bnd, synth, dev, name, layers)), flush=True)
+            if args.decode_workload in (None, name):
+                print(json.dumps(measure_decode(bnd, synth, dev, name, layers)), flush=True)
         return 0
     if args.chunk_only:
         from decode_attention_head_b200 import binding as bnd
